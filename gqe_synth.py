@@ -1,0 +1,153 @@
+"""Seeded synthetic inputs for the GQE attention forward pass.
+
+This module is the one thing the CUDA path and the CPU oracle share: it draws
+input tensors and nothing else (no routing, no attention, no reductions).
+
+Workloads (sizes, distributions and skews of the GQE prefill/decode cases):
+
+  tiny_f32      B=1  T=128  d_model=256  h=8  g=2 d_h=32  k=1  fp32,
+                W_r std 0.02
+  dense_gqa     B=4  T=2048 d_model=4096 h=32 g=8 d_h=128 k=4  bf16,
+                W_r std 1/64 (every head of every group selected: dense GQA
+                up to the gates)
+  gqe_prefill   B=8  T=4096 d_model=4096 h=32 g=8 d_h=128 k=2  bf16,
+                W_r std 1/64 (near-uniform head loads)
+  gqe_long      B=2  T=8192 d_model=2048 h=16 g=8 d_h=128 k=1  bf16,
+                W_r std 1/sqrt(2048), +1.0 logit bias on head 0 of each group
+                (skewed per-head token counts, about 76 % / 24 %)
+  gqe_decode    B=64 one query token, cache lengths uniform in [1024, 16384],
+                Lmax=16384, h=32 g=8 d_h=128 d_model=4096 k=2 bf16,
+                W_r std 1/64, caches [B, Lmax, g, d_h]
+
+Recipe: one CPU ``torch.Generator`` seeded with the workload's seed draws, in
+this order, lengths (decode only), x, W_r, Q, K, V as fp32 standard normals
+(W_r scaled by its std), then rounds bf16 workloads to bf16.  Decode caches are
+drawn per sequence for rows 0 .. L_b-1 only; rows at or beyond L_b are zero and
+are never read by the method.  The same values feed the GPU and the oracle.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    T: int
+    d_model: int
+    h: int
+    g: int
+    d_h: int
+    k: int
+    dtype: str  # "f32" | "bf16"
+    wr_std: float
+    head0_bias: float = 0.0  # added to the logit of head 0 of every group
+    decode: bool = False
+    Lmin: int = 0
+    Lmax: int = 0
+    seed: int = 0
+
+    @property
+    def hpg(self) -> int:
+        return self.h // self.g
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def describe(self) -> str:
+        s = (f"B={self.B} T={self.T} d_model={self.d_model} h={self.h} g={self.g} "
+             f"d_h={self.d_h} k={self.k} {self.dtype}")
+        if self.decode:
+            s = (f"decode B={self.B} L~U[{self.Lmin},{self.Lmax}] d_model={self.d_model} "
+                 f"h={self.h} g={self.g} d_h={self.d_h} k={self.k} {self.dtype}")
+        return s
+
+
+WORKLOADS = {
+    "tiny_f32": Workload("tiny_f32", 1, 128, 256, 8, 2, 32, 1, "f32", 0.02, seed=0),
+    "dense_gqa": Workload("dense_gqa", 4, 2048, 4096, 32, 8, 128, 4, "bf16", 1.0 / 64, seed=1),
+    "gqe_prefill": Workload("gqe_prefill", 8, 4096, 4096, 32, 8, 128, 2, "bf16", 1.0 / 64, seed=2),
+    "gqe_long": Workload("gqe_long", 2, 8192, 2048, 16, 8, 128, 1, "bf16", 1.0 / math.sqrt(2048),
+                         head0_bias=1.0, seed=3),
+    "gqe_decode": Workload("gqe_decode", 64, 1, 4096, 32, 8, 128, 2, "bf16", 1.0 / 64, decode=True,
+                           Lmin=1024, Lmax=16384, seed=4),
+}
+
+
+def custom(name="custom", *, B, T, d_model, h, g, d_h, k, dtype="bf16", wr_std=None,
+           head0_bias=0.0, decode=False, Lmin=0, Lmax=0, seed=0) -> Workload:
+    """A workload of any shape, with the same recipe (for parity tests)."""
+    if wr_std is None:
+        wr_std = 1.0 / math.sqrt(d_model)
+    return Workload(name, B, T, d_model, h, g, d_h, k, dtype, wr_std, head0_bias, decode,
+                    Lmin, Lmax, seed)
+
+
+def _normal(shape, gen, std=1.0, chunk=1 << 25):
+    """fp32 normals drawn in fixed-size chunks (deterministic for a given shape)."""
+    n = math.prod(shape)
+    out = torch.empty(n, dtype=torch.float32)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        out[s:e] = torch.randn(e - s, generator=gen)
+    if std != 1.0:
+        out.mul_(std)
+    return out.view(*shape)
+
+
+def bias_vector(w: Workload):
+    """Per-head logit bias of the workload, or None (float32 [h])."""
+    if w.head0_bias == 0.0:
+        return None
+    b = torch.zeros(w.h, dtype=torch.float32)
+    b[:: w.hpg] = w.head0_bias
+    return b
+
+
+def make_inputs(w: Workload):
+    """Draw the workload's inputs on the CPU.  Returns a dict of CPU tensors.
+
+    prefill: x [B,T,d_model], W_r [d_model,h], Q [B,T,h,d_h], K/V [B,T,g,d_h], bias
+    decode:  lengths [B] int32, x [B,1,d_model], W_r, q [B,1,h,d_h],
+             K_cache/V_cache [B,Lmax,g,d_h], bias
+    """
+    gen = torch.Generator().manual_seed(w.seed)
+    dt = w.torch_dtype
+    out = {}
+    if w.decode:
+        lengths = torch.randint(w.Lmin, w.Lmax + 1, (w.B,), generator=gen, dtype=torch.int64)
+        out["lengths"] = lengths.to(torch.int32)
+        out["x"] = _normal((w.B, 1, w.d_model), gen).to(dt)
+        out["W_r"] = _normal((w.d_model, w.h), gen, w.wr_std).to(dt)
+        out["q"] = _normal((w.B, 1, w.h, w.d_h), gen).to(dt)
+        for name in ("K_cache", "V_cache"):
+            cache = torch.zeros((w.B, w.Lmax, w.g, w.d_h), dtype=dt)
+            for b in range(w.B):
+                L = int(lengths[b])
+                cache[b, :L] = _normal((L, w.g, w.d_h), gen).to(dt)
+            out[name] = cache
+    else:
+        out["x"] = _normal((w.B, w.T, w.d_model), gen).to(dt)
+        out["W_r"] = _normal((w.d_model, w.h), gen, w.wr_std).to(dt)
+        out["Q"] = _normal((w.B, w.T, w.h, w.d_h), gen).to(dt)
+        out["K"] = _normal((w.B, w.T, w.g, w.d_h), gen).to(dt)
+        out["V"] = _normal((w.B, w.T, w.g, w.d_h), gen).to(dt)
+    out["bias"] = bias_vector(w)
+    return out
+
+
+def sample_rows(w: Workload, n: int, seed: int = 1234):
+    """A seeded sample of n flattened token rows (b*T + t) that always includes
+    the last position of every sequence and the first position of batch 0."""
+    gen = torch.Generator().manual_seed(seed)
+    total = w.B * w.T
+    n = min(n, total)
+    must = {0} | {b * w.T + w.T - 1 for b in range(w.B)}
+    picks = torch.randperm(total, generator=gen)[: max(0, n - len(must))].tolist()
+    rows = sorted(must | set(picks))
+    return torch.tensor(rows, dtype=torch.int64)

@@ -1,0 +1,216 @@
+"""CPU oracle for the GQE attention forward pass -- test infrastructure only.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` use this package.  The product library (``routed_head_gqa_b200``)
+never imports it, and it never imports the product library.
+
+The arithmetic lives in ``gqe_oracle.c`` (plain C, double accumulation).  This
+module only compiles it and marshals numpy arrays.  bf16 inputs are passed as
+their raw 16-bit patterns (``uint16`` arrays); fp32 inputs as ``float32``.
+
+Sources, per function (the same citations are in ``gqe_oracle.c``):
+  route    -- "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention"
+              (gist.science), "Architecture et Routage": top-k query-head
+              experts per GQA group, renormalised router probabilities.
+  compact  -- the per-(batch, head) packed position lists that the routed
+              kernels consume (bookkeeping of the selection made by ``route``).
+  attn_rows, decode -- IBM "Que es la atencion de consultas agrupadas"
+              (scaled dot-product attention, 1/sqrt(d_k)), ml-canon "56 GQA /
+              MQA" (KV head expansion), freenetmedia.pl "Grouped-Query
+              Attention" (contiguous head -> group mapping).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "gqe_oracle.c")
+LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+
+def compile_source(src: str, out: str, strict: bool = True) -> str:
+    """Compile an oracle C source file into a shared library (gcc, OpenMP).
+    ``strict`` turns warnings into errors."""
+    tmp = out + f".tmp{os.getpid()}"
+    flags = ["-Wall", "-Werror"] if strict else []
+    subprocess.check_call(["gcc", "-O2", *flags, "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile gqe_oracle.c into liboracle.so next to it (if stale)."""
+    if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(SOURCE):
+        compile_source(SOURCE, LIB_PATH)
+    return LIB_PATH
+
+
+def _as_input(a):
+    """Return (contiguous numpy array, dtype code) for an fp32 or bf16 input.
+
+    Accepts numpy float32 / uint16 arrays or CPU torch tensors (float32 or
+    bfloat16); bf16 is handed over as its raw bit pattern."""
+    if hasattr(a, "detach"):  # torch tensor
+        import torch
+
+        t = a.detach().cpu().contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16), BF16
+        if t.dtype == torch.float32:
+            return t.numpy(), F32
+        raise TypeError(f"oracle input dtype {t.dtype} not supported")
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError(f"oracle input dtype {a.dtype} not supported")
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _threads(n):
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+class Oracle:
+    """The oracle functions bound to one compiled library."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int, ctypes.c_int64
+        lib.oracle_route.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P]
+        lib.oracle_compact.argtypes = [i32, i32, i32, i32, i32, P, P, P]
+        lib.oracle_attn_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, i32]
+        lib.oracle_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32]
+        for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode):
+            f.restype = ctypes.c_int
+        self.lib = lib
+        self.path = lib_path
+
+    def route(self, x, W_r, h: int, g: int, k: int, bias=None):
+        """Router: returns (idx int32 [..., g, k], gate float64 [..., g, k],
+        logits float32 [..., h], margin float64 [..., g]) for x [..., d_model]."""
+        xa, dt = _as_input(x)
+        wa, dt2 = _as_input(W_r)
+        if dt != dt2:
+            raise TypeError("x and W_r must share a dtype")
+        lead = xa.shape[:-1]
+        d_model = xa.shape[-1]
+        if wa.shape != (d_model, h):
+            raise ValueError(f"W_r must be [{d_model}, {h}]")
+        BT = int(np.prod(lead)) if lead else 1
+        ba = None
+        if bias is not None:
+            ba = np.ascontiguousarray(np.asarray(bias, dtype=np.float32).reshape(h))
+        logits = np.empty(lead + (h,), np.float32)
+        idx = np.empty(lead + (g, k), np.int32)
+        gate = np.empty(lead + (g, k), np.float64)
+        margin = np.empty(lead + (g,), np.float64)
+        rc = self.lib.oracle_route(BT, d_model, h, g, k, dt, _ptr(xa), _ptr(wa), _ptr(ba),
+                                   _ptr(logits), _ptr(idx), _ptr(gate), _ptr(margin))
+        if rc:
+            raise ValueError(f"oracle_route failed ({rc})")
+        return idx, gate, logits, margin
+
+    def compact(self, idx, h: int, g: int, k: int):
+        """Per-(batch, head) ascending position lists:
+        (head_offsets int32 [B*h+1], head_pos int32 [B*T*g*k]) for idx [B, T, g, k]."""
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        B, T = ia.shape[0], ia.shape[1]
+        offs = np.empty(B * h + 1, np.int32)
+        pos = np.empty(B * T * g * k, np.int32)
+        rc = self.lib.oracle_compact(B, T, h, g, k, _ptr(ia), _ptr(offs), _ptr(pos))
+        if rc:
+            raise ValueError(f"oracle_compact failed ({rc})")
+        return offs, pos
+
+    def attn_rows(self, Q, K, V, idx, gate, rows=None, n_threads=None):
+        """GQE output rows O[b, t, :, :] (float64 [n_rows, h, d_h]) for the
+        flattened token indices ``rows`` (b*T + t); all rows when None."""
+        qa, dt = _as_input(Q)
+        ka, dk = _as_input(K)
+        va, dv = _as_input(V)
+        if not (dt == dk == dv):
+            raise TypeError("Q, K, V must share a dtype")
+        B, T, h, d_h = qa.shape
+        g = ka.shape[2]
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        ga = np.ascontiguousarray(gate, dtype=np.float64)
+        k = ia.shape[-1]
+        if rows is None:
+            rows = np.arange(B * T, dtype=np.int64)
+        ra = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+        out = np.empty((ra.shape[0], h, d_h), np.float64)
+        rc = self.lib.oracle_attn_rows(B, T, h, g, d_h, k, dt, _ptr(qa), _ptr(ka), _ptr(va),
+                                       _ptr(ia), _ptr(ga), ra.shape[0], _ptr(ra), _ptr(out),
+                                       _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_attn_rows failed ({rc})")
+        return out
+
+    def attn(self, Q, K, V, idx, gate, n_threads=None):
+        """Full GQE output O [B, T, h, d_h] (float64)."""
+        B, T, h, d_h = tuple(Q.shape)
+        return self.attn_rows(Q, K, V, idx, gate, None, n_threads).reshape(B, T, h, d_h)
+
+    def decode(self, q, K_cache, V_cache, lengths, idx, gate, n_threads=None):
+        """GQE decode output O [B, h, d_h] (float64) for q [B, h, d_h] (or
+        [B,1,h,d_h]), caches [B, Lmax, g, d_h], lengths [B], idx/gate [B, g, k]."""
+        qa, dt = _as_input(q)
+        ka, dk = _as_input(K_cache)
+        va, dv = _as_input(V_cache)
+        if not (dt == dk == dv):
+            raise TypeError("q and the caches must share a dtype")
+        B, Lmax, g, d_h = ka.shape
+        h = qa.shape[-2]
+        ia = np.ascontiguousarray(idx, dtype=np.int32).reshape(B, g, -1)
+        ga = np.ascontiguousarray(gate, dtype=np.float64).reshape(B, g, -1)
+        k = ia.shape[-1]
+        la = np.ascontiguousarray(np.asarray(lengths), dtype=np.int32).reshape(B)
+        out = np.empty((B, h, d_h), np.float64)
+        rc = self.lib.oracle_decode(B, Lmax, h, g, d_h, k, dt, _ptr(qa), _ptr(ka), _ptr(va),
+                                    _ptr(la), _ptr(ia), _ptr(ga), _ptr(out), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_decode failed ({rc})")
+        return out
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def route(*a, **kw):
+    return default().route(*a, **kw)
+
+
+def compact(*a, **kw):
+    return default().compact(*a, **kw)
+
+
+def attn_rows(*a, **kw):
+    return default().attn_rows(*a, **kw)
+
+
+def attn(*a, **kw):
+    return default().attn(*a, **kw)
+
+
+def decode(*a, **kw):
+    return default().decode(*a, **kw)

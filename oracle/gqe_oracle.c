@@ -1,0 +1,277 @@
+/*
+ * gqe_oracle.c -- CPU oracle for the forward pass of a Grouped Query Experts
+ * (GQE) attention layer.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check
+ * and the CPU-baseline leg of the benchmark are the only callers.  Nothing in
+ * the product library links or loads this file, and this file uses nothing from
+ * the product library.
+ *
+ * Plain, slow and direct: every floating-point sum is accumulated in double,
+ * one element at a time, in index order.  Inputs are fp32 or bf16 (bf16 is
+ * widened exactly to float, then to double).
+ *
+ * What it computes, with its sources:
+ *  - Router.  "Grouped Query Experts: Mixture-of-Experts on GQA
+ *    Self-Attention" (gist.science summary, section "Architecture et
+ *    Routage"): for each token a router picks a sparse subset of k query-head
+ *    experts in every GQA group, and the K/V path stays dense.  The page gives
+ *    no router formula; the reading used here is a linear router
+ *    l = x . W_r (+ an optional per-head bias), its logits rounded to fp32,
+ *    top-k per group on those fp32 logits with equal logits going to the
+ *    lower head index.
+ *  - Gates.  Same page, "Somme Ponderee Renormalisee": the router
+ *    probabilities are renormalised over the selected experts:
+ *    gate_j = exp(l_j - m) / sum_{i in S} exp(l_i - m), m = max_{i in S} l_i.
+ *  - Head -> group mapping.  "Grouped-Query Attention" (freenetmedia.pl),
+ *    section "Jak dzialaja...": with 8 query heads and 2 groups the first 4
+ *    heads share KV head 0 and the next 4 share KV head 1, i.e. head j uses
+ *    KV head j / (h/g).  The ml-canon page "56 GQA / MQA", section "PyTorch
+ *    GQA", expands KV heads the same way (repeat each KV head h/g times).
+ *  - Attention.  IBM "Que es la atencion de consultas agrupadas": scores are
+ *    q . k scaled by 1/sqrt(d_k), normalised by a softmax, and used to weight
+ *    the value vectors.  Causal: key s is visible to query t iff s <= t (the
+ *    pages' autoregressive setting; the positions are the original ones).
+ *  - Output.  Each selected head's attention output is multiplied by its gate
+ *    and written to that head's slot; every unselected head's slot is zero.
+ *  - Decode.  One new query per sequence at position L_b - 1 against a cache
+ *    holding keys 0 .. L_b - 1 of that sequence (the KV cache of the GQA
+ *    pages, which stays dense under GQE).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+static double load_elem(const void* p, size_t i, int dtype) {
+    if (dtype == ORACLE_F32) return (double)((const float*)p)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t*)p)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router: logits, per-group top-k with ties to the lower head index, gates. */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * x      [B*T, d_model]  (dtype)
+ * W_r    [d_model, h]    (dtype)
+ * bias   [h] float or NULL
+ * logits [B*T, h]   out: fp32-rounded logits
+ * idx    [B*T, g, k] out: selected global head indices, ordered by
+ *                         (logit descending, head index ascending)
+ * gate   [B*T, g, k] out: renormalised gates (double)
+ * margin [B*T, g]    out: l_(k) - l_(k+1) within the group, +inf when k == h/g
+ */
+int oracle_route(int64_t BT, int d_model, int h, int g, int k, int dtype,
+                 const void* x, const void* W_r, const float* bias,
+                 float* logits, int32_t* idx, double* gate, double* margin) {
+    if (BT < 0 || d_model < 1 || h < 1 || g < 1 || h % g != 0) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    int* order = (int*)malloc(sizeof(int) * (size_t)hpg);
+    if (!order) return 2;
+    for (int64_t r = 0; r < BT; ++r) {
+        for (int j = 0; j < h; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < d_model; ++i)
+                acc += load_elem(x, (size_t)r * d_model + i, dtype) *
+                       load_elem(W_r, (size_t)i * h + j, dtype);
+            if (bias) acc += (double)bias[j];
+            logits[(size_t)r * h + j] = (float)acc;
+        }
+        for (int q = 0; q < g; ++q) {
+            const float* lg = logits + (size_t)r * h + (size_t)q * hpg;
+            /* insertion sort of the group's heads by (logit desc, index asc) */
+            for (int a = 0; a < hpg; ++a) {
+                int pos = a;
+                while (pos > 0) {
+                    int prev = order[pos - 1];
+                    if (lg[prev] < lg[a]) {
+                        order[pos] = prev;
+                        --pos;
+                    } else {
+                        break;
+                    }
+                }
+                order[pos] = a;
+            }
+            const double m = (double)lg[order[0]];
+            double denom = 0.0;
+            for (int s = 0; s < k; ++s) denom += exp((double)lg[order[s]] - m);
+            for (int s = 0; s < k; ++s) {
+                size_t o = ((size_t)r * g + q) * k + s;
+                idx[o] = q * hpg + order[s];
+                gate[o] = exp((double)lg[order[s]] - m) / denom;
+            }
+            margin[(size_t)r * g + q] =
+                (k == hpg) ? INFINITY : (double)lg[order[k - 1]] - (double)lg[order[k]];
+        }
+    }
+    free(order);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Compaction: per (batch, head) the ascending list of routed positions.     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * idx          [B, T, g, k]
+ * head_offsets [B*h + 1] out: start of the list of (b, j) in head_pos
+ * head_pos     [B*T*g*k] out: positions t, ascending within each list
+ */
+int oracle_compact(int B, int T, int h, int g, int k, const int32_t* idx,
+                   int32_t* head_offsets, int32_t* head_pos) {
+    if (B < 0 || T < 0 || h < 1 || g < 1 || h % g != 0) return 1;
+    const int hpg = h / g;
+    int64_t n = 0;
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < h; ++j) {
+            const int q = j / hpg;
+            head_offsets[(size_t)b * h + j] = (int32_t)n;
+            for (int t = 0; t < T; ++t) {
+                const int32_t* sel = idx + (((size_t)b * T + t) * g + q) * k;
+                int hit = 0;
+                for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
+                if (hit) head_pos[n++] = t;
+            }
+        }
+    }
+    head_offsets[(size_t)B * h] = (int32_t)n;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention for one routed (b, t, j): causal scaled dot-product attention.  */
+/* ------------------------------------------------------------------------ */
+
+/* One query vector against keys 0..n_keys-1 taken with a row stride.  The
+ * result o[d_h] is the softmax-weighted mean of the value rows. */
+static void attend_one(const void* qv, size_t q_off, const void* K, const void* V,
+                       size_t kv_base, size_t kv_row_stride, int64_t n_keys, int d_h,
+                       int dtype, double* scores, double* o) {
+    const double scale = 1.0 / sqrt((double)d_h);
+    double mx = -INFINITY;
+    for (int64_t s = 0; s < n_keys; ++s) {
+        double dot = 0.0;
+        const size_t kr = kv_base + (size_t)s * kv_row_stride;
+        for (int d = 0; d < d_h; ++d)
+            dot += load_elem(qv, q_off + d, dtype) * load_elem(K, kr + d, dtype);
+        scores[s] = dot * scale;
+        if (scores[s] > mx) mx = scores[s];
+    }
+    double denom = 0.0;
+    for (int64_t s = 0; s < n_keys; ++s) {
+        scores[s] = exp(scores[s] - mx);
+        denom += scores[s];
+    }
+    for (int d = 0; d < d_h; ++d) o[d] = 0.0;
+    for (int64_t s = 0; s < n_keys; ++s) {
+        const size_t vr = kv_base + (size_t)s * kv_row_stride;
+        const double w = scores[s] / denom;
+        for (int d = 0; d < d_h; ++d) o[d] += w * load_elem(V, vr + d, dtype);
+    }
+}
+
+/*
+ * Full GQE output for a list of token rows.
+ * Q [B, T, h, d_h], K/V [B, T, g, d_h] (dtype); idx/gate [B, T, g, k]
+ * rows [n_rows]: flattened token index b*T + t
+ * O_rows [n_rows, h, d_h] out (double): gate * attention for selected heads,
+ *                                        0 for unselected heads
+ */
+int oracle_attn_rows(int B, int T, int h, int g, int d_h, int k, int dtype,
+                     const void* Q, const void* K, const void* V,
+                     const int32_t* idx, const double* gate,
+                     int64_t n_rows, const int64_t* rows, double* O_rows, int n_threads) {
+    if (B < 0 || T < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * T) return 1;
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)T);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d_h);
+        if (!scores || !o) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n_rows; ++r) {
+                const int64_t bt = rows[r];
+                const int64_t b = bt / T, t = bt % T;
+                double* out = O_rows + (size_t)r * h * d_h;
+                for (int i = 0; i < h * d_h; ++i) out[i] = 0.0;
+                for (int q = 0; q < g; ++q) {
+                    for (int s = 0; s < k; ++s) {
+                        const size_t sel = ((size_t)bt * g + q) * k + s;
+                        const int j = idx[sel];
+                        const size_t q_off = ((size_t)bt * h + j) * d_h;
+                        const size_t kv_base = ((size_t)b * T * g + q) * d_h;
+                        attend_one(Q, q_off, K, V, kv_base, (size_t)g * d_h, t + 1, d_h, dtype,
+                                   scores, o);
+                        for (int d = 0; d < d_h; ++d) out[(size_t)j * d_h + d] = gate[sel] * o[d];
+                    }
+                }
+            }
+        }
+        free(scores);
+        free(o);
+    }
+    return err;
+}
+
+/*
+ * Decode: one query token per sequence.
+ * query [B, h, d_h]; K_cache/V_cache [B, Lmax, g, d_h] (dtype); lengths [B]
+ * idx/gate [B, g, k]; O [B, h, d_h] out (double).
+ * The query sits at position lengths[b] - 1 and sees cache rows 0 .. lengths[b]-1.
+ */
+int oracle_decode(int B, int Lmax, int h, int g, int d_h, int k, int dtype,
+                  const void* query, const void* K_cache, const void* V_cache,
+                  const int32_t* lengths, const int32_t* idx, const double* gate,
+                  double* O, int n_threads) {
+    if (B < 0 || Lmax < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    for (int b = 0; b < B; ++b)
+        if (lengths[b] < 1 || lengths[b] > Lmax) return 1;
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)Lmax);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d_h);
+        if (!scores || !o) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1) collapse(2)
+            for (int b = 0; b < B; ++b) {
+                for (int q = 0; q < g; ++q) {
+                    for (int jj = 0; jj < hpg; ++jj)
+                        for (int d = 0; d < d_h; ++d)
+                            O[((size_t)b * h + q * hpg + jj) * d_h + d] = 0.0;
+                    for (int s = 0; s < k; ++s) {
+                        const size_t sel = ((size_t)b * g + q) * k + s;
+                        const int j = idx[sel];
+                        const size_t q_off = ((size_t)b * h + j) * d_h;
+                        const size_t kv_base = ((size_t)b * Lmax * g + q) * d_h;
+                        attend_one(query, q_off, K_cache, V_cache, kv_base, (size_t)g * d_h,
+                                   lengths[b], d_h, dtype, scores, o);
+                        for (int d = 0; d < d_h; ++d)
+                            O[((size_t)b * h + j) * d_h + d] = gate[sel] * o[d];
+                    }
+                }
+            }
+        }
+        free(scores);
+        free(o);
+    }
+    return err;
+}

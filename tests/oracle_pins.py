@@ -1,0 +1,378 @@
+"""Pins for the CPU oracle: facts fixed by the pages and by mathematics,
+independent of the oracle's own code.
+
+Every check takes an ``oracle.Oracle`` instance and raises AssertionError on a
+mismatch, so the same checks run against the real oracle (test_oracle_pins.py)
+and against deliberately broken copies of it (test_oracle_mutants.py).
+
+Sources of the pinned facts:
+  * torch.nn.functional.scaled_dot_product_attention (fp64, CPU, causal,
+    enable_gqa) -- a library routine that expands KV heads by repetition
+    like the ml-canon "56 GQA / MQA" page, section "PyTorch GQA", and scales
+    by 1/sqrt(d) like IBM's GQA page (scaled dot-product attention).
+  * freenetmedia.pl "Grouped-Query Attention", section "Jak dzialaja...":
+    8 query heads in 2 groups -> heads 0-3 share KV head 0, heads 4-7 KV head 1
+    (tests/golden/head_group_map.txt).
+  * gist.science "Grouped Query Experts", "Resultats Experimentaux": with 16
+    query heads, 8 KV groups and k=1, 8 routed query-head computations per
+    token (tests/golden/active_heads.txt).
+  * Brute force over all C(h/g, k) subsets for the top-k selection; closed
+    forms (T=1, zero keys, constant values, one dominant key, k=2 gate =
+    logistic of the logit gap, W_r=0 ties).
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+from scipy.special import expit, softmax
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _f32(shape, seed, scale=1.0):
+    return (_rng(seed).standard_normal(shape) * scale).astype(np.float32)
+
+
+def read_golden(name):
+    """Rows of integers from a golden fixture (lines starting with # are comments)."""
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([int(v) for v in line.split()])
+    return rows
+
+
+# --------------------------------------------------------------------------
+# Router
+# --------------------------------------------------------------------------
+
+def check_router_onehot(o):
+    """x = e_i gives logits = fp32(W_r[i, :] + bias): pins the orientation of
+    W_r ([d_model, h]) and the bias term."""
+    d_model, h, g = 6, 4, 2
+    W = _f32((d_model, h), 1)
+    bias = _f32((h,), 2)
+    x = np.eye(d_model, dtype=np.float32)
+    _, _, logits, _ = o.route(x, W, h, g, 1, bias=bias)
+    expect = (W.astype(np.float64) + bias.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(logits, expect), "one-hot logits differ from W_r rows + bias"
+    # doubling x doubles every logit exactly (linear, no constant term besides bias)
+    x2 = _f32((5, d_model), 3)
+    _, _, l1, _ = o.route(x2, W, h, g, 1)
+    _, _, l2, _ = o.route(2 * x2, W, h, g, 1)
+    assert np.array_equal(2 * l1, l2), "router is not linear in x"
+
+
+def _bruteforce_select(lg, k):
+    """Subset of size k with the largest exact logit sum; equal sums -> the
+    lexicographically smallest index tuple.  Returned in (logit desc, index asc) order."""
+    best, best_sum = None, None
+    for comb in itertools.combinations(range(len(lg)), k):
+        s = sum(Fraction(float(lg[i])) for i in comb)
+        if best is None or s > best_sum:
+            best, best_sum = comb, s
+    return sorted(best, key=lambda i: (-float(lg[i]), i))
+
+
+def check_router_bruteforce(o):
+    """Selected heads equal the brute-force best subset per (token, group),
+    including heavy ties (logits drawn from 3 values)."""
+    for (h, g, k, seed, quant) in [(8, 2, 1, 10, False), (8, 2, 2, 11, False), (12, 3, 3, 12, False),
+                                   (8, 2, 2, 13, True), (12, 2, 4, 14, True), (6, 6, 1, 15, False)]:
+        hpg = h // g
+        d_model = 16
+        if quant:
+            # one-hot tokens and a W_r with values in {-1, 0, 1}: many exact ties
+            W = _rng(seed).integers(-1, 2, size=(d_model, h)).astype(np.float32)
+            x = np.eye(d_model, dtype=np.float32)
+        else:
+            W = _f32((d_model, h), seed, 0.5)
+            x = _f32((20, d_model), seed + 100)
+        idx, gate, logits, margin = o.route(x, W, h, g, k)
+        for r in range(x.shape[0]):
+            for q in range(g):
+                lg = logits[r, q * hpg:(q + 1) * hpg]
+                want = [q * hpg + i for i in _bruteforce_select(lg, k)]
+                assert list(idx[r, q]) == want, f"selection {list(idx[r, q])} != brute force {want}"
+                srt = np.sort(lg.astype(np.float64))[::-1]
+                exp_margin = math.inf if k == hpg else srt[k - 1] - srt[k]
+                assert margin[r, q] == exp_margin, "margin is not l_(k) - l_(k+1)"
+
+
+def check_router_zero_weights(o):
+    """W_r = 0: every logit ties, so the first k heads of every group win and
+    each gate is exactly 1/k."""
+    h, g, k = 12, 3, 2
+    x = _f32((7, 10), 5)
+    idx, gate, _, _ = o.route(x, np.zeros((10, h), np.float32), h, g, k)
+    hpg = h // g
+    for q in range(g):
+        assert (idx[:, q, :] == np.arange(q * hpg, q * hpg + k)).all(), "tie rule: lower index first"
+    assert (gate == 1.0 / k).all(), "tied gates must be exactly 1/k"
+
+
+def check_gates(o):
+    """Gates are the router softmax renormalised over the k selected heads."""
+    x = _f32((30, 16), 21)
+    W = _f32((16, 8), 22, 0.7)
+    # k = 1: gate is exactly 1
+    _, gate1, _, _ = o.route(x, W, 8, 2, 1)
+    assert (gate1 == 1.0).all(), "k=1 gates must be 1"
+    # k = 2: gate of the top head is the logistic function of the logit gap
+    idx, gate, logits, _ = o.route(x, W, 8, 2, 2)
+    for r in range(x.shape[0]):
+        for q in range(2):
+            l0 = float(logits[r, idx[r, q, 0]])
+            l1 = float(logits[r, idx[r, q, 1]])
+            assert abs(gate[r, q, 0] - expit(l0 - l1)) < 1e-14
+            assert abs(gate[r, q, 1] - expit(l1 - l0)) < 1e-14
+    # k = 3 of 4: scipy softmax over the selected logits
+    idx, gate, logits, _ = o.route(x, W, 8, 2, 3)
+    for r in range(x.shape[0]):
+        for q in range(2):
+            sel = logits[r, idx[r, q]].astype(np.float64)
+            assert np.allclose(gate[r, q], softmax(sel), rtol=0, atol=1e-14)
+            assert abs(gate[r, q].sum() - 1.0) < 1e-14 and (gate[r, q] > 0).all()
+
+
+# --------------------------------------------------------------------------
+# Compaction
+# --------------------------------------------------------------------------
+
+def check_compact(o):
+    """Packed lists equal np.nonzero of the selection mask; lists strictly
+    increasing; every selected (t, j) appears once; totals are T*g*k."""
+    B, T, h, g, k = 3, 37, 8, 2, 2
+    x = _f32((B, T, 12), 31)
+    W = _f32((12, h), 32)
+    idx, _, _, _ = o.route(x, W, h, g, k)
+    offs, pos = o.compact(idx, h, g, k)
+    mask = np.zeros((B, T, h), bool)
+    for b in range(B):
+        for t in range(T):
+            mask[b, t, idx[b, t].reshape(-1)] = True
+    assert offs[0] == 0 and offs[-1] == B * T * g * k
+    for b in range(B):
+        for j in range(h):
+            lst = pos[offs[b * h + j]:offs[b * h + j + 1]]
+            assert np.array_equal(lst, np.nonzero(mask[b, :, j])[0]), "list != nonzero(mask)"
+            assert (np.diff(lst) > 0).all()
+        assert offs[(b + 1) * h] - offs[b * h] == T * g * k
+
+
+# --------------------------------------------------------------------------
+# Attention
+# --------------------------------------------------------------------------
+
+def _random_routing(B, T, h, g, k, seed):
+    """Random valid routing (k distinct heads of each group, positive gates
+    summing to one), independent of the router."""
+    r = _rng(seed)
+    hpg = h // g
+    idx = np.empty((B, T, g, k), np.int32)
+    gate = np.empty((B, T, g, k), np.float64)
+    for b in range(B):
+        for t in range(T):
+            for q in range(g):
+                idx[b, t, q] = q * hpg + r.permutation(hpg)[:k]
+                w = r.random(k) + 0.1
+                gate[b, t, q] = w / w.sum()
+    return idx, gate
+
+
+def _sdpa_expected(Q, K, V, idx, gate):
+    """gate * causal SDPA (torch, fp64, GQA expansion) for selected heads, 0 elsewhere."""
+    q = torch.from_numpy(Q.astype(np.float64)).transpose(1, 2)
+    kk = torch.from_numpy(K.astype(np.float64)).transpose(1, 2)
+    vv = torch.from_numpy(V.astype(np.float64)).transpose(1, 2)
+    full = F.scaled_dot_product_attention(q, kk, vv, is_causal=True, enable_gqa=True)
+    full = full.transpose(1, 2).numpy()  # [B, T, h, d]
+    B, T, h, d = Q.shape
+    out = np.zeros_like(full)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(idx.shape[2]):
+                for s in range(idx.shape[3]):
+                    j = idx[b, t, q_, s]
+                    out[b, t, j] = gate[b, t, q_, s] * full[b, t, j]
+    return out
+
+
+def check_attn_sdpa(o):
+    """Routed output = gate x torch SDPA(causal, GQA) on selected heads, zero elsewhere."""
+    for (B, T, h, g, d, k, seed) in [(2, 19, 8, 2, 16, 2, 40), (1, 33, 6, 3, 8, 1, 41),
+                                     (1, 12, 4, 1, 8, 4, 42), (1, 9, 4, 4, 8, 1, 43)]:
+        Q = _f32((B, T, h, d), seed)
+        K = _f32((B, T, g, d), seed + 1)
+        V = _f32((B, T, g, d), seed + 2)
+        idx, gate = _random_routing(B, T, h, g, k, seed + 3)
+        got = o.attn(Q, K, V, idx, gate)
+        want = _sdpa_expected(Q, K, V, idx, gate)
+        assert np.abs(got - want).max() < 1e-12, f"SDPA mismatch {np.abs(got - want).max()}"
+
+
+def check_attn_closed_forms(o):
+    B, T, h, g, d, k = 1, 11, 4, 2, 8, 1
+    idx, gate = _random_routing(B, T, h, g, k, 50)
+    Q = _f32((B, T, h, d), 51)
+    V = _f32((B, T, g, d), 52)
+    # T = 1: the only visible key is the token itself -> O = gate * V[0]
+    O1 = o.attn(Q[:, :1], _f32((B, 1, g, d), 53), V[:, :1], idx[:, :1], gate[:, :1])
+    for q_ in range(g):
+        j = idx[0, 0, q_, 0]
+        assert np.allclose(O1[0, 0, j], gate[0, 0, q_, 0] * V[0, 0, q_].astype(np.float64), atol=1e-15)
+    # K = 0: uniform weights over s <= t -> running mean of V
+    O0 = o.attn(Q, np.zeros((B, T, g, d), np.float32), V, idx, gate)
+    Vd = V.astype(np.float64)
+    run_mean = np.cumsum(Vd, axis=1) / np.arange(1, T + 1)[None, :, None, None]
+    for t in range(T):
+        for q_ in range(g):
+            j = idx[0, t, q_, 0]
+            assert np.allclose(O0[0, t, j], gate[0, t, q_, 0] * run_mean[0, t, q_], atol=1e-13)
+    # constant V rows: output equals that row whatever the weights
+    vc = _f32((g, d), 54)
+    Vc = np.broadcast_to(vc, (B, T, g, d)).copy()
+    Oc = o.attn(Q, _f32((B, T, g, d), 55), Vc, idx, gate)
+    for t in range(T):
+        for q_ in range(g):
+            j = idx[0, t, q_, 0]
+            assert np.allclose(Oc[0, t, j], gate[0, t, q_, 0] * vc[q_].astype(np.float64), atol=1e-13)
+    # one dominant key at s* = 4: rows t >= 4 return V[s*], rows t < 4 see only zero scores
+    Qd = np.zeros((B, T, h, d), np.float32)
+    Qd[..., 0] = 30.0
+    Kd = np.zeros((B, T, g, d), np.float32)
+    Kd[0, 4, :, 0] = 30.0
+    Od = o.attn(Qd, Kd, V, idx, gate)
+    for t in range(T):
+        for q_ in range(g):
+            j = idx[0, t, q_, 0]
+            want = Vd[0, 4, q_] if t >= 4 else run_mean[0, t, q_]
+            assert np.allclose(Od[0, t, j], gate[0, t, q_, 0] * want, atol=1e-12), f"dominant key t={t}"
+
+
+def check_mha_mqa(o):
+    """g = h (MHA): one head per group, gate 1, output = causal SDPA without
+    expansion.  g = 1 (MQA) with k = h: every head attends the single KV head."""
+    B, T, h, d = 1, 14, 4, 8
+    Q = _f32((B, T, h, d), 60)
+    K = _f32((B, T, h, d), 61)
+    V = _f32((B, T, h, d), 62)
+    x = _f32((B, T, 5), 63)
+    idx, gate, _, _ = o.route(x, _f32((5, h), 64), h, h, 1)
+    assert (gate == 1.0).all()
+    got = o.attn(Q, K, V, idx, gate)
+    t = lambda a: torch.from_numpy(a.astype(np.float64)).transpose(1, 2)
+    want = F.scaled_dot_product_attention(t(Q), t(K), t(V), is_causal=True).transpose(1, 2).numpy()
+    assert np.abs(got - want).max() < 1e-12
+    K1, V1 = K[:, :, :1], V[:, :, :1]
+    idx, gate, _, _ = o.route(x, _f32((5, h), 65), h, 1, h)
+    got = o.attn(Q, K1, V1, idx, gate)
+    base = F.scaled_dot_product_attention(t(Q), t(K1).expand(B, h, T, d), t(V1).expand(B, h, T, d),
+                                          is_causal=True).transpose(1, 2).numpy()
+    g_of_head = np.zeros((B, T, h))
+    for s in range(h):
+        g_of_head[0, np.arange(T), idx[0, :, 0, s]] = gate[0, :, 0, s]
+    assert np.abs(got - g_of_head[..., None] * base).max() < 1e-12
+
+
+def check_prefix_invariance(o):
+    """Truncating the sequence leaves the earlier rows bit-identical (causality)."""
+    B, T, h, g, d, k = 2, 24, 8, 2, 16, 2
+    Q = _f32((B, T, h, d), 70)
+    K = _f32((B, T, g, d), 71)
+    V = _f32((B, T, g, d), 72)
+    idx, gate = _random_routing(B, T, h, g, k, 73)
+    full = o.attn(Q, K, V, idx, gate)
+    Tp = 13
+    part = o.attn(Q[:, :Tp].copy(), K[:, :Tp].copy(), V[:, :Tp].copy(), idx[:, :Tp].copy(), gate[:, :Tp].copy())
+    assert np.array_equal(full[:, :Tp], part)
+
+
+def check_decode(o):
+    """Decode of a query at position L-1 equals SDPA over cache rows 0..L-1, and
+    equals the prefill row t = L-1 built from the same rows."""
+    B, Lmax, h, g, d, k = 3, 21, 8, 2, 16, 2
+    lengths = np.array([1, 13, 21], np.int32)
+    q = _f32((B, 1, h, d), 80)
+    Kc = _f32((B, Lmax, g, d), 81)
+    Vc = _f32((B, Lmax, g, d), 82)
+    idx, gate = _random_routing(B, 1, h, g, k, 83)
+    got = o.decode(q, Kc, Vc, lengths, idx, gate)
+    for b in range(B):
+        L = int(lengths[b])
+        qq = torch.from_numpy(q[b:b + 1].astype(np.float64)).transpose(1, 2)  # [1,h,1,d]
+        kk = torch.from_numpy(Kc[b:b + 1, :L].astype(np.float64)).transpose(1, 2)
+        vv = torch.from_numpy(Vc[b:b + 1, :L].astype(np.float64)).transpose(1, 2)
+        full = F.scaled_dot_product_attention(qq, kk, vv, enable_gqa=True)[0, :, 0]  # [h, d]
+        want = np.zeros((h, d))
+        for q_ in range(g):
+            for s in range(k):
+                j = idx[b, 0, q_, s]
+                want[j] = gate[b, 0, q_, s] * full[j].numpy()
+        assert np.abs(got[b] - want).max() < 1e-12, f"decode b={b}"
+        # decode <-> prefill: put q at position L-1 of a prefill over the cache rows
+        Qp = np.zeros((1, L, h, d), np.float32)
+        Qp[0, L - 1] = q[b, 0]
+        ip = np.repeat(idx[b:b + 1], L, axis=1)
+        gp = np.repeat(gate[b:b + 1], L, axis=1)
+        row = o.attn_rows(Qp, Kc[b:b + 1, :L].copy(), Vc[b:b + 1, :L].copy(), ip, gp, rows=[L - 1])
+        assert np.abs(row[0] - got[b]).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
+# Worked examples printed on the pages (tests/golden)
+# --------------------------------------------------------------------------
+
+def check_group_map_golden(o):
+    """freenetmedia.pl example: h=8, g=2 -> heads 0-3 use KV head 0, 4-7 KV head 1."""
+    rows = read_golden("head_group_map.txt")
+    h, g = rows[0][0], rows[0][1]
+    expect = {r[0]: r[1] for r in rows[1:]}
+    B, T, d = 1, 3, 4
+    Q = _f32((B, T, h, d), 90)
+    K = _f32((B, T, g, d), 91)
+    V = np.zeros((B, T, g, d), np.float32)
+    for q_ in range(g):
+        V[:, :, q_, :] = float(q_ + 1)  # KV head q carries the constant value q + 1
+    x = _f32((B, T, 6), 92)
+    idx, gate, _, _ = o.route(x, _f32((6, h), 93), h, g, h // g)  # every head selected
+    O = o.attn(Q, K, V, idx, gate)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                for s in range(h // g):
+                    j = idx[b, t, q_, s]
+                    kv = O[b, t, j, 0] / gate[b, t, q_, s] - 1.0
+                    assert abs(kv - expect[j]) < 1e-12, f"head {j} read KV head {kv}, pages say {expect[j]}"
+
+
+def check_active_heads_golden(o):
+    """gist.science main configuration: 16 query heads, 8 KV groups, k=1 ->
+    8 routed query-head computations per token (the always-on shared head is a
+    separate, extra head and not part of the routed output)."""
+    h, g, k, routed = read_golden("active_heads.txt")[0]
+    B, T, d = 1, 10, 8
+    x = _f32((B, T, 32), 95)
+    idx, gate, _, _ = o.route(x, _f32((32, h), 96), h, g, k)
+    O = o.attn(_f32((B, T, h, d), 97), _f32((B, T, g, d), 98), _f32((B, T, g, d), 99), idx, gate)
+    nonzero = (np.abs(O).sum(axis=-1) > 0).sum(axis=-1)
+    assert (nonzero == routed).all(), f"nonzero head slots per token {set(nonzero.ravel())} != {routed}"
+
+
+ALL_CHECKS = [
+    check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
+    check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
+    check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
+]

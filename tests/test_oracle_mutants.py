@@ -1,0 +1,62 @@
+"""The pins have teeth: each plausible mistake, planted in a copy of the
+oracle's C source on the CPU, makes at least one pin in oracle_pins.py fail.
+
+Each mutant is compiled into a temporary library and checked in a child
+process (a broken copy may crash)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# (name, original text, planted mistake)
+MUTANTS = [
+    ("scale_1_over_d", "1.0 / sqrt((double)d_h)", "1.0 / (double)d_h"),
+    ("causal_excludes_diagonal", "t + 1, d_h, dtype,", "t, d_h, dtype,"),
+    ("causal_sees_one_future_key", "t + 1, d_h, dtype,", "(t + 1 < T ? t + 2 : t + 1), d_h, dtype,"),
+    ("strided_head_group_map", "idx[o] = q * hpg + order[s];", "idx[o] = order[s] * g + q;"),
+    ("ties_to_higher_index", "if (lg[prev] < lg[a]) {", "if (lg[prev] <= lg[a]) {"),
+    ("gate_over_all_group_heads", "for (int s = 0; s < k; ++s) denom +=", "for (int s = 0; s < hpg; ++s) denom +="),
+    ("transposed_router_weight", "load_elem(W_r, (size_t)i * h + j, dtype)", "load_elem(W_r, ((size_t)j * d_model + i) % ((size_t)d_model * h), dtype)"),
+    ("dropped_bias", "if (bias) acc += (double)bias[j];", "(void)bias;"),
+    ("unnormalised_weights", "const double w = scores[s] / denom;", "const double w = scores[s];"),
+    ("decode_query_position", "lengths[b], d_h, dtype, scores, o);", "lengths[b] - 1 > 0 ? lengths[b] - 1 : 1, d_h, dtype, scores, o);"),
+    ("gate_not_applied", "out[(size_t)j * d_h + d] = gate[sel] * o[d];", "out[(size_t)j * d_h + d] = o[d];"),
+    ("unselected_heads_not_zero", "for (int i = 0; i < h * d_h; ++i) out[i] = 0.0;", "for (int i = 0; i < h * d_h; ++i) out[i] = 1e-3;"),
+    ("transposed_qk_index", "load_elem(K, kr + d, dtype)", "load_elem(K, kv_base + (size_t)d * kv_row_stride + (size_t)s % (size_t)d_h, dtype)"),
+    ("compact_strided_group", "const int q = j / hpg;", "const int q = j % g;"),
+]
+
+_CHILD = r"""
+import sys
+sys.path.insert(0, {root!r})
+import oracle
+from tests import oracle_pins
+o = oracle.Oracle({lib!r})
+failed = []
+for c in oracle_pins.ALL_CHECKS:
+    try:
+        c(o)
+    except Exception as e:
+        failed.append(c.__name__)
+print("FAILED:" + ",".join(failed))
+"""
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    mutated = src.replace(old, new)
+    c_path = tmp_path / "mutant.c"
+    c_path.write_text(mutated)
+    lib = str(tmp_path / "libmutant.so")
+    oracle.compile_source(str(c_path), lib, strict=False)
+    proc = subprocess.run([sys.executable, "-c", _CHILD.format(root=ROOT, lib=lib)],
+                          capture_output=True, text=True, timeout=300)
+    caught = proc.returncode != 0 or ("FAILED:" in proc.stdout and proc.stdout.split("FAILED:")[1].strip())
+    assert caught, f"mutant {name} passed every pin:\n{proc.stdout}\n{proc.stderr[-2000:]}"
