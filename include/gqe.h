@@ -1,0 +1,168 @@
+/*
+ * gqe.h -- C ABI of libgqe: the forward pass of a Grouped Query Experts (GQE)
+ * attention layer on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention",
+ * gist.science summary, section "Architecture et Routage"): the KV heads of
+ * grouped-query attention stay dense; inside each KV group a per-token router
+ * picks k of the group's query heads ("experts"); those heads run causal
+ * attention against the group's shared K/V; each selected head's output is
+ * scaled by its router probability renormalised over the k selected heads
+ * ("Somme Ponderee Renormalisee"); unselected heads output zero.
+ *
+ * Notation.  B batch, T sequence length, d_model router input width, h query
+ * heads, g KV heads (groups), d_h head width, k heads selected per group,
+ * hpg = h / g.  Query head j belongs to group j / hpg (contiguous blocks, as in
+ * the 8-heads / 2-groups example of the freenetmedia.pl GQA page, section
+ * "Jak dzialaja...").
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named as device pointers must point to device memory of the
+ *    current CUDA device; the caller owns every buffer (this library never
+ *    allocates or frees memory, and never synchronises except in
+ *    gqe_get_device_status).
+ *  - Tensors are dense, row-major, last index fastest.  Activation tensors
+ *    (x, W_r, Q, K, V, caches, O) must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously; a call returns once its kernels are launched.
+ *  - Arguments are validated on the host before anything is enqueued.  An
+ *    invalid argument returns GQE_ERR_INVALID_ARGUMENT and enqueues nothing; a
+ *    valid request outside the implemented cases returns GQE_ERR_UNSUPPORTED and
+ *    enqueues nothing; a failed launch returns GQE_ERR_CUDA.
+ *  - `workspace` is caller-owned device scratch of at least
+ *    gqe_workspace_bytes() bytes, 256-byte aligned.  Its first 256 bytes hold a
+ *    device status word: zero it once with gqe_workspace_init() after
+ *    allocation.  A kernel whose bounded wait expires records
+ *    GQE_ERR_DEVICE_TIMEOUT there and returns early; read it with
+ *    gqe_get_device_status().  Calls that share a workspace must be ordered on
+ *    one stream.
+ *  - Outputs must not alias inputs.
+ */
+#ifndef GQE_H
+#define GQE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQE_OK = 0,
+    GQE_ERR_INVALID_ARGUMENT = 1,
+    GQE_ERR_UNSUPPORTED = 2,
+    GQE_ERR_CUDA = 3,
+    GQE_ERR_DEVICE_TIMEOUT = 4
+} gqe_status;
+
+typedef enum { GQE_F32 = 0, GQE_BF16 = 1 } gqe_dtype;
+
+typedef struct {
+    int B, T, d_model, h, g, d_h, k;
+    int dtype; /* gqe_dtype: element type of x, W_r, Q, K, V, caches and O */
+} gqe_shape;
+
+/* Number of 32-token chunks per sequence: ceil(T / 32).  Sizes the
+ * head_chunk_offsets array of gqe_route. */
+int gqe_chunk_count(int T);
+
+/* Bytes of device workspace needed by the calls on shape *s.  Lmax is the
+ * cache capacity for gqe_attn_decode (0 for prefill-only use).  Returns 0 for
+ * an invalid shape. */
+size_t gqe_workspace_bytes(const gqe_shape* s, int Lmax);
+
+/* Zero the status word of a workspace (asynchronous, on `stream`). */
+gqe_status gqe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_route -- router, per-group top-k and token compaction.
+ *
+ * Router (gist.science GQE summary, "Architecture et Routage"; the linear form
+ * is this library's reading, the page gives no formula):
+ *   l[b,t,j] = sum_i x[b,t,i] * W_r[i,j] + bias[j], accumulated in fp32.
+ * Per token and group q, the k heads of q with the largest fp32 logits are
+ * selected; equal logits go to the lower head index.  gate = the softmax of
+ * the selected logits (the group softmax renormalised over the selection,
+ * "Somme Ponderee Renormalisee").
+ * Compaction: for every (b, j), the ascending list of positions t whose
+ * selection contains j, built by warp ballots and prefix sums.
+ *
+ *   x        [B, T, d_model]   device, dtype
+ *   W_r      [d_model, h]      device, dtype
+ *   bias     [h]               device fp32, or NULL for no bias
+ *   idx      [B, T, g, k]      device int32 out: selected global head indices
+ *                              per (token, group), by logit descending (ties:
+ *                              lower index first)
+ *   gate     [B, T, g, k]      device fp32 out: renormalised gates, same order
+ *   head_offsets [B*h + 1]     device int32 out: head_pos index of the first
+ *                              entry of (b, j) at [b*h + j]; [B*h] = B*T*g*k
+ *   head_pos [B*T*g*k]         device int32 out: positions t, ascending within
+ *                              each (b, j) list
+ *   head_chunk_offsets [B*h*gqe_chunk_count(T)]
+ *                              device int32 out: at [(b*h + j)*nchunk + c] the
+ *                              head_pos index of the first entry of (b, j) with
+ *                              t >= 32*c
+ * Requires h % g == 0, 1 <= k <= h/g, B*T*g*k < 2^31.
+ */
+gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                     int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                     int32_t* head_chunk_offsets, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
+ * gqe_attn_prefill -- routed causal attention with the gated scatter.
+ *
+ * For every routed (b, t, j), with q = Q[b,t,j,:] and group q_ = j / hpg:
+ *   o = sum_{s <= t} softmax_s(q . K[b,s,q_,:] / sqrt(d_h)) V[b,s,q_,:]
+ * (scaled dot-product attention, IBM GQA page; KV heads shared per group,
+ * ml-canon "56 GQA / MQA", "PyTorch GQA"; causal on the original positions),
+ * and O[b,t,j,:] = gate * o.  O[b,t,j,:] = 0 for every unselected (t, j).
+ * O is written in full.
+ *
+ *   Q [B, T, h, d_h], K/V [B, T, g, d_h]   device, dtype
+ *   idx, gate, head_offsets, head_pos, head_chunk_offsets
+ *                                          device, exactly as written by gqe_route
+ *   O [B, T, h, d_h]                       device, dtype, out
+ * Implemented cases: bf16 with d_h = 128 (tensor cores); fp32 with
+ * d_h in {32, 64, 128} (CUDA cores).
+ */
+gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                            const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                            const int32_t* head_pos, const int32_t* head_chunk_offsets, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_attn_decode -- one new query token per sequence against a KV cache.
+ *
+ * The cache of sequence b holds rows 0 .. lengths[b]-1 (the new token's own
+ * K/V included); the query sits at position lengths[b]-1 and sees all of them.
+ * The KV cache stays dense under GQE (gist.science summary, "Chemin KV
+ * Dense"), so every group's cache rows are read once and shared by the k
+ * routed heads of that group.  Output as for prefill with T = 1.
+ *
+ *   s->T must be 1.  q [B, 1, h, d_h] device, dtype.
+ *   K_cache, V_cache [B, Lmax, g, d_h]   device, dtype
+ *   lengths [B]     device int32, each in [1, Lmax] (device-side contract: the
+ *                   kernels clamp out-of-range lengths into [1, Lmax])
+ *   idx, gate       [B, 1, g, k] as written by gqe_route for the new tokens
+ *   O [B, 1, h, d_h] device, dtype, out
+ * Implemented cases: bf16 or fp32, d_h in {32, 64, 128}, k <= 8.
+ */
+gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cache,
+                           const void* V_cache, int Lmax, const int32_t* lengths,
+                           const int32_t* idx, const float* gate, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, read the workspace status word, reset it to zero and
+ * return it (GQE_OK when no kernel reported a failure). */
+gqe_status gqe_get_device_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* gqe_status_string(gqe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQE_H */

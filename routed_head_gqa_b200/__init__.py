@@ -1,0 +1,174 @@
+"""Python binding of libgqe (include/gqe.h): the GQE attention forward pass on B200.
+
+Argument marshalling only.  Every step of the routed path (router, top-k,
+compaction, routed prefill, decode) runs in the library's CUDA kernels; PyTorch
+supplies device memory and the current CUDA stream.  The functions keep the C
+names and raise ``GQEError`` on a non-OK status.  Importing this package fails
+if ``libgqe.so`` has not been built (``python -m routed_head_gqa_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m routed_head_gqa_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+GQE_OK = 0
+GQE_ERR_INVALID_ARGUMENT = 1
+GQE_ERR_UNSUPPORTED = 2
+GQE_ERR_CUDA = 3
+GQE_ERR_DEVICE_TIMEOUT = 4
+GQE_F32 = 0
+GQE_BF16 = 1
+
+EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route",
+            "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status", "gqe_status_string"]
+
+
+class GqeShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("d_model", ctypes.c_int), ("h", ctypes.c_int),
+                ("g", ctypes.c_int), ("d_h", ctypes.c_int), ("k", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class GQEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {gqe_status_string(status)} ({status})")
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+_lib.gqe_chunk_count.argtypes = [_I]
+_lib.gqe_chunk_count.restype = _I
+_lib.gqe_workspace_bytes.argtypes = [ctypes.POINTER(GqeShape), _I]
+_lib.gqe_workspace_bytes.restype = _SZ
+_lib.gqe_workspace_init.argtypes = [_P, _SZ, _P]
+_lib.gqe_route.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.gqe_attn_prefill.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.gqe_attn_decode.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.gqe_get_device_status.argtypes = [_P, _P]
+_lib.gqe_status_string.argtypes = [_I]
+_lib.gqe_status_string.restype = ctypes.c_char_p
+for _f in ("gqe_workspace_init", "gqe_route", "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status"):
+    getattr(_lib, _f).restype = _I
+
+
+def make_shape(B, T, d_model, h, g, d_h, k, dtype) -> GqeShape:
+    """dtype: GQE_F32 / GQE_BF16 or a torch dtype."""
+    if isinstance(dtype, torch.dtype):
+        dtype = GQE_BF16 if dtype == torch.bfloat16 else GQE_F32
+    return GqeShape(int(B), int(T), int(d_model), int(h), int(g), int(d_h), int(k), int(dtype))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _check(fn, status):
+    if status != GQE_OK:
+        raise GQEError(fn, status)
+
+
+def gqe_status_string(status: int) -> str:
+    return _lib.gqe_status_string(int(status)).decode()
+
+
+def gqe_chunk_count(T: int) -> int:
+    return _lib.gqe_chunk_count(int(T))
+
+
+def gqe_workspace_bytes(shape: GqeShape, Lmax: int = 0) -> int:
+    return _lib.gqe_workspace_bytes(ctypes.byref(shape), int(Lmax))
+
+
+def gqe_workspace_init(workspace, stream=None) -> None:
+    _check("gqe_workspace_init", _lib.gqe_workspace_init(_ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def gqe_route(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, head_chunk_offsets, workspace,
+              stream=None) -> None:
+    _check("gqe_route", _lib.gqe_route(ctypes.byref(shape), _ptr(x), _ptr(W_r), _ptr(bias), _ptr(idx),
+                                       _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
+                                       _ptr(head_chunk_offsets), _ptr(workspace), _nbytes(workspace),
+                                       _stream(stream)))
+
+
+def gqe_attn_prefill(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, O, workspace,
+                     stream=None) -> None:
+    _check("gqe_attn_prefill", _lib.gqe_attn_prefill(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                                     _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
+                                                     _ptr(head_chunk_offsets), _ptr(O), _ptr(workspace),
+                                                     _nbytes(workspace), _stream(stream)))
+
+
+def gqe_attn_decode(shape, q, K_cache, V_cache, Lmax, lengths, idx, gate, O, workspace, stream=None) -> None:
+    _check("gqe_attn_decode", _lib.gqe_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache),
+                                                   int(Lmax), _ptr(lengths), _ptr(idx), _ptr(gate), _ptr(O),
+                                                   _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def gqe_get_device_status(workspace, stream=None) -> int:
+    return _lib.gqe_get_device_status(_ptr(workspace), _stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# Buffer helpers: device memory for the calls above, allocated through torch.
+# ---------------------------------------------------------------------------
+class Buffers:
+    """Routing outputs, O and the workspace for one shape on one device."""
+
+    def __init__(self, shape: GqeShape, device="cuda", Lmax: int = 0):
+        B, T, h, g, k, d_h = shape.B, shape.T, shape.h, shape.g, shape.k, shape.d_h
+        dt = torch.bfloat16 if shape.dtype == GQE_BF16 else torch.float32
+        self.shape = shape
+        self.idx = torch.empty((B, T, g, k), dtype=torch.int32, device=device)
+        self.gate = torch.empty((B, T, g, k), dtype=torch.float32, device=device)
+        self.head_offsets = torch.empty(B * h + 1, dtype=torch.int32, device=device)
+        self.head_pos = torch.empty(B * T * g * k, dtype=torch.int32, device=device)
+        self.head_chunk_offsets = torch.empty(B * h * gqe_chunk_count(T), dtype=torch.int32, device=device)
+        self.O = torch.empty((B, T, h, d_h), dtype=dt, device=device)
+        nbytes = gqe_workspace_bytes(shape, Lmax)
+        if nbytes == 0:
+            raise GQEError("gqe_workspace_bytes", GQE_ERR_INVALID_ARGUMENT)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        gqe_workspace_init(self.workspace)
+
+    def route(self, x, W_r, bias=None, stream=None):
+        gqe_route(self.shape, x, W_r, bias, self.idx, self.gate, self.head_offsets, self.head_pos,
+                  self.head_chunk_offsets, self.workspace, stream)
+
+    def prefill(self, Q, K, V, stream=None):
+        gqe_attn_prefill(self.shape, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
+                         self.head_chunk_offsets, self.O, self.workspace, stream)
+
+    def decode(self, q, K_cache, V_cache, lengths, stream=None):
+        gqe_attn_decode(self.shape, q, K_cache, V_cache, K_cache.shape[1], lengths, self.idx, self.gate, self.O,
+                        self.workspace, stream)
+
+    def status(self, stream=None) -> int:
+        return gqe_get_device_status(self.workspace, stream)

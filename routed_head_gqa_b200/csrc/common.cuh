@@ -1,0 +1,139 @@
+// common.cuh -- shared device helpers and internal launch declarations of libgqe.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gqe.h"
+
+namespace gqe {
+
+constexpr int kChunk = 32;             // compaction chunk (one warp ballot)
+constexpr size_t kStatusBytes = 256;   // status word region at the start of the workspace
+
+// Status word layout (uint32 each): [0] error code, [1] kernel id, [2] detail.
+struct DeviceStatus {
+    uint32_t code;
+    uint32_t where;
+    uint32_t detail;
+};
+
+__device__ __forceinline__ void report_error(void* status, uint32_t code, uint32_t where,
+                                             uint32_t detail) {
+    DeviceStatus* st = reinterpret_cast<DeviceStatus*>(status);
+    if (atomicCAS(&st->code, 0u, code) == 0u) {
+        st->where = where;
+        st->detail = detail;
+    }
+}
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <>
+struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+// 16-byte vector <-> fp32 lanes.  For bf16, 8 elements; for fp32, 4.
+template <typename T>
+struct Vec16 {
+    static constexpr int N = 16 / sizeof(T);
+};
+
+__device__ __forceinline__ void unpack16(const uint4& v, float (&f)[8], const __nv_bfloat16*) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void unpack16(const uint4& v, float (&f)[4], const float*) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Streaming (read-once) 16-byte global load.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ------------------------------------------------------------------------
+// Internal launchers (host).  Each returns cudaSuccess or the launch error.
+// ------------------------------------------------------------------------
+struct RouteArgs {
+    const gqe_shape* s;
+    const void* x;
+    const void* W_r;
+    const float* bias;
+    int32_t* idx;
+    float* gate;
+    int32_t* head_offsets;
+    int32_t* head_pos;
+    int32_t* head_chunk_offsets;
+    int32_t* counts;  // workspace: [B*h*nchunk]
+    void* status;
+    cudaStream_t stream;
+};
+cudaError_t launch_route(const RouteArgs& a);
+
+struct PrefillArgs {
+    const gqe_shape* s;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const int32_t* idx;
+    const float* gate;
+    const int32_t* head_offsets;
+    const int32_t* head_pos;
+    const int32_t* head_chunk_offsets;
+    void* O;
+    void* status;
+    cudaStream_t stream;
+};
+cudaError_t launch_prefill_simt(const PrefillArgs& a);
+cudaError_t launch_prefill_tc(const PrefillArgs& a);
+
+struct DecodeArgs {
+    const gqe_shape* s;
+    const void* q;
+    const void* K_cache;
+    const void* V_cache;
+    int Lmax;
+    const int32_t* lengths;
+    const int32_t* idx;
+    const float* gate;
+    void* O;
+    float* partials;  // workspace
+    void* status;
+    cudaStream_t stream;
+};
+int decode_chunk_tokens(const gqe_shape* s);
+size_t decode_partials_bytes(const gqe_shape* s, int Lmax);
+cudaError_t launch_decode(const DecodeArgs& a);
+
+}  // namespace gqe

@@ -1,0 +1,182 @@
+// gqe_api.cu -- extern "C" entry points of libgqe: argument validation on the
+// host, then kernel launches on the caller's stream.  See include/gqe.h.
+#include <cstring>
+
+#include "common.cuh"
+
+using namespace gqe;
+
+namespace {
+
+constexpr int kMaxK = 16;
+constexpr int kMaxH = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gqe_status check_shape(const gqe_shape* s) {
+    if (!s) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->B < 1 || s->T < 1 || s->h < 1 || s->g < 1 || s->d_h < 1 || s->k < 1 || s->d_model < 1)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (s->h % s->g != 0) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->k > s->h / s->g) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->dtype != GQE_F32 && s->dtype != GQE_BF16) return GQE_ERR_INVALID_ARGUMENT;
+    const int64_t rows = (int64_t)s->B * s->T * s->g * s->k;
+    if (rows >= ((int64_t)1 << 31)) return GQE_ERR_UNSUPPORTED;
+    if (s->k > kMaxK || s->h > kMaxH) return GQE_ERR_UNSUPPORTED;
+    return GQE_OK;
+}
+
+gqe_status check_workspace(void* ws, size_t bytes, size_t need) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return GQE_ERR_INVALID_ARGUMENT;
+    if (bytes < need) return GQE_ERR_INVALID_ARGUMENT;
+    return GQE_OK;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+size_t route_scratch_bytes(const gqe_shape* s) {
+    return align256((size_t)s->B * s->h * gqe_chunk_count(s->T) * sizeof(int32_t));
+}
+
+gqe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int gqe_chunk_count(int T) { return T <= 0 ? 0 : (T + kChunk - 1) / kChunk; }
+
+size_t gqe_workspace_bytes(const gqe_shape* s, int Lmax) {
+    if (check_shape(s) == GQE_ERR_INVALID_ARGUMENT || Lmax < 0) return 0;
+    size_t need = kStatusBytes + route_scratch_bytes(s);
+    if (Lmax > 0) {
+        const size_t dec = kStatusBytes + align256(decode_partials_bytes(s, Lmax));
+        if (dec > need) need = dec;
+    }
+    return need;
+}
+
+gqe_status gqe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != GQE_OK) return st;
+    return from_cuda(cudaMemsetAsync(workspace, 0, kStatusBytes, (cudaStream_t)stream));
+}
+
+gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                     int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                     int32_t* head_chunk_offsets, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!x || !W_r || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(W_r)) return GQE_ERR_INVALID_ARGUMENT;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + route_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    RouteArgs a;
+    a.s = s;
+    a.x = x;
+    a.W_r = W_r;
+    a.bias = bias;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_route(a));
+}
+
+gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                            const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                            const int32_t* head_pos, const int32_t* head_chunk_offsets, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!Q || !K || !V || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets || !O)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return GQE_ERR_INVALID_ARGUMENT;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != GQE_OK) return st;
+    PrefillArgs a;
+    a.s = s;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.O = O;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    if (s->dtype == GQE_BF16) {
+        if (s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+        return from_cuda(launch_prefill_tc(a));
+    }
+    if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+    if (s->h / s->g > 64) return GQE_ERR_UNSUPPORTED;
+    return from_cuda(launch_prefill_simt(a));
+}
+
+gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cache,
+                           const void* V_cache, int Lmax, const int32_t* lengths,
+                           const int32_t* idx, const float* gate, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (s->T != 1 || Lmax < 1) return GQE_ERR_INVALID_ARGUMENT;
+    if (!q || !K_cache || !V_cache || !lengths || !idx || !gate || !O) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O))
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+    if (s->k > 8) return GQE_ERR_UNSUPPORTED;
+    if ((int64_t)s->B * Lmax * s->g * s->d_h >= ((int64_t)1 << 40)) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + align256(decode_partials_bytes(s, Lmax)));
+    if (st != GQE_OK) return st;
+    DecodeArgs a;
+    a.s = s;
+    a.q = q;
+    a.K_cache = K_cache;
+    a.V_cache = V_cache;
+    a.Lmax = Lmax;
+    a.lengths = lengths;
+    a.idx = idx;
+    a.gate = gate;
+    a.O = O;
+    a.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_decode(a));
+}
+
+gqe_status gqe_get_device_status(void* workspace, void* stream) {
+    if (!workspace) return GQE_ERR_INVALID_ARGUMENT;
+    DeviceStatus host{};
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&host, workspace, sizeof host, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GQE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GQE_ERR_CUDA;
+    if (host.code != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof host, st) != cudaSuccess) return GQE_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return GQE_ERR_CUDA;
+        return (gqe_status)host.code;
+    }
+    return GQE_OK;
+}
+
+const char* gqe_status_string(gqe_status s) {
+    switch (s) {
+        case GQE_OK: return "GQE_OK";
+        case GQE_ERR_INVALID_ARGUMENT: return "GQE_ERR_INVALID_ARGUMENT";
+        case GQE_ERR_UNSUPPORTED: return "GQE_ERR_UNSUPPORTED";
+        case GQE_ERR_CUDA: return "GQE_ERR_CUDA";
+        case GQE_ERR_DEVICE_TIMEOUT: return "GQE_ERR_DEVICE_TIMEOUT";
+    }
+    return "GQE_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

@@ -1,0 +1,242 @@
+// router.cu -- GQE router (fp32 logits, per-group top-k, renormalised gates)
+// and token compaction (warp ballot + prefix sum), on CUDA cores.
+//
+// Router: "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention"
+// (gist.science summary), "Architecture et Routage": per token, k query-head
+// experts are selected in every GQA group; "Somme Ponderee Renormalisee": the
+// router probabilities are renormalised over the selected experts.  The linear
+// router x . W_r (+ bias) and the tie rule (lower head index first) are this
+// library's reading of an unspecified router.
+#include "common.cuh"
+
+namespace gqe {
+namespace {
+
+constexpr int kRouterThreads = 256;
+constexpr int kRouterTokPerThread = 4;
+constexpr int kRouterKC = 32;  // d_model chunk staged in shared memory
+
+// One block: kRouterTokPerThread * tokgroups tokens, all h heads.
+// Thread (tg, j): head j, tokens tg*4 .. tg*4+3 of the block.
+template <typename T>
+__global__ void __launch_bounds__(kRouterThreads)
+router_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ bias,
+              int64_t BT, int d_model, int h, int g, int k, int32_t* __restrict__ idx,
+              float* __restrict__ gate) {
+    extern __shared__ float smem[];
+    const int tokgroups = blockDim.x / h;
+    const int tok_per_block = tokgroups * kRouterTokPerThread;
+    float* xs = smem;                                   // [tok_per_block][kRouterKC + 1]
+    float* ws = xs + tok_per_block * (kRouterKC + 1);   // [kRouterKC][h]
+    float* lg = ws + kRouterKC * h;                     // [tok_per_block][h]
+
+    const int64_t tok0 = (int64_t)blockIdx.x * tok_per_block;
+    const int tid = threadIdx.x;
+    const int j = tid % h;
+    const int tg = tid / h;
+    const bool active = tg < tokgroups;
+
+    float acc[kRouterTokPerThread];
+#pragma unroll
+    for (int r = 0; r < kRouterTokPerThread; ++r) acc[r] = 0.f;
+
+    for (int c0 = 0; c0 < d_model; c0 += kRouterKC) {
+        const int kc = min(kRouterKC, d_model - c0);
+        for (int e = tid; e < tok_per_block * kRouterKC; e += blockDim.x) {
+            const int tt = e / kRouterKC, cc = e % kRouterKC;
+            const int64_t tok = tok0 + tt;
+            float v = 0.f;
+            if (tok < BT && cc < kc) v = Elem<T>::to_f(x[tok * d_model + c0 + cc]);
+            xs[tt * (kRouterKC + 1) + cc] = v;
+        }
+        for (int e = tid; e < kRouterKC * h; e += blockDim.x) {
+            const int cc = e / h, jj = e % h;
+            ws[e] = (cc < kc) ? Elem<T>::to_f(W[(int64_t)(c0 + cc) * h + jj]) : 0.f;
+        }
+        __syncthreads();
+        if (active) {
+            for (int cc = 0; cc < kc; ++cc) {
+                const float w = ws[cc * h + j];
+#pragma unroll
+                for (int r = 0; r < kRouterTokPerThread; ++r)
+                    acc[r] = fmaf(xs[(tg * kRouterTokPerThread + r) * (kRouterKC + 1) + cc], w, acc[r]);
+            }
+        }
+        __syncthreads();
+    }
+    if (active) {
+        const float bj = bias ? bias[j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < kRouterTokPerThread; ++r)
+            lg[(tg * kRouterTokPerThread + r) * h + j] = acc[r] + bj;
+    }
+    __syncthreads();
+
+    // Per (token, group): top-k by logit, ties to the lower head index; gates.
+    const int hpg = h / g;
+    for (int e = tid; e < tok_per_block * g; e += blockDim.x) {
+        const int tt = e / g, q = e % g;
+        const int64_t tok = tok0 + tt;
+        if (tok >= BT) continue;
+        const float* l = lg + tt * h + q * hpg;
+        int sel[16];
+        float sel_l[16];
+        float m = 0.f, denom = 0.f;
+        for (int s = 0; s < k; ++s) {
+            int best = -1;
+            float bv = 0.f;
+            for (int a = 0; a < hpg; ++a) {
+                bool taken = false;
+                for (int u = 0; u < s; ++u) taken |= (sel[u] == a);
+                if (taken) continue;
+                if (best < 0 || l[a] > bv) {  // strict: equal logits keep the lower index
+                    best = a;
+                    bv = l[a];
+                }
+            }
+            sel[s] = best;
+            sel_l[s] = bv;
+            if (s == 0) m = bv;
+            denom += expf(bv - m);
+        }
+        const int64_t o = (tok * g + q) * k;
+        for (int s = 0; s < k; ++s) {
+            idx[o + s] = q * hpg + sel[s];
+            gate[o + s] = expf(sel_l[s] - m) / denom;
+        }
+    }
+}
+
+// Compaction pass 1/3: per (b, chunk of 32 tokens, head) the number of tokens
+// routed to the head.  One warp per (b, chunk, group); lane = token.
+__global__ void compact_count_kernel(const int32_t* __restrict__ idx, int T, int h, int g, int k,
+                                     int nchunk, int32_t* __restrict__ counts) {
+    const int c = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int hpg = h / g;
+    const int t = c * kChunk + lane;
+    for (int q = warp; q < g; q += nwarps) {
+        int sel[16];
+        for (int s = 0; s < k; ++s) sel[s] = (t < T) ? idx[(((int64_t)b * T + t) * g + q) * k + s] : -1;
+        for (int jj = 0; jj < hpg; ++jj) {
+            const int j = q * hpg + jj;
+            bool hit = false;
+            for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
+            const unsigned ball = __ballot_sync(0xffffffffu, hit);
+            if (lane == 0) counts[((int64_t)b * h + j) * nchunk + c] = __popc(ball);
+        }
+    }
+}
+
+// Compaction pass 2/3: per batch, exclusive prefix sum over (head, chunk) in
+// head-major order -> absolute head_pos offsets.  One block per batch.
+__global__ void compact_scan_kernel(const int32_t* __restrict__ counts, int B, int T, int h, int g,
+                                    int k, int nchunk, int32_t* __restrict__ head_offsets,
+                                    int32_t* __restrict__ head_chunk_offsets) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    const int b = blockIdx.x;
+    const int n = h * nchunk;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t base = (int64_t)b * T * g * k;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+        const int i = i0 + threadIdx.x;
+        const int v = (i < n) ? counts[(int64_t)b * n + i] : 0;
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int nw = blockDim.x >> 5;
+            int ws = (lane < nw) ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, ws, d);
+                if (lane >= d) ws += y;
+            }
+            if (lane < nw) warp_sums[lane] = ws;  // inclusive over warps
+        }
+        __syncthreads();
+        const int warp_prefix = (warp > 0) ? warp_sums[warp - 1] : 0;
+        const int excl = carry + warp_prefix + incl - v;
+        if (i < n) {
+            const int32_t off = (int32_t)(base + excl);
+            head_chunk_offsets[(int64_t)b * n + i] = off;
+            if (i % nchunk == 0) head_offsets[(int64_t)b * h + i / nchunk] = off;
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = excl + v;
+        __syncthreads();
+    }
+    if (b == B - 1 && threadIdx.x == 0) head_offsets[(int64_t)B * h] = (int32_t)((int64_t)B * T * g * k);
+}
+
+// Compaction pass 3/3: write positions.  Same tiling as pass 1; a lane's rank
+// within its head's chunk is the popcount of the ballot below it.
+__global__ void compact_scatter_kernel(const int32_t* __restrict__ idx, int T, int h, int g, int k,
+                                       int nchunk, const int32_t* __restrict__ head_chunk_offsets,
+                                       int32_t* __restrict__ head_pos) {
+    const int c = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int hpg = h / g;
+    const int t = c * kChunk + lane;
+    const unsigned below = (1u << lane) - 1u;
+    for (int q = warp; q < g; q += nwarps) {
+        int sel[16];
+        for (int s = 0; s < k; ++s) sel[s] = (t < T) ? idx[(((int64_t)b * T + t) * g + q) * k + s] : -1;
+        for (int jj = 0; jj < hpg; ++jj) {
+            const int j = q * hpg + jj;
+            bool hit = false;
+            for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
+            const unsigned ball = __ballot_sync(0xffffffffu, hit);
+            if (hit) {
+                const int32_t off = head_chunk_offsets[((int64_t)b * h + j) * nchunk + c];
+                head_pos[off + __popc(ball & below)] = t;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteArgs& a) {
+    const gqe_shape& s = *a.s;
+    const int64_t BT = (int64_t)s.B * s.T;
+    const int tokgroups = kRouterThreads / s.h;
+    const int tok_per_block = tokgroups * kRouterTokPerThread;
+    const int threads = tokgroups * s.h;
+    const size_t smem = sizeof(float) * ((size_t)tok_per_block * (kRouterKC + 1) +
+                                         (size_t)kRouterKC * s.h + (size_t)tok_per_block * s.h);
+    const unsigned blocks = (unsigned)((BT + tok_per_block - 1) / tok_per_block);
+    if (s.dtype == GQE_BF16) {
+        auto kern = router_kernel<__nv_bfloat16>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<blocks, threads, smem, a.stream>>>((const __nv_bfloat16*)a.x, (const __nv_bfloat16*)a.W_r,
+                                                  a.bias, BT, s.d_model, s.h, s.g, s.k, a.idx, a.gate);
+    } else {
+        auto kern = router_kernel<float>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<blocks, threads, smem, a.stream>>>((const float*)a.x, (const float*)a.W_r, a.bias, BT,
+                                                  s.d_model, s.h, s.g, s.k, a.idx, a.gate);
+    }
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+
+    const int nchunk = gqe_chunk_count(s.T);
+    const int cwarps = s.g < 8 ? s.g : 8;
+    dim3 cgrid(nchunk, s.B);
+    compact_count_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk, a.counts);
+    compact_scan_kernel<<<s.B, 1024, 0, a.stream>>>(a.counts, s.B, s.T, s.h, s.g, s.k, nchunk,
+                                                   a.head_offsets, a.head_chunk_offsets);
+    compact_scatter_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk,
+                                                                a.head_chunk_offsets, a.head_pos);
+    return cudaGetLastError();
+}
+
+}  // namespace gqe

@@ -1,0 +1,127 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/gqe.h declares; host-side validation rejects bad arguments before any
+CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from routed_head_gqa_b200 import build as gqe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = gqe_build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for required in ("gqe_route", "gqe_attn_prefill", "gqe_attn_decode"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in gqe.h but not exported"
+
+
+def test_binding_names_match_header():
+    import routed_head_gqa_b200 as g
+
+    for name in declared_functions():
+        assert callable(getattr(g, name)), f"binding lacks {name}"
+    assert sorted(g.EXPORTED) == declared_functions()
+
+
+def test_status_strings_and_chunks():
+    import routed_head_gqa_b200 as g
+
+    assert g.gqe_status_string(g.GQE_OK) == "GQE_OK"
+    assert g.gqe_status_string(g.GQE_ERR_DEVICE_TIMEOUT) == "GQE_ERR_DEVICE_TIMEOUT"
+    assert g.gqe_status_string(99) == "GQE_UNKNOWN_STATUS"
+    assert [g.gqe_chunk_count(t) for t in (0, 1, 32, 33, 4096)] == [0, 1, 1, 2, 128]
+
+
+def test_workspace_bytes():
+    import routed_head_gqa_b200 as g
+
+    s = g.make_shape(8, 4096, 4096, 32, 8, 128, 2, g.GQE_BF16)
+    n = g.gqe_workspace_bytes(s, 0)
+    assert n >= 256 + 8 * 32 * 128 * 4
+    assert g.gqe_workspace_bytes(s, 16384) >= n
+    bad = g.make_shape(8, 4096, 4096, 30, 8, 128, 2, g.GQE_BF16)  # h % g != 0
+    assert g.gqe_workspace_bytes(bad, 0) == 0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("h", 30, 1),       # h % g != 0
+    ("k", 5, 1),        # k > h/g
+    ("k", 0, 1),
+    ("T", 0, 1),
+    ("dtype", 7, 1),
+])
+def test_route_rejects_bad_shapes(field, value, code):
+    import routed_head_gqa_b200 as g
+
+    s = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_BF16)
+    setattr(s, field, value)
+    fake = 0x10000  # never dereferenced: validation fails first
+    rc = g._lib.gqe_route(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake, 1 << 20, None)
+    assert rc == code
+
+
+def test_null_and_misaligned_pointers_rejected():
+    import routed_head_gqa_b200 as g
+
+    s = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_BF16)
+    fake = 0x10000
+    assert g._lib.gqe_route(ctypes.byref(s), None, fake, None, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 1
+    assert g._lib.gqe_route(ctypes.byref(s), fake + 2, fake, None, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 1
+    # workspace too small / misaligned
+    assert g._lib.gqe_route(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake, 16, None) == 1
+    assert g._lib.gqe_route(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake + 16, 1 << 20, None) == 1
+    assert g._lib.gqe_attn_prefill(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                   1 << 20, None) == 1
+    # decode requires T == 1 and Lmax >= 1
+    assert g._lib.gqe_attn_decode(ctypes.byref(s), fake, fake, fake, 128, fake, fake, fake, fake, fake,
+                                  1 << 30, None) == 1
+    s1 = g.make_shape(2, 1, 128, 32, 8, 128, 2, g.GQE_BF16)
+    assert g._lib.gqe_attn_decode(ctypes.byref(s1), fake, fake, fake, 0, fake, fake, fake, fake, fake,
+                                  1 << 30, None) == 1
+
+
+def test_unsupported_cases_report_unsupported():
+    import routed_head_gqa_b200 as g
+
+    fake = 0x10000
+    # bf16 prefill is implemented for d_h = 128 only
+    s = g.make_shape(2, 64, 128, 8, 2, 64, 2, g.GQE_BF16)
+    assert g._lib.gqe_attn_prefill(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                                   1 << 20, None) == 2
+    # decode: d_h 96 not implemented
+    s = g.make_shape(2, 1, 128, 8, 2, 96, 2, g.GQE_BF16)
+    assert g._lib.gqe_attn_decode(ctypes.byref(s), fake, fake, fake, 64, fake, fake, fake, fake, fake,
+                                  1 << 30, None) == 2
+
+
+def test_kv_cache_ratio_golden():
+    """The decode byte accounting reproduces the pages' KV-cache reduction
+    (32 query heads over 8 KV groups -> 4x smaller cache than MHA)."""
+    from routed_head_gqa_b200 import metrics
+    from tests.oracle_pins import read_golden
+
+    h, g_, ratio = read_golden("kv_cache_ratio.txt")[0]
+    mha = metrics.kv_cache_bytes(n_kv=h, d_h=128, T=4096)
+    gqa = metrics.kv_cache_bytes(n_kv=g_, d_h=128, T=4096)
+    assert mha == ratio * gqa
