@@ -72,47 +72,56 @@ int oracle_route(int64_t BT, int d_model, int h, int g, int k, int dtype,
     if (BT < 0 || d_model < 1 || h < 1 || g < 1 || h % g != 0) return 1;
     const int hpg = h / g;
     if (k < 1 || k > hpg) return 1;
-    int* order = (int*)malloc(sizeof(int) * (size_t)hpg);
-    if (!order) return 2;
-    for (int64_t r = 0; r < BT; ++r) {
-        for (int j = 0; j < h; ++j) {
-            double acc = 0.0;
-            for (int i = 0; i < d_model; ++i)
-                acc += load_elem(x, (size_t)r * d_model + i, dtype) *
-                       load_elem(W_r, (size_t)i * h + j, dtype);
-            if (bias) acc += (double)bias[j];
-            logits[(size_t)r * h + j] = (float)acc;
-        }
-        for (int q = 0; q < g; ++q) {
-            const float* lg = logits + (size_t)r * h + (size_t)q * hpg;
-            /* insertion sort of the group's heads by (logit desc, index asc) */
-            for (int a = 0; a < hpg; ++a) {
-                int pos = a;
-                while (pos > 0) {
-                    int prev = order[pos - 1];
-                    if (lg[prev] < lg[a]) {
-                        order[pos] = prev;
-                        --pos;
-                    } else {
-                        break;
-                    }
+    int err = 0;
+#pragma omp parallel
+    {
+        int* order = (int*)malloc(sizeof(int) * (size_t)hpg);
+        if (!order) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t r = 0; r < BT; ++r) {
+                for (int j = 0; j < h; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < d_model; ++i)
+                        acc += load_elem(x, (size_t)r * d_model + i, dtype) *
+                               load_elem(W_r, (size_t)i * h + j, dtype);
+                    if (bias) acc += (double)bias[j];
+                    logits[(size_t)r * h + j] = (float)acc;
                 }
-                order[pos] = a;
+                for (int q = 0; q < g; ++q) {
+                    const float* lg = logits + (size_t)r * h + (size_t)q * hpg;
+                    /* insertion sort of the group's heads by (logit desc, index asc) */
+                    for (int a = 0; a < hpg; ++a) {
+                        int pos = a;
+                        while (pos > 0) {
+                            int prev = order[pos - 1];
+                            if (lg[prev] < lg[a]) {
+                                order[pos] = prev;
+                                --pos;
+                            } else {
+                                break;
+                            }
+                        }
+                        order[pos] = a;
+                    }
+                    const double m = (double)lg[order[0]];
+                    double denom = 0.0;
+                    for (int s = 0; s < k; ++s) denom += exp((double)lg[order[s]] - m);
+                    for (int s = 0; s < k; ++s) {
+                        size_t o = ((size_t)r * g + q) * k + s;
+                        idx[o] = q * hpg + order[s];
+                        gate[o] = exp((double)lg[order[s]] - m) / denom;
+                    }
+                    margin[(size_t)r * g + q] =
+                        (k == hpg) ? INFINITY : (double)lg[order[k - 1]] - (double)lg[order[k]];
+                }
             }
-            const double m = (double)lg[order[0]];
-            double denom = 0.0;
-            for (int s = 0; s < k; ++s) denom += exp((double)lg[order[s]] - m);
-            for (int s = 0; s < k; ++s) {
-                size_t o = ((size_t)r * g + q) * k + s;
-                idx[o] = q * hpg + order[s];
-                gate[o] = exp((double)lg[order[s]] - m) / denom;
-            }
-            margin[(size_t)r * g + q] =
-                (k == hpg) ? INFINITY : (double)lg[order[k - 1]] - (double)lg[order[k]];
         }
+        free(order);
     }
-    free(order);
-    return 0;
+    return err;
 }
 
 /* ------------------------------------------------------------------------ */
