@@ -1,0 +1,492 @@
+"""Benchmark of the GQE attention forward pass on B200 (routed prefill and decode).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl gqe|reference]
+
+A step is one pass of the whole routed path over one batch of seeded synthetic
+input, with inputs resident in HBM:
+  prefill workloads: gqe_route (router, per-group top-k, compaction) +
+                     gqe_attn_prefill (routed causal attention + gated scatter)
+  decode workload:   gqe_route on the new tokens + gqe_attn_decode
+Metric: active-head TFLOP/s for prefill (4*d_h*(t+1) per routed row), KV-cache
+GB/s for decode (2*g*d_h*L_b bf16 elements per sequence).  The L2 is flushed
+(256 MB memset) before every timed step, outside the step's CUDA events.
+
+With N > 1 (torchrun) every rank runs an independent replica on its own batch
+(the path has no exchange step); value = all ranks' work / the slowest rank's time.
+``--impl reference`` times the CPU oracle instead, on bounded samples of the
+same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gqe_synth  # noqa: E402
+
+PRIMARY = "dense_gqa"
+SECONDARY = ["gqe_prefill", "gqe_long", "gqe_decode"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernels, from `ncu` captures
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source they were taken on (sha256 of the listed files).  See profiles/.
+NCU_TRAFFIC = {
+    ("prefill_tc_kernel", "dense_gqa"): {
+        "sha": "5f91ce8539ca033d", "bytes_per_launch": 104152576 + 31594496,
+        "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
+}
+
+
+def kernel_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "routed_head_gqa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_FILES = {
+    "prefill_tc_kernel": ["prefill_tc.cu", "sm100.cuh", "units.cuh", "common.cuh"],
+    "decode_partial_kernel": ["decode.cu", "common.cuh"],
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        mhz, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only: barrier and max of the step times)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def workload_for_rank(w, rank):
+    if rank == 0:
+        return w
+    import dataclasses
+
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+class Runner:
+    """Holds one workload's device inputs and buffers; runs steps."""
+
+    def __init__(self, w, dev):
+        import routed_head_gqa_b200 as g
+
+        self.g = g
+        self.w = w
+        self.inp = gqe_synth.make_inputs(w)
+        self.dev = dev
+        self.d = {k: (v.to(dev) if v is not None else None) for k, v in self.inp.items()}
+        T = 1 if w.decode else w.T
+        self.shape = g.make_shape(w.B, T, w.d_model, w.h, w.g, w.d_h, w.k, w.torch_dtype)
+        self.buf = g.Buffers(self.shape, dev, Lmax=w.Lmax if w.decode else 0)
+        self.stream = torch.cuda.current_stream()
+
+    def route(self):
+        self.buf.route(self.d["x"], self.d["W_r"], self.d["bias"])
+
+    def attend(self):
+        if self.w.decode:
+            self.buf.decode(self.d["q"], self.d["K_cache"], self.d["V_cache"], self.d["lengths"])
+        else:
+            self.buf.prefill(self.d["Q"], self.d["K"], self.d["V"])
+
+    def step(self):
+        self.route()
+        self.attend()
+
+    def launches_per_step(self):
+        route = 4  # router + compaction count / scan / scatter
+        return route + (2 if self.w.decode else 1)
+
+    def work(self):
+        """(work units per step, unit string, scale to the unit)."""
+        from routed_head_gqa_b200 import metrics
+
+        w = self.w
+        if w.decode:
+            return float(metrics.decode_kv_bytes(self.inp["lengths"], w.g, w.d_h, 2)), "GB/s", 1e-9
+        flops = metrics.prefill_active_flops(w.B, w.T, w.g, w.k, w.d_h)
+        return float(flops), "TFLOP/s", 1e-12
+
+
+def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, with_e2e):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    r = Runner(workload_for_rank(w, rank), dev)
+    work, unit, scale = r.work()
+    if not w.decode:
+        from routed_head_gqa_b200 import metrics
+
+        r.step()
+        torch.cuda.synchronize()
+        assert metrics.prefill_active_flops_from_routing(r.buf.idx, w.d_h) == int(work)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        flush.zero_()
+        r.step()
+    torch.cuda.synchronize()
+    st = r.buf.status()
+    if st != 0:
+        raise RuntimeError(f"device status {r.g.gqe_status_string(st)} during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(dev.index) if with_clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record()
+        r.route()
+        e1.record()
+        r.attend()
+        e2.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop() if sampler else None
+    st = r.buf.status()
+    if st != 0:
+        raise RuntimeError(f"device status {r.g.gqe_status_string(st)} in the timed region")
+    step_ms = sum(a.elapsed_time(c) for a, _, c in ev)
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    route_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    step_ms_max = max_over_ranks(step_ms, ws)
+    value = work * ws * steps / (step_ms_max * 1e-3) * scale
+
+    kern = "decode_partial_kernel" if w.decode else "prefill_tc_kernel"
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    if w.decode:
+        achieved = work / (attn_avg_ms * 1e-3) * 1e-9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"hbm_gbs ({peak_kind})",
+                "kernel": "gqe_attn_decode (decode_partial_kernel + decode_combine_kernel)"}
+    else:
+        achieved = work / (attn_avg_ms * 1e-3) * 1e-12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"bf16_tflops burst ({peak_kind})",
+                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "kernel": "gqe_attn_prefill (prefill_tc_kernel)"}
+    tr = NCU_TRAFFIC.get((kern, w.name))
+    roof["traffic"] = None
+    if tr and tr["sha"] == kernel_sha(KERNEL_FILES[kern]):
+        roof["traffic"] = tr["bytes_per_launch"]
+        roof["traffic_note"] = tr["note"]
+    roof["algorithmic_per_launch"] = work
+    res = {
+        "value": value, "unit": unit, "ms_per_step": step_ms_max / steps,
+        "attn_ms": attn_avg_ms, "route_ms": sum(route_ms) / len(route_ms),
+        "roofline": roof, "clocks": clocks, "gpu_launches": r.launches_per_step() * steps,
+    }
+    if with_e2e:
+        res["e2e"] = time_e2e(r, steps, ws, work, scale, unit)
+    del r, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_e2e(r, steps, ws, work, scale, unit):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device and the output back."""
+    w = r.w
+    names = ["x", "q"] if w.decode else ["x", "Q", "K", "V"]
+    host = {n: r.inp[n].pin_memory() for n in names}
+    dev_in = {n: torch.empty_like(r.d[n]) for n in names}
+    out_host = torch.empty(r.buf.O.shape, dtype=r.buf.O.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        for n in names:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        r.buf.route(dev_in["x"], r.d["W_r"], r.d["bias"])
+        if w.decode:
+            r.buf.decode(dev_in["q"], r.d["K_cache"], r.d["V_cache"], r.d["lengths"])
+        else:
+            r.buf.prefill(dev_in["Q"], dev_in["K"], dev_in["V"])
+        out_host.copy_(r.buf.O, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    return {"value": work * ws * steps / (ms * 1e-3) * scale, "unit": unit, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "note": ("KV caches stay resident (decoder state); per step: x and q in, "
+                                                "O out") if w.decode else "per step: x, Q, K, V in; O out"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, inp, n_rows, seed):
+    """Run the oracle on a sample of n_rows token rows of the workload.  Returns
+    (work done in the metric's units, seconds, sample description)."""
+    import numpy as np
+
+    import oracle
+
+    if w.decode:
+        gen = torch.Generator().manual_seed(seed)
+        bs = torch.randperm(w.B, generator=gen)[: max(1, min(w.B, n_rows))].sort().values
+        t0 = time.perf_counter()
+        idx, gate, _, _ = oracle.route(inp["x"][bs], inp["W_r"], w.h, w.g, w.k, bias=inp["bias"])
+        oracle.decode(inp["q"][bs], inp["K_cache"][bs], inp["V_cache"][bs], inp["lengths"][bs], idx, gate)
+        dt = time.perf_counter() - t0
+        work = float(inp["lengths"][bs].to(torch.int64).sum().item()) * 2 * w.g * w.d_h * 2
+        return work, dt, f"{len(bs)} of {w.B} sequences (full cache each)"
+    rows = gqe_synth.sample_rows(w, n_rows, seed=seed).numpy()
+    t0 = time.perf_counter()
+    xr = inp["x"].reshape(w.B * w.T, w.d_model)[torch.from_numpy(rows)]
+    idx_s, gate_s, _, _ = oracle.route(xr, inp["W_r"], w.h, w.g, w.k, bias=inp["bias"])
+    idx = np.zeros((w.B * w.T, w.g, w.k), np.int32)
+    gate = np.zeros((w.B * w.T, w.g, w.k), np.float64)
+    # rows outside the sample keep a valid placeholder routing (never computed)
+    idx[:] = (np.arange(w.g)[:, None] * w.hpg + np.arange(w.k)[None, :])[None]
+    idx[rows] = idx_s
+    gate[rows] = gate_s
+    oracle.attn_rows(inp["Q"], inp["K"], inp["V"], idx.reshape(w.B, w.T, w.g, w.k),
+                     gate.reshape(w.B, w.T, w.g, w.k), rows=rows)
+    dt = time.perf_counter() - t0
+    t = rows % w.T
+    work = float(4 * w.d_h * w.g * w.k * (t + 1).sum())
+    return work, dt, f"{len(rows)} of {w.B * w.T} token rows (route + all routed heads)"
+
+
+def cpu_baseline(w, inp, target_s):
+    """Calibrate a sample to about target_s seconds of oracle work, time it."""
+    n = 8 if w.decode else 64
+    work, dt, _ = oracle_sample(w, inp, n, 7)
+    total = w.B if w.decode else w.B * w.T
+    per = dt / n
+    n2 = int(min(total, max(n, target_s / max(per, 1e-9))))
+    work, dt, desc = oracle_sample(w, inp, n2, 8)
+    scale = 1e-9 if w.decode else 1e-12
+    unit = "GB/s" if w.decode else "TFLOP/s"
+    return {"value": work / dt * scale, "unit": unit, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": desc, "seconds": round(dt, 2)}
+
+
+def run_reference(w, steps, warmup):
+    inp = gqe_synth.make_inputs(w)
+    # size each step to ~2 s of oracle work so K+W steps end within minutes
+    n = 8 if w.decode else 64
+    work, dt, _ = oracle_sample(w, inp, n, 1)
+    total = w.B if w.decode else w.B * w.T
+    n_step = int(min(total, max(1, 2.0 / max(dt / n, 1e-9))))
+    for i in range(warmup):
+        oracle_sample(w, inp, max(1, n_step // 8), 100 + i)
+    tot_work, tot_s, desc = 0.0, 0.0, ""
+    for i in range(steps):
+        wk, s, desc = oracle_sample(w, inp, n_step, 200 + i)
+        tot_work += wk
+        tot_s += s
+    scale = 1e-9 if w.decode else 1e-12
+    unit = "GB/s" if w.decode else "TFLOP/s"
+    value = tot_work / tot_s * scale
+    return value, unit, tot_s, desc
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=PRIMARY, choices=sorted(gqe_synth.WORKLOADS))
+    ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = gqe_synth.WORKLOADS[args.workload]
+    metric = "routed GQE attn TFLOP/s (prefill), KV-read GB/s (decode), % of B200 roofline"
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        value, unit, secs, desc = run_reference(w, args.steps, args.warmup)
+        line = {"metric": metric, "impl": "reference", "value": value, "unit": unit, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded, gqe_synth recipe)",
+                "config": {"workload": w.name, "shape": w.describe()},
+                "cpu_baseline": {"value": value, "unit": unit, "cores": os.cpu_count(), "kind": "oracle",
+                                 "sample": desc + " per step"},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    ws, rank, local = dist_setup()
+    from routed_head_gqa_b200 import build as gqe_build
+
+    if rank == 0:
+        gqe_build.build()
+    barrier(ws)
+    peaks, peak_kind = load_peaks()
+    res = time_workload(w, args.steps, args.warmup, ws, rank, peaks, peak_kind, with_clocks=(rank == 0),
+                        with_e2e=True)
+    secondary = {}
+    if not args.no_secondary and args.workload == PRIMARY:
+        for name in SECONDARY:
+            sw = gqe_synth.WORKLOADS[name]
+            r2 = time_workload(sw, max(5, args.steps // 2), 3, ws, rank, peaks, peak_kind, with_clocks=False,
+                               with_e2e=False)
+            secondary[name] = {"value": r2["value"], "unit": r2["unit"], "ms_per_step": r2["ms_per_step"],
+                               "attn_ms": r2["attn_ms"], "route_ms": r2["route_ms"], "roofline": r2["roofline"],
+                               "shape": sw.describe()}
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": metric, "value": res["value"], "unit": res["unit"], "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded, gqe_synth recipe)",
+            "config": {"workload": w.name, "shape": w.describe(), "per_gpu_batch": w.B,
+                       "global_batch": w.B * ws, "parallelism": f"replicas x{ws} (no exchange step)",
+                       "l2": "flushed (256 MB memset) before every timed step, outside the step events",
+                       "attn_ms": res["attn_ms"], "route_ms": res["route_ms"]},
+            "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"],
+            "gpu_launches": res["gpu_launches"],
+        }
+        if secondary:
+            line["workloads"] = secondary
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
