@@ -3,8 +3,9 @@
 Argument marshalling only.  Every step of the routed path (router, top-k,
 compaction, routed prefill, decode) runs in the library's CUDA kernels; PyTorch
 supplies device memory and the current CUDA stream.  The functions keep the C
-names and raise ``GQEError`` on a non-OK status.  Importing this package fails
-if ``libgqe.so`` has not been built (``python -m routed_head_gqa_b200.build``).
+names and raise ``GQEError`` on a non-OK status.  The first call loads
+``libgqe.so`` and raises ImportError if it has not been built
+(``python -m routed_head_gqa_b200.build``); there is no fallback.
 """
 from __future__ import annotations
 
@@ -16,11 +17,6 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgqe.so")
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m routed_head_gqa_b200.build`")
-
-_lib = ctypes.CDLL(LIB_PATH)
-
 GQE_OK = 0
 GQE_ERR_INVALID_ARGUMENT = 1
 GQE_ERR_UNSUPPORTED = 2
@@ -29,7 +25,7 @@ GQE_ERR_DEVICE_TIMEOUT = 4
 GQE_F32 = 0
 GQE_BF16 = 1
 
-EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route",
+EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route",,
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -47,19 +43,42 @@ class GQEError(RuntimeError):
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
-_lib.gqe_chunk_count.argtypes = [_I]
-_lib.gqe_chunk_count.restype = _I
-_lib.gqe_workspace_bytes.argtypes = [ctypes.POINTER(GqeShape), _I]
-_lib.gqe_workspace_bytes.restype = _SZ
-_lib.gqe_workspace_init.argtypes = [_P, _SZ, _P]
-_lib.gqe_route.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
-_lib.gqe_attn_prefill.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
-_lib.gqe_attn_decode.argtypes = [ctypes.POINTER(GqeShape), _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
-_lib.gqe_get_device_status.argtypes = [_P, _P]
-_lib.gqe_status_string.argtypes = [_I]
-_lib.gqe_status_string.restype = ctypes.c_char_p
-for _f in ("gqe_workspace_init", "gqe_route", "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status"):
-    getattr(_lib, _f).restype = _I
+_lib_handle = None
+
+
+def _load():
+    """Load libgqe.so on first use; fail loudly when it has not been built."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m routed_head_gqa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    S = ctypes.POINTER(GqeShape)
+    lib.gqe_chunk_count.argtypes = [_I]
+    lib.gqe_chunk_count.restype = _I
+    lib.gqe_workspace_bytes.argtypes = [S, _I]
+    lib.gqe_workspace_bytes.restype = _SZ
+    lib.gqe_workspace_init.argtypes = [_P, _SZ, _P]
+    lib.gqe_route.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_prefill.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_get_device_status.argtypes = [_P, _P]
+    lib.gqe_status_string.argtypes = [_I]
+    lib.gqe_status_string.restype = ctypes.c_char_p
+    for f in ("gqe_workspace_init", "gqe_route", "gqe_attn_prefill", "gqe_attn_decode",
+              "gqe_get_device_status"):
+        getattr(lib, f).restype = _I
+    _lib_handle = lib
+    return lib
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(_load(), name)
+
+
+_lib = _LazyLib()
 
 
 def make_shape(B, T, d_model, h, g, d_h, k, dtype) -> GqeShape:
