@@ -53,7 +53,8 @@ typedef enum {
     GQE_ERR_INVALID_ARGUMENT = 1,
     GQE_ERR_UNSUPPORTED = 2,
     GQE_ERR_CUDA = 3,
-    GQE_ERR_DEVICE_TIMEOUT = 4
+    GQE_ERR_DEVICE_TIMEOUT = 4,
+    GQE_ERR_SCRATCH_LIMIT = 5
 } gqe_status;
 
 typedef enum { GQE_F32 = 0, GQE_BF16 = 1 } gqe_dtype;
@@ -109,6 +110,33 @@ gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const f
                      int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
                      int32_t* head_chunk_offsets, void* workspace, size_t workspace_bytes,
                      void* stream);
+
+/*
+ * gqe_route_static -- gqe_route without a workspace argument: it allocates
+ * nothing and takes no scratch from the caller.  The paper has no counterpart
+ * for this entry point; it exists for callers that cannot allocate device
+ * memory, such as a serving runtime whose memory is planned up front and
+ * handed out by its own arena, code that may not call cudaMalloc or an
+ * allocating library (PyTorch's caching allocator included) at the point of
+ * the call, or a host that only passes pointers it already owns.
+ *
+ * Inputs, outputs and results are exactly those of gqe_route.  The per-chunk
+ * counts that gqe_route keeps in its workspace live instead in one 4 MiB
+ * array of device memory owned by this library (every GPU that loads the
+ * library holds its own copy until the process exits), so
+ * B * h * gqe_chunk_count(T) must not exceed 1,048,576; larger shapes return
+ * GQE_ERR_SCRATCH_LIMIT and enqueue nothing.
+ * The first call on a device looks up that device's copy of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call before
+ * any stream capture.  Every call shares the array and it keeps the last
+ * call's contents (each call writes every count before reading it, so nothing
+ * needs clearing): calls whose kernels may overlap on the GPU (different
+ * streams, or concurrent host threads on one device) race on it and must be
+ * serialised by the caller.
+ */
+gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                            int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                            int32_t* head_chunk_offsets, void* stream);
 
 /*
  * gqe_attn_prefill -- routed causal attention with the gated scatter.

@@ -22,10 +22,11 @@ GQE_ERR_INVALID_ARGUMENT = 1
 GQE_ERR_UNSUPPORTED = 2
 GQE_ERR_CUDA = 3
 GQE_ERR_DEVICE_TIMEOUT = 4
+GQE_ERR_SCRATCH_LIMIT = 5
 GQE_F32 = 0
 GQE_BF16 = 1
 
-EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route",,
+EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -61,12 +62,13 @@ def _load():
     lib.gqe_workspace_bytes.restype = _SZ
     lib.gqe_workspace_init.argtypes = [_P, _SZ, _P]
     lib.gqe_route.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_route_static.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.gqe_attn_prefill.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
-    for f in ("gqe_workspace_init", "gqe_route", "gqe_attn_prefill", "gqe_attn_decode",
+    for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
@@ -135,6 +137,16 @@ def gqe_route(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, head_chunk
                                        _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
                                        _ptr(head_chunk_offsets), _ptr(workspace), _nbytes(workspace),
                                        _stream(stream)))
+
+
+def gqe_route_static(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, head_chunk_offsets,
+                     stream=None) -> None:
+    """gqe_route with the library's own scratch: no workspace, no allocation.
+    For callers that cannot allocate device memory; see include/gqe.h for the
+    size limit and the rule that overlapping calls race on the shared scratch."""
+    _check("gqe_route_static", _lib.gqe_route_static(ctypes.byref(shape), _ptr(x), _ptr(W_r), _ptr(bias),
+                                                     _ptr(idx), _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
+                                                     _ptr(head_chunk_offsets), _stream(stream)))
 
 
 def gqe_attn_prefill(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, O, workspace,

@@ -101,6 +101,12 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a);
 
+// Library-held scratch for gqe_route_static: per-(b, head, chunk) counts,
+// at most kRouteStaticScratchBytes.  Resolves the calling thread's current
+// device's copy of the array (once per device) into *out.
+constexpr size_t kRouteStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+cudaError_t route_static_scratch(int32_t** out);
+
 struct PrefillArgs {
     const gqe_shape* s;
     const void* Q;

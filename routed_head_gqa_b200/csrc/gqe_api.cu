@@ -89,6 +89,34 @@ gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const f
     return from_cuda(launch_route(a));
 }
 
+gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                            int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                            int32_t* head_chunk_offsets, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!x || !W_r || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(W_r)) return GQE_ERR_INVALID_ARGUMENT;
+    const size_t need = (size_t)s->B * s->h * gqe_chunk_count(s->T) * sizeof(int32_t);
+    if (need > kRouteStaticScratchBytes) return GQE_ERR_SCRATCH_LIMIT;
+    int32_t* scratch = nullptr;
+    if (route_static_scratch(&scratch) != cudaSuccess) return GQE_ERR_CUDA;
+    RouteArgs a;
+    a.s = s;
+    a.x = x;
+    a.W_r = W_r;
+    a.bias = bias;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.counts = scratch;  // every count is written before it is read: nothing to clear
+    a.status = nullptr;  // the route kernels report nothing through the status word
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_route(a));
+}
+
 gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, const void* V,
                             const int32_t* idx, const float* gate, const int32_t* head_offsets,
                             const int32_t* head_pos, const int32_t* head_chunk_offsets, void* O,
@@ -175,6 +203,7 @@ const char* gqe_status_string(gqe_status s) {
         case GQE_ERR_UNSUPPORTED: return "GQE_ERR_UNSUPPORTED";
         case GQE_ERR_CUDA: return "GQE_ERR_CUDA";
         case GQE_ERR_DEVICE_TIMEOUT: return "GQE_ERR_DEVICE_TIMEOUT";
+        case GQE_ERR_SCRATCH_LIMIT: return "GQE_ERR_SCRATCH_LIMIT";
     }
     return "GQE_UNKNOWN_STATUS";
 }

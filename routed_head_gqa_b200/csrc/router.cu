@@ -240,3 +240,37 @@ cudaError_t launch_route(const RouteArgs& a) {
 }
 
 }  // namespace gqe
+
+// ---------------------------------------------------------------------------
+// Scratch owned by the library, for callers that cannot allocate device memory
+// (gqe_route_static).  Every device that loads this library holds one copy of
+// the array until the process exits.  In host code the array's name is only a
+// host-side stand-in: the device address of this device's copy comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+static __device__ __align__(256) int32_t g_route_static_scratch[gqe::kRouteStaticScratchBytes / sizeof(int32_t)];
+
+namespace gqe {
+
+cudaError_t route_static_scratch(int32_t** out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int32_t* addr[kMaxDevices] = {};
+    int dev = -1;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_route_static_scratch);
+        if (err != cudaSuccess) return err;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace gqe
