@@ -100,6 +100,8 @@ struct RouteArgs {
     cudaStream_t stream;
 };
 cudaError_t launch_route(const RouteArgs& a);
+bool router_tc_supported(const gqe_shape* s);
+cudaError_t launch_router_tc(const RouteArgs& a);  // a1+a2 on tensor cores (bf16)
 
 // Library-held scratch for gqe_route_static: per-(b, head, chunk) counts,
 // at most kRouteStaticScratchBytes.  Resolves the calling thread's current

@@ -1,5 +1,7 @@
 // router.cu -- GQE router (fp32 logits, per-group top-k, renormalised gates)
-// and token compaction (warp ballot + prefix sum), on CUDA cores.
+// on CUDA cores for the inputs the tensor-core router (router_tc.cu) does not
+// take (fp32, or h not a multiple of 8), and token compaction (warp ballot +
+// prefix sum).
 //
 // Router: "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention"
 // (gist.science summary), "Architecture et Routage": per token, k query-head
@@ -214,7 +216,10 @@ cudaError_t launch_route(const RouteArgs& a) {
     const size_t smem = sizeof(float) * ((size_t)tok_per_block * (kRouterKC + 1) +
                                          (size_t)kRouterKC * s.h + (size_t)tok_per_block * s.h);
     const unsigned blocks = (unsigned)((BT + tok_per_block - 1) / tok_per_block);
-    if (s.dtype == GQE_BF16) {
+    if (router_tc_supported(a.s)) {
+        cudaError_t e = launch_router_tc(a);
+        if (e != cudaSuccess) return e;
+    } else if (s.dtype == GQE_BF16) {
         auto kern = router_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<blocks, threads, smem, a.stream>>>((const __nv_bfloat16*)a.x, (const __nv_bfloat16*)a.W_r,
