@@ -7,18 +7,25 @@
 //   O[b,t,j,:] = gate * sum_{s<=t} softmax_s(Q[b,t,j] . K[b,s,j/hpg] / sqrt(128)) V[b,s,j/hpg]
 // and O[b,t,j,:] = 0 for the unselected (t, j).
 //
-// Work unit: (b, KV group q, window of W = 128/k.. positions), whose k*W routed
-// rows (from the per-head packed position lists) form one M=128 tile.  Each
-// K/V tile of group q is loaded once per unit by TMA and used by every routed
-// head of the group in that window.
+// Work unit: (b, KV group q, window of W = 32*floor(4/k) positions).  Every
+// token selects exactly k heads per group, so the window holds k*W <= 128 routed
+// rows (taken from the per-head packed position lists): one M=128 Q tile.  Each
+// K/V tile of the group is loaded once per unit by TMA and serves every routed
+// head of the group in the window.
 //
-// Roles (256 threads, one persistent CTA per SM):
+// Roles (384 threads, one persistent CTA per SM):
 //   warp 0      TMA producer for K/V tiles; owns the TMEM allocation
-//   warp 1      MMA issuer (one thread): S = Q K^T and O += P V on tcgen05
-//   warp 2      row table and Q gather (cp.async, 128B-swizzled)
+//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered S and
+//               O += P V, both on tcgen05
+//   warp 2      row tables, L2 prefetch and Q gather (TMA tile::gather4,
+//               128B-swizzled) into a double-buffered Q tile
 //   warp 3      zero fill of the window's unselected output slots
-//   warps 4-7   softmax (one row per thread, S read from TMEM, P written back
-//               to TMEM as bf16) and the gated epilogue
+//   warps 4-7   softmax + epilogue, key columns 0-63 of every row
+//   warps 8-11  softmax + epilogue, key columns 64-127 of every row
+// The two softmax warpgroups share each row: they exchange their partial row
+// maxima through shared memory (an mbarrier, bounded wait) and each writes its
+// half of P and of the output row.  S(i+1) runs on the tensor core while the
+// softmax of tile i runs, and P.V(i) right after it.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
 #include <climits>
 
@@ -34,28 +41,30 @@ using namespace sm100;
 constexpr int kD = 128;          // head width
 constexpr int kBM = 128;         // routed rows per unit (UMMA M)
 constexpr int kBN = 128;         // keys per KV tile (UMMA N of S, K of P.V)
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kHalf = 128 * 64 * 2;   // one [128][64] bf16 box, 16 KB
 constexpr uint32_t kTileBytes = 2 * kHalf; // [128][128] bf16, 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
-constexpr uint32_t kWhereTc = 2;           // status "where" id of this kernel
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;  // S_b at kColS + 128 b, P_b at kColP + 64 b
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: p <= 2^8 between rescales
+constexpr int kPolyPairs = 7;               // of every 16 element pairs, exp2 on the FMA pipe
+constexpr uint32_t kWhereTc = 2;            // status "where" id of this kernel
 
 struct Smem {
-    uint8_t q[2][kTileBytes];
-    uint8_t k[2][kTileBytes];
-    uint8_t v[2][kTileBytes];
-    int32_t row_t[2][kBM];
+    uint8_t q[2][kTileBytes];        // Q tile, double buffered by unit
+    uint8_t k[2][kTileBytes];        // K ring
+    uint8_t v[2][kTileBytes];        // V ring
+    int32_t row_t[2][kBM];           // row tables, double buffered by unit
     int32_t row_j[2][kBM];
     float row_gate[2][kBM];
-    int32_t nrows[2];
     int32_t cut_start[2][32];
     int32_t cut_prefix[2][33];
+    float xmax[2][2][kBM];           // [tile parity][warpgroup][row] partial row maxima
+    float xsum[2][kBM];              // [warpgroup][row] partial row sums
     uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
-    uint64_t s_full[2], p_full[2], pv_done[2];
+    uint64_t s_full[2], p_full[2], pv_done[2], xchg[2];
     uint64_t q_full[2], q_empty[2], rows_free[2];
-    uint64_t o_full, o_empty, mma_drain;
+    uint64_t o_full, o_empty, sum_xchg, mma_drain;
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -71,11 +80,21 @@ struct Params {
     __nv_bfloat16* O;
     uint32_t* status;
     float scale_log2;
+    int q_rows;  // B*T*h: rows of Q viewed as [B*T*h, 128]
 };
 
+// Keys needed by the unit at window w: 0 .. end-1, end = min((w+1) W, T).
 __device__ __forceinline__ int unit_kv_tiles(const UnitGeom& u, int w) {
-    const int end = min((w + 1) * u.W, u.T);  // keys 0 .. end-1
+    const int end = min((w + 1) * u.W, u.T);
     return (end + kBN - 1) / kBN;
+}
+
+// The j-th unit of this CTA: heavy windows first, zig-zag over the CTAs so that
+// each CTA's share pairs heavy and light windows.  Returns -1 past the end.
+__device__ __forceinline__ int64_t cta_unit(int64_t j, int64_t n_units) {
+    const int64_t base = j * gridDim.x;
+    const int64_t unit = base + ((j & 1) ? (int64_t)(gridDim.x - 1 - blockIdx.x) : (int64_t)blockIdx.x);
+    return unit < n_units ? unit : -1;
 }
 
 __device__ __forceinline__ bool aborted(Smem& sm) { return *((volatile int32_t*)&sm.abort_flag) != 0; }
@@ -85,11 +104,8 @@ __device__ __forceinline__ void fail(Smem& sm, const Params& p, uint32_t detail)
     report_error(p.status, GQE_ERR_DEVICE_TIMEOUT, kWhereTc, detail);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
+// tcgen05.wait::ld that also ties the loaded registers, so no use of them can
+// be scheduled before the wait.
 __device__ __forceinline__ void ld_wait_bind(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
@@ -111,10 +127,62 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
                  : "memory");
 }
 
+// ---------------------------------------------------------------- packed fp32 pairs (sm_100 f32x2)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe, x in [-126, 8]: Cody-Waite
+// style range reduction x = n + f, n = round(x), f in [-1/2, 1/2], 2^f by a
+// cubic fitted by least squares on Chebyshev nodes (exp2_poly_fit.py; max
+// relative error 1.2e-4), 2^n added to the exponent field.  Adding 1.5 * 2^23
+// leaves round(x) in the low mantissa bits of t, so t's bit pattern shifted
+// left by 23 is n << 23.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    const uint64_t kMagic = pk2(12582912.0f, 12582912.0f);
+    const uint64_t kNegMagic = pk2(-12582912.0f, -12582912.0f);
+    const uint64_t kNeg1 = pk2(-1.0f, -1.0f);
+    const uint64_t c0 = pk2(1.0f, 1.0f);
+    const uint64_t c1 = pk2(6.933686137e-01f, 6.933686137e-01f);
+    const uint64_t c2 = pk2(2.422178388e-01f, 2.422178388e-01f);
+    const uint64_t c3 = pk2(5.459282547e-02f, 5.459282547e-02f);
+    const uint64_t t = fadd2(x, kMagic);
+    const uint64_t n = fadd2(t, kNegMagic);
+    const uint64_t f = ffma2(n, kNeg1, x);
+    uint64_t q = ffma2(c3, f, c2);
+    q = ffma2(q, f, c1);
+    q = ffma2(q, f, c0);
+    float t0, t1, q0, q1;
+    up2(t, t0, t1);
+    up2(q, q0, q1);
+    return pk2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+               __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap mapQ, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -128,14 +196,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             mbar_init(&sm.kv_empty_k[i], 1);
             mbar_init(&sm.kv_empty_v[i], 1);
             mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.p_full[i], 128);
+            mbar_init(&sm.p_full[i], 256);
             mbar_init(&sm.pv_done[i], 1);
-            mbar_init(&sm.q_full[i], 32);
+            mbar_init(&sm.xchg[i], 256);
+            mbar_init(&sm.q_full[i], 1);
             mbar_init(&sm.q_empty[i], 1);
-            mbar_init(&sm.rows_free[i], 128);
+            mbar_init(&sm.rows_free[i], 256);
         }
         mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_empty, 128);
+        mbar_init(&sm.o_empty, 256);
+        mbar_init(&sm.sum_xchg, 256);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -154,29 +224,34 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         if (lane == 0) {
             tma_prefetch_desc(&mapK);
             tma_prefetch_desc(&mapV);
+            tma_prefetch_desc(&mapQ);
             uint32_t kv_it = 0;
-            for (int64_t unit = blockIdx.x; unit < n_units && !aborted(sm); unit += gridDim.x) {
+            bool k_pending = false;
+            for (int64_t j = 0;; ++j) {
+                const int64_t unit = cta_unit(j, n_units);
+                if (unit < 0 || aborted(sm)) break;
                 int b, q, w;
                 unit_coords(u, unit, b, q, w);
                 const int n = unit_kv_tiles(u, w);
+                bool ok = true;
                 for (int i = 0; i < n; ++i, ++kv_it) {
                     const int st = kv_it & 1;
                     const uint32_t par = ((kv_it >> 1) & 1) ^ 1;
-                    if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(sm, p, 1); break; }
+                    if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(sm, p, 1); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_k[st], kTileBytes);
                     tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, q, i * kBN, b);
                     tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, q, i * kBN, b);
-                    if (!mbar_wait(&sm.kv_empty_v[st], par)) {
-                        fail(sm, p, 2);
-                        mbar_wait(&sm.kv_full_k[st], (kv_it >> 1) & 1);
-                        break;
-                    }
+                    k_pending = true;
+                    if (!mbar_wait(&sm.kv_empty_v[st], par)) { fail(sm, p, 2); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_v[st], kTileBytes);
                     tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, q, i * kBN, b);
                     tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, q, i * kBN, b);
+                    k_pending = false;
                 }
+                if (!ok) break;
             }
             // Drain: every issued load lands before the CTA may exit.
+            if (k_pending) mbar_wait(&sm.kv_full_k[kv_it & 1], (kv_it >> 1) & 1);
             for (uint32_t back = 1; back <= 2 && back <= kv_it; ++back) {
                 const uint32_t it = kv_it - back;
                 mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1);
@@ -189,138 +264,190 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, kD, false, true);
             uint32_t kv_it = 0, u_it = 0;
-            bool ok = true;
+            auto issue_s = [&](uint32_t qaddr, uint32_t it) {
+                const uint32_t kaddr = smem_u32(sm.k[it & 1]);
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    const uint64_t adesc = smem_desc(qaddr + off, 16, 1024, kSwizzle128B);
+                    const uint64_t bdesc = smem_desc(kaddr + off, 16, 1024, kSwizzle128B);
+                    umma_ss(tmem + kColS + (it & 1) * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.s_full[it & 1]);
+                umma_commit(&sm.kv_empty_k[it & 1]);
+            };
+            // O += P(it) V(it), after both softmax warpgroups released P(it).
             auto issue_pv = [&](uint32_t it, bool first) -> bool {
                 const int sb = it & 1;
                 if (!mbar_wait(&sm.p_full[sb], (it >> 1) & 1)) return false;
+                if (first && !mbar_wait(&sm.o_empty, (u_it & 1) ^ 1)) return false;
                 if (!mbar_wait(&sm.kv_full_v[sb], (it >> 1) & 1)) return false;
                 tc_fence_after();
                 const uint32_t vaddr = smem_u32(sm.v[sb]);
                 for (int kk = 0; kk < kBN / 16; ++kk) {
                     const uint64_t bdesc = smem_desc(vaddr + kk * 2048, kHalf, 1024, kSwizzle128B);
-                    umma_ts(tmem + kColO, tmem + kColP0 + sb * 64 + kk * 8, bdesc, idesc_pv,
+                    umma_ts(tmem + kColO, tmem + kColP + sb * 64 + kk * 8, bdesc, idesc_pv,
                             (first && kk == 0) ? 0u : 1u);
                 }
                 umma_commit(&sm.kv_empty_v[sb]);
                 umma_commit(&sm.pv_done[sb]);
                 return true;
             };
-            for (int64_t unit = blockIdx.x; unit < n_units && ok && !aborted(sm); unit += gridDim.x, ++u_it) {
+            bool ok = true;
+            for (int64_t j = 0; ok; ++j, ++u_it) {
+                const int64_t unit = cta_unit(j, n_units);
+                if (unit < 0 || aborted(sm)) break;
                 int b, q, w;
                 unit_coords(u, unit, b, q, w);
                 const int n = unit_kv_tiles(u, w);
                 const int qs = u_it & 1;
-                if (!mbar_wait(&sm.q_full[qs], (u_it >> 1) & 1)) { fail(sm, p, 10); ok = false; break; }
+                if (!mbar_wait(&sm.q_full[qs], (u_it >> 1) & 1)) { fail(sm, p, 10); break; }
                 tc_fence_after();
                 const uint32_t qaddr = smem_u32(sm.q[qs]);
-                for (int i = 0; i < n; ++i, ++kv_it) {
-                    const int st = kv_it & 1;
-                    if (!mbar_wait(&sm.kv_full_k[st], (kv_it >> 1) & 1)) { fail(sm, p, 11); ok = false; break; }
+                for (int i = 0; i < n; ++i) {
+                    const uint32_t it = kv_it + i;
+                    if (!mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1)) { fail(sm, p, 11); ok = false; break; }
                     tc_fence_after();
-                    const uint32_t kaddr = smem_u32(sm.k[st]);
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                        const uint64_t adesc = smem_desc(qaddr + off, 16, 1024, kSwizzle128B);
-                        const uint64_t bdesc = smem_desc(kaddr + off, 16, 1024, kSwizzle128B);
-                        umma_ss(tmem + kColS0 + st * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sm.kv_empty_k[st]);
-                    umma_commit(&sm.s_full[st]);
+                    issue_s(qaddr, it);
                     if (i == n - 1) umma_commit(&sm.q_empty[qs]);
-                    if (i >= 1) {
-                        if (i == 1 && !mbar_wait(&sm.o_empty, (u_it & 1) ^ 1)) { fail(sm, p, 12); ok = false; break; }
-                        if (!issue_pv(kv_it - 1, i == 1)) { fail(sm, p, 13); ok = false; break; }
-                    }
+                    if (i >= 1 && !issue_pv(it - 1, i == 1)) { fail(sm, p, 12); ok = false; break; }
                 }
                 if (!ok) break;
-                if (n == 1 && !mbar_wait(&sm.o_empty, (u_it & 1) ^ 1)) { fail(sm, p, 14); break; }
-                if (!issue_pv(kv_it - 1, n == 1)) { fail(sm, p, 15); break; }
+                if (!issue_pv(kv_it + n - 1, n == 1)) { fail(sm, p, 13); break; }
                 umma_commit(&sm.o_full);
+                kv_it += n;
             }
             // Drain: all issued MMAs complete before TMEM is released.
             umma_commit(&sm.mma_drain);
             mbar_wait(&sm.mma_drain, 0);
         }
     } else if (warp == 2) {
-        // ------------------------------------------------------------ row table + Q gather
+        // ------------------------------------------------------------ row tables + Q gather
         uint32_t u_it = 0;
-        for (int64_t unit = blockIdx.x; unit < n_units && !aborted(sm); unit += gridDim.x, ++u_it) {
+        int64_t armed = -1;  // last unit whose Q loads were issued
+        const int32_t total = (int32_t)((int64_t)u.B * u.T * u.g * u.k);
+        for (int64_t j = 0;; ++j, ++u_it) {
+            const int64_t unit = cta_unit(j, n_units);
+            if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
-            const int qs = u_it & 1;
+            const int rs = u_it & 1;
             const uint32_t par = ((u_it >> 1) & 1) ^ 1;
-            bool ok = mbar_wait(&sm.q_empty[qs], par);
-            ok = ok && mbar_wait(&sm.rows_free[qs], par);
-            if (!__all_sync(0xffffffffu, ok)) { if (lane == 0) fail(sm, p, 20); break; }
+            // Row table and Q tile are double buffered: this unit's are built
+            // while the previous unit computes.
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_free[rs], par))) {
+                if (lane == 0) fail(sm, p, 20);
+                break;
+            }
             const int w0 = w * u.W;
             // 1. per-head slices of the window in the packed position lists
             if (lane < u.hpg) {
-                const int j = q * u.hpg + lane;
-                const int32_t total = (int32_t)((int64_t)u.B * u.T * u.g * u.k);
-                int32_t a0 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, j, w0);
-                int32_t a1 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, j, w0 + u.W);
+                const int jh = q * u.hpg + lane;
+                int32_t a0 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0);
+                int32_t a1 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0 + u.W);
                 if (a0 < 0 || a1 < a0 || a1 > total) {  // malformed lists: report, use none
                     report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 41);
                     a0 = a1 = 0;
                 }
-                sm.cut_start[qs][lane] = a0;
-                sm.cut_prefix[qs][lane + 1] = a1 - a0;
+                sm.cut_start[rs][lane] = a0;
+                sm.cut_prefix[rs][lane + 1] = a1 - a0;
             }
             __syncwarp();
             if (lane == 0) {
                 int acc = 0;
-                sm.cut_prefix[qs][0] = 0;
+                sm.cut_prefix[rs][0] = 0;
                 for (int jj = 0; jj < u.hpg; ++jj) {
-                    acc += sm.cut_prefix[qs][jj + 1];
-                    sm.cut_prefix[qs][jj + 1] = acc;
+                    acc = min(acc + sm.cut_prefix[rs][jj + 1], kBM);
+                    sm.cut_prefix[rs][jj + 1] = acc;
                 }
-                sm.nrows[qs] = min(acc, kBM);
             }
             __syncwarp();
-            const int nrows = sm.nrows[qs];
-            // 2. row table: position, head and gate of each routed row
-            for (int r = lane; r < kBM; r += 32) {
-                int t = -1, j = 0;
-                float gv = 0.f;
+            const int nrows = sm.cut_prefix[rs][u.hpg];
+            // 2. row table: position, head and gate of each routed row.  Each
+            // lane's 4 rows issue their loads together (two dependent rounds:
+            // head_pos, then the token's k (idx, gate) pairs).
+            int tt[kBM / 32], jh[kBM / 32];
+#pragma unroll
+            for (int i = 0; i < kBM / 32; ++i) {
+                const int r = lane + 32 * i;
+                tt[i] = -1;
+                jh[i] = 0;
                 if (r < nrows) {
                     int jj = 0;
-                    while (sm.cut_prefix[qs][jj + 1] <= r) ++jj;
-                    j = q * u.hpg + jj;
-                    t = p.head_pos[sm.cut_start[qs][jj] + (r - sm.cut_prefix[qs][jj])];
-                    if (t < w0 || t >= min(w0 + u.W, u.T)) {  // outside the window: report, drop the row
+                    while (sm.cut_prefix[rs][jj + 1] <= r) ++jj;
+                    jh[i] = q * u.hpg + jj;
+                    tt[i] = p.head_pos[sm.cut_start[rs][jj] + (r - sm.cut_prefix[rs][jj])];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kBM / 32; ++i) {
+                const int r = lane + 32 * i;
+                float gv = 0.f;
+                if (tt[i] >= 0) {
+                    if (tt[i] < w0 || tt[i] >= min(w0 + u.W, u.T)) {  // outside the window: report, drop
                         report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 40);
-                        t = -1;
+                        tt[i] = -1;
                     } else {
-                        const int64_t sel = (((int64_t)b * u.T + t) * u.g + q) * u.k;
-                        for (int s = 0; s < u.k; ++s)
-                            if (p.idx[sel + s] == j) gv = p.gate[sel + s];
+                        const int64_t sel = (((int64_t)b * u.T + tt[i]) * u.g + q) * u.k;
+                        int sj[4];
+                        float sg[4];
+#pragma unroll
+                        for (int s2 = 0; s2 < 4; ++s2) {
+                            if (s2 < u.k) {
+                                sj[s2] = p.idx[sel + s2];
+                                sg[s2] = p.gate[sel + s2];
+                            }
+                        }
+#pragma unroll
+                        for (int s2 = 0; s2 < 4; ++s2)
+                            if (s2 < u.k && sj[s2] == jh[i]) gv = sg[s2];
                     }
                 }
-                sm.row_t[qs][r] = t;
-                sm.row_j[qs][r] = j;
-                sm.row_gate[qs][r] = gv;
+                sm.row_t[rs][r] = tt[i];
+                sm.row_j[rs][r] = jh[i];
+                sm.row_gate[rs][r] = gv;
+                // pull the row into L2 while the previous unit still computes
+                if (tt[i] >= 0) {
+                    const __nv_bfloat16* row = p.Q + (((int64_t)b * u.T + tt[i]) * u.h + jh[i]) * kD;
+                    prefetch_l2(row);
+                    prefetch_l2(row + 64);
+                }
             }
             __syncwarp();
-            // 3. Q gather: row r, 16-byte chunk c -> half c/8, 128B-swizzled slot
-            const uint32_t qbase = smem_u32(sm.q[qs]);
-            for (int e = lane; e < kBM * 16; e += 32) {
-                const int r = e >> 4, c = e & 15;
-                const int t = sm.row_t[qs][r];
-                const int j = sm.row_j[qs][r];
-                const uint32_t dst = qbase + (c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                const __nv_bfloat16* src =
-                    (t >= 0) ? p.Q + (((int64_t)b * u.T + t) * u.h + j) * kD + c * 8 : p.Q;
-                cp_async16(dst, src, t >= 0 ? 16u : 0u);
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_empty[rs], par))) {
+                if (lane == 0) fail(sm, p, 21);
+                break;
             }
-            cp_async_wait_all();
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.q_full[qs]);
+            // 3. Q gather by TMA: each routed row is one row of Q viewed as
+            // [B*T*h, 128].  One tile::gather4 copy moves four rows' 64-column
+            // halves (box one row high) to rows r..r+3 of a tile half; the
+            // 128-byte swizzle follows the shared-memory address, so each row
+            // gets its own chunk permutation.  Padding rows name an
+            // out-of-range row, which the TMA zero-fills.
+            if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[rs], kTileBytes);
+            __syncwarp();
+            {
+                const int r0 = lane * 4;  // four rows per lane
+                int row[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tr = sm.row_t[rs][r0 + e];
+                    row[e] = (tr >= 0) ? (int)(((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][r0 + e]) : p.q_rows;
+                }
+                uint8_t* dst = sm.q[rs] + r0 * 128;
+                tma_gather4_2d(&mapQ, &sm.q_full[rs], dst, 0, row[0], row[1], row[2], row[3]);
+                tma_gather4_2d(&mapQ, &sm.q_full[rs], dst + kHalf, 64, row[0], row[1], row[2], row[3]);
+            }
+            armed = u_it;
         }
+        // Drain: the last issued Q loads land before the CTA may exit.
+        if (armed >= 0) mbar_wait(&sm.q_full[armed & 1], (armed >> 1) & 1);
     } else if (warp == 3) {
         // ------------------------------------------------------------ zero fill of unselected slots
-        // Each unit's window [w0, w0+W) x heads of group q: slots whose head the
+        // The unit's window [w0, w0 + W) x heads of group q: slots whose head the
         // token did not select are written as zeros (16 lanes per 256-byte slot).
-        for (int64_t unit = blockIdx.x; unit < n_units && !aborted(sm); unit += gridDim.x) {
+        for (int64_t j = 0;; ++j) {
+            const int64_t unit = cta_unit(j, n_units);
+            if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
             const int w0 = w * u.W;
@@ -328,121 +455,175 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             const int slots = (wend - w0) * u.hpg;
             for (int e = lane >> 4; e < slots; e += 2) {
                 const int t = w0 + e / u.hpg;
-                const int j = q * u.hpg + e % u.hpg;
+                const int jh = q * u.hpg + e % u.hpg;
                 const int64_t sel = (((int64_t)b * u.T + t) * u.g + q) * u.k;
                 bool hit = false;
-                for (int s = 0; s < u.k; ++s) hit |= (p.idx[sel + s] == j);
+                for (int s = 0; s < u.k; ++s) hit |= (p.idx[sel + s] == jh);
                 if (!hit) {
-                    uint4* o = reinterpret_cast<uint4*>(p.O + (((int64_t)b * u.T + t) * u.h + j) * kD);
+                    uint4* o = reinterpret_cast<uint4*>(p.O + (((int64_t)b * u.T + t) * u.h + jh) * kD);
                     o[lane & 15] = make_uint4(0, 0, 0, 0);
                 }
             }
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        const int wg = (warp - 4) >> 2;    // key-column half of this warpgroup
         const int wq = warp & 3;           // TMEM lane quarter of this warp
         const int r = wq * 32 + lane;      // routed row owned by this thread
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        uint32_t kv_it = 0, u_it = 0;
-        for (int64_t unit = blockIdx.x; unit < n_units && !aborted(sm); unit += gridDim.x, ++u_it) {
+        const uint32_t o_addr = tmem + lane_off + kColO + wg * 64;
+        uint32_t ctile = 0, u_it = 0;
+        for (int64_t j = 0;; ++j, ++u_it) {
+            const int64_t unit = cta_unit(j, n_units);
+            if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
             const int n = unit_kv_tiles(u, w);
-            const int qs = u_it & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[qs], (u_it >> 1) & 1))) { if (lane == 0) fail(sm, p, 30); break; }
-            const int t_row = sm.row_t[qs][r];
+            const int rs = u_it & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[rs], (u_it >> 1) & 1))) {
+                if (lane == 0) fail(sm, p, 30);
+                break;
+            }
+            const int t_row = sm.row_t[rs][r];
             const int t_eff = (t_row >= 0) ? t_row : INT_MAX;  // padding rows: unmasked, output dropped
-            const int w0 = w * u.W;
+            const int lo = w * u.W;                           // first position of the window
             float m = -INFINITY, l = 0.f;
             bool ok = true;
-            for (int i = 0; i < n; ++i, ++kv_it) {
-                const int sb = kv_it & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (kv_it >> 1) & 1))) { if (lane == 0) fail(sm, p, 31); ok = false; break; }
+            for (int i = 0; i < n; ++i, ++ctile) {
+                const int sb = ctile & 1;
+                const uint32_t ph = (ctile >> 1) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], ph))) {
+                    if (lane == 0) fail(sm, p, 31);
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                uint32_t s[4][32];
-                const uint32_t sa = tmem + lane_off + kColS0 + sb * 128;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(sa + c * 32, s[c]);
+                uint32_t s[2][32];
+                const uint32_t s_addr = tmem + lane_off + kColS + sb * 128 + wg * 64;
+                tmem_ld32(s_addr, s[0]);
+                tmem_ld32(s_addr + 32, s[1]);
                 ld_wait_bind(s[0]);
                 ld_bind(s[1]);
-                ld_bind(s[2]);
-                ld_bind(s[3]);
-                const int kv0 = i * kBN;
-                const bool need_mask = kv0 + kBN - 1 > w0;
-                float mx = -INFINITY;
+                const int kv0 = i * kBN + wg * 64;  // key index of this half's first column
+                const bool need_mask = i * kBN + kBN - 1 > lo;
+                if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                    for (int cb = 0; cb < 2; ++cb)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float v = __uint_as_float(s[c][e]) * p.scale_log2;
-                        if (need_mask && kv0 + c * 32 + e > t_eff) v = -INFINITY;
-                        s[c][e] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
-                    }
+                        for (int e = 0; e < 32; ++e)
+                            if (kv0 + cb * 32 + e > t_eff) s[cb][e] = __float_as_uint(-INFINITY);
                 }
-                // Lazy rescaling: keep the running max unless it grows by more than the threshold.
+                // partial row max of the raw scores, then the exchange with the other half
+                float mq[2];
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    float a0 = __uint_as_float(s[cb][0]);
+#pragma unroll
+                    for (int e = 1; e < 31; e += 2)
+                        a0 = fmax3(a0, __uint_as_float(s[cb][e]), __uint_as_float(s[cb][e + 1]));
+                    mq[cb] = fmaxf(a0, __uint_as_float(s[cb][31]));
+                }
+                sm.xmax[sb][wg][r] = fmaxf(mq[0], mq[1]);
+                mbar_arrive(&sm.xchg[sb]);
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.xchg[sb], ph))) {
+                    if (lane == 0) fail(sm, p, 32);
+                    ok = false;
+                    break;
+                }
+                const float mx = fmaxf(sm.xmax[sb][0][r], sm.xmax[sb][1][r]) * p.scale_log2;
+                // Lazy rescaling (identical decision in both halves): keep the running
+                // max unless it grows by more than the threshold.
                 float m_use = m;
                 bool rescale = false;
                 if (mx > m + kRescaleThreshold || m == -INFINITY) {
                     m_use = mx;
                     rescale = (i > 0);
                 }
-                // P buffer sb is free once P.V of tile kv_it-2 is done.
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[sb], ((kv_it >> 1) & 1) ^ 1))) { if (lane == 0) fail(sm, p, 32); ok = false; break; }
-                float rowsum = 0.f;
-                const uint32_t pa = tmem + lane_off + kColP0 + sb * 64;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = fast_exp2(__uint_as_float(s[c][2 * e]) - m_use);
-                        const float p1 = fast_exp2(__uint_as_float(s[c][2 * e + 1]) - m_use);
-                        rowsum += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(pa + c * 16, pk);
-                }
                 if (__any_sync(0xffffffffu, rescale)) {
-                    // O holds P.V of tiles < i once P.V of tile kv_it-1 is done.
-                    const uint32_t prev = kv_it - 1;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[prev & 1], (prev >> 1) & 1))) { if (lane == 0) fail(sm, p, 33); ok = false; break; }
+                    // O must hold P.V of every earlier tile before it is rescaled.
+                    const uint32_t prev = ctile - 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[prev & 1], (prev >> 1) & 1))) {
+                        if (lane == 0) fail(sm, p, 33);
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const float alpha = rescale ? fast_exp2(m - m_use) : 1.0f;
-                    const uint32_t oa = tmem + lane_off + kColO;
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int cb = 0; cb < 2; ++cb) {
                         uint32_t o[32];
-                        tmem_ld32(oa + c * 32, o);
+                        tmem_ld32(o_addr + cb * 32, o);
                         ld_wait_bind(o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st16(oa + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-                        tmem_st16(oa + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+                        tmem_st16(o_addr + cb * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+                        tmem_st16(o_addr + cb * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
                     }
                     l *= alpha;
                 }
-                l += rowsum;
+                // P buffer sb is free once P.V of tile ctile-2 is done.
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[sb], ph ^ 1))) {
+                    if (lane == 0) fail(sm, p, 34);
+                    ok = false;
+                    break;
+                }
+                // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
+                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
+                const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);
+                const uint64_t NM2 = pk2(-m_use, -m_use);
+                const uint32_t pa = tmem + lane_off + kColP + sb * 64 + wg * 32;
+                uint64_t sum2[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x2 =
+                            ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2);
+                        float x0, x1, p0, p1;
+                        up2(x2, x0, x1);
+                        if (e < kPolyPairs && !need_mask) {
+                            up2(exp2_poly2(pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p0, p1);
+                        } else {
+                            p0 = fast_exp2(x0);
+                            p1 = fast_exp2(x1);
+                        }
+                        sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(pa + cb * 16, pk);
+                }
+                float sa, sb2;
+                up2(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])), sa, sb2);
+                l += sa + sb2;
                 m = m_use;
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.p_full[sb]);
             }
             if (!ok) break;
-            // Epilogue: O / l * gate -> bf16 row of O[b, t, j, :].
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full, u_it & 1))) { if (lane == 0) fail(sm, p, 34); break; }
+            // Epilogue: O / l * gate -> bf16 half row of O[b, t, j, :].  The row sum
+            // is the sum of the two halves' partial sums.
+            sm.xsum[wg][r] = l;
+            mbar_arrive(&sm.sum_xchg);
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.sum_xchg, u_it & 1)) ||
+                !__all_sync(0xffffffffu, mbar_wait(&sm.o_full, u_it & 1))) {
+                if (lane == 0) fail(sm, p, 35);
+                break;
+            }
             tc_fence_after();
-            const int j_row = sm.row_j[qs][r];
-            const float f = (t_row >= 0) ? sm.row_gate[qs][r] / l : 0.f;
-            __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD;
-            const uint32_t oa = tmem + lane_off + kColO;
+            const float lt = sm.xsum[0][r] + sm.xsum[1][r];
+            const int j_row = sm.row_j[rs][r];
+            const float f = (t_row >= 0) ? sm.row_gate[rs][r] / lt : 0.f;
+            __nv_bfloat16* orow =
+                p.O + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD + wg * 64;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int cb = 0; cb < 2; ++cb) {
                 uint32_t o[32];
-                tmem_ld32(oa + c * 32, o);
+                tmem_ld32(o_addr + cb * 32, o);
                 ld_wait_bind(o);
                 if (t_row >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 pk;
@@ -456,7 +637,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             }
             tc_fence_before();
             mbar_arrive(&sm.o_empty);
-            mbar_arrive(&sm.rows_free[qs]);
+            mbar_arrive(&sm.rows_free[rs]);
         }
     }
 
@@ -476,16 +657,24 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     if (s.k > 4 || s.h / s.g > 32) return cudaErrorNotSupported;
     UnitGeom u;
     u.B = s.B; u.T = s.T; u.h = s.h; u.g = s.g; u.k = s.k; u.hpg = s.h / s.g;
-    u.W = 32 * (4 / s.k);  // k*W <= 128 rows, W a multiple of the 32-token chunk
+    u.W = 32 * (4 / s.k);  // k*W <= 128 rows per unit, W a multiple of the 32-token chunk
     u.nwin = (s.T + u.W - 1) / u.W;
     u.nchunk = gqe_chunk_count(s.T);
 
-    CUtensorMap mapK, mapV;
+    CUtensorMap mapK, mapV, mapQ;
     const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
     const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kBN, 1};
     if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    const int64_t q_rows = (int64_t)s.B * s.T * s.h;
+    if (q_rows >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
+    {
+        const uint64_t qdims[2] = {(uint64_t)kD, (uint64_t)q_rows};
+        const uint64_t qstrides[1] = {(uint64_t)kD * 2};
+        const uint32_t qbox[2] = {64, 1};
+        if (!make_bf16_map(&mapQ, a.Q, 2, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
+    }
 
     Params p;
     p.u = u;
@@ -498,6 +687,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     p.O = (__nv_bfloat16*)a.O;
     p.status = (uint32_t*)a.status;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    p.q_rows = (int)q_rows;
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -507,7 +697,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    prefill_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, p);
+    prefill_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, p);
     return cudaGetLastError();
 }
 
