@@ -14,9 +14,9 @@
 namespace gqe {
 namespace {
 
-constexpr int kDecodeChunk = 256;   // cache rows per block
+constexpr int kDecodeChunk = 512;   // cache rows per block
 constexpr int kDecodeThreads = 256; // 8 warps; warp w serves groups w, w+8, ...
-constexpr int kDecodeUnroll = 4;    // token steps in flight per lane
+constexpr int kDecodeUnroll = 8;    // token steps in flight per lane
 
 template <int D>
 struct PartRec {

@@ -561,12 +561,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     }
                     l *= alpha;
                 }
-                // P buffer sb is free once P.V of tile ctile-2 is done.
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[sb], ph ^ 1))) {
-                    if (lane == 0) fail(sm, p, 34);
-                    ok = false;
-                    break;
-                }
+                // P buffer sb was last read by P.V(ctile-2), issued before S(ctile):
+                // the commit that signalled s_full covers it, so the buffer is free.
                 // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
                 // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
                 const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);

@@ -46,16 +46,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// As above, but a thread whose phase is not complete is suspended in hardware
+// until the phase completes or suspend_ns elapse, instead of spinning on the
+// issue slots the compute warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
 
 // Wait for the phase with the given parity to complete.  Bounded: gives up
 // after kWaitTimeoutNs of wall time (or 2^26 polls) and returns false.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+constexpr uint32_t kSuspendHintNs = 1000000u;       // 1 ms per suspended poll
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; it < (1u << 26); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+        if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
     }
     return false;
 }
