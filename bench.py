@@ -163,9 +163,15 @@ def max_over_ranks(v: float, ws: int) -> float:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_value(work: float, ws: int, steps: int, step_ms_max: float, scale: float) -> float:
+    """Whole-job throughput: the work of all ranks' steps over the slowest rank's time."""
+    return work * ws * steps / (step_ms_max * 1e-3) * scale
 
 
 # ---------------------------------------------------------------------------
@@ -268,7 +274,7 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
     attn_ms = [b.elapsed_time(c) for _, b, c in ev]
     route_ms = [a.elapsed_time(b) for a, b, _ in ev]
     step_ms_max = max_over_ranks(step_ms, ws)
-    value = work * ws * steps / (step_ms_max * 1e-3) * scale
+    value = aggregate_value(work, ws, steps, step_ms_max, scale)
 
     kern = "decode_partial_kernel" if w.decode else "prefill_tc_kernel"
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
