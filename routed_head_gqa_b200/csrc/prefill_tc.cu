@@ -444,24 +444,56 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     } else if (warp == 3) {
         // ------------------------------------------------------------ zero fill of unselected slots
         // The unit's window [w0, w0 + W) x heads of group q: slots whose head the
-        // token did not select are written as zeros (16 lanes per 256-byte slot).
+        // token did not select are written as zeros.  Each lane owns up to 4 of
+        // the window's tokens and loads their k selections at once (one round
+        // of loads per window, not one per slot); the warp then zeroes the
+        // unselected 256-byte slots, 16 lanes per slot.
+        const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
         for (int64_t j = 0;; ++j) {
             const int64_t unit = cta_unit(j, n_units);
             if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
             const int w0 = w * u.W;
-            const int wend = min(w0 + u.W, u.T);
-            const int slots = (wend - w0) * u.hpg;
-            for (int e = lane >> 4; e < slots; e += 2) {
-                const int t = w0 + e / u.hpg;
-                const int jh = q * u.hpg + e % u.hpg;
-                const int64_t sel = (((int64_t)b * u.T + t) * u.g + q) * u.k;
-                bool hit = false;
-                for (int s = 0; s < u.k; ++s) hit |= (p.idx[sel + s] == jh);
-                if (!hit) {
-                    uint4* o = reinterpret_cast<uint4*>(p.O + (((int64_t)b * u.T + t) * u.h + jh) * kD);
-                    o[lane & 15] = make_uint4(0, 0, 0, 0);
+            const int nt = min(w0 + u.W, u.T) - w0;  // tokens in the window, <= 128
+            int sj[kBM / 32][4];
+#pragma unroll
+            for (int i = 0; i < kBM / 32; ++i) {
+                const int tt = lane + 32 * i;
+                const int64_t sel = (((int64_t)b * u.T + w0 + tt) * u.g + q) * u.k;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) sj[i][s] = (tt < nt && s < u.k) ? p.idx[sel + s] : -1;
+            }
+            uint32_t unsel[kBM / 32];
+            bool any = false;
+#pragma unroll
+            for (int i = 0; i < kBM / 32; ++i) {
+                uint32_t m = 0;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const int a = sj[i][s] - q * u.hpg;  // head within the group
+                    if (a >= 0 && a < u.hpg) m |= 1u << a;
+                }
+                unsel[i] = (lane + 32 * i < nt) ? (~m & group_mask) : 0u;
+                any |= unsel[i] != 0u;
+            }
+            if (!__any_sync(0xffffffffu, any)) continue;
+            for (int tt = 0; tt < nt; ++tt) {
+                uint32_t un = __shfl_sync(0xffffffffu, unsel[0], tt & 31);
+#pragma unroll
+                for (int i = 1; i < kBM / 32; ++i) {
+                    const uint32_t v = __shfl_sync(0xffffffffu, unsel[i], tt & 31);
+                    if ((tt >> 5) == i) un = v;
+                }
+                __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + w0 + tt) * u.h + q * u.hpg) * kD;
+                while (un != 0u) {
+                    // two slots per pass: the lowest set bit for lanes 0-15, the next for 16-31
+                    const int a0 = __ffs(un) - 1;
+                    un &= un - 1u;
+                    const int a1 = (un != 0u) ? __ffs(un) - 1 : -1;
+                    if (a1 >= 0) un &= un - 1u;
+                    const int a = (lane < 16) ? a0 : a1;
+                    if (a >= 0) reinterpret_cast<uint4*>(orow + (int64_t)a * kD)[lane & 15] = make_uint4(0, 0, 0, 0);
                 }
             }
         }
