@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "5f91ce8539ca033d", "bytes_per_launch": 104152576 + 31594496,
+        "sha": "52eb0dd68639c989", "bytes_per_launch": 104635904 + 31958016,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
 }
 
