@@ -7,26 +7,23 @@
 //   O[b,t,j,:] = gate * sum_{s<=t} softmax_s(Q[b,t,j] . K[b,s,j/hpg] / sqrt(128)) V[b,s,j/hpg]
 // and O[b,t,j,:] = 0 for the unselected (t, j).
 //
-// Work unit: (b, KV group q, window of W = 32*floor(4/k) positions).  Every
-// token selects exactly k heads per group, so the window holds k*W <= 128 routed
-// rows (taken from the per-head packed position lists): one M=128 Q tile.  Each
-// K/V tile of the group is loaded once per unit by TMA and serves every routed
-// head of the group in the window.
+// Work unit: (b, KV group q, window of 2W positions), W = 32*floor(4/k).  Every
+// token selects exactly k heads per group, so each W-position half of the
+// window holds k*W <= 128 routed rows (taken from the per-head packed position
+// lists): two M=128 Q tiles.  Both tiles share every K/V tile of the group,
+// which is loaded once per unit by TMA.
 //
 // Roles (384 threads, one persistent CTA per SM):
 //   warp 0      TMA producer for K/V tiles; owns the TMEM allocation
-//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered S and
-//               O += P V, both on tcgen05
-//   warp 2      row tables, L2 prefetch and Q gather (TMA tile::gather4,
-//               128B-swizzled) into a double-buffered Q tile
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V on tcgen05
+//   warp 2      row tables and Q gather (TMA tile::gather4 of routed rows, 128B-swizzled)
 //   warp 3      zero fill of the window's unselected output slots
-//   warps 4-7   softmax + epilogue, key columns 0-63 of every row
-//   warps 8-11  softmax + epilogue, key columns 64-127 of every row
-// The two softmax warpgroups share each row: they exchange their partial row
-// maxima through shared memory (an mbarrier, bounded wait) and each writes its
-// half of P and of the output row.  S(i+1) runs on the tensor core while the
-// softmax of tile i runs, and P.V(i) right after it.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+//   warps 4-7   softmax + epilogue of Q tile 0 (one row per thread)
+//   warps 8-11  softmax + epilogue of Q tile 1
+// The two softmax warpgroups alternate with the tensor core: while one turns
+// S into P, the tensor core runs the other tile's P.V and next QK^T.
+// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512); P_t (bf16
+// pairs) overwrites the first 64 columns of S_t once S_t is in registers.
 #include <climits>
 
 #include "sm100.cuh"
@@ -39,32 +36,34 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;          // head width
-constexpr int kBM = 128;         // routed rows per unit (UMMA M)
+constexpr int kBM = 128;         // routed rows per Q tile (UMMA M)
 constexpr int kBN = 128;         // keys per KV tile (UMMA N of S, K of P.V)
+constexpr int kQT = 2;           // Q tiles per unit
 constexpr int kThreads = 384;
 constexpr uint32_t kHalf = 128 * 64 * 2;   // one [128][64] bf16 box, 16 KB
 constexpr uint32_t kTileBytes = 2 * kHalf; // [128][128] bf16, 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;  // S_b at kColS + 128 b, P_b at kColP + 64 b
+constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * tile
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: p <= 2^8 between rescales
 constexpr int kPolyPairs = 7;               // of every 16 element pairs, exp2 on the FMA pipe
 constexpr uint32_t kWhereTc = 2;            // status "where" id of this kernel
+// Register split (setmaxnreg): 4 control warps at 88, 8 softmax warps at 208.
+// 128*88 + 256*208 = 64512 = 384 * 168, the block's registers at launch.
+constexpr int kRegsLaunch = 168, kRegsCtl = 88, kRegsSoftmax = 208;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
 
 struct Smem {
-    uint8_t q[2][kTileBytes];        // Q tile, double buffered by unit
+    uint8_t q[kQT][kTileBytes];      // Q tiles (single buffer, guarded by q_empty)
     uint8_t k[2][kTileBytes];        // K ring
     uint8_t v[2][kTileBytes];        // V ring
-    int32_t row_t[2][kBM];           // row tables, double buffered by unit
-    int32_t row_j[2][kBM];
-    float row_gate[2][kBM];
-    int32_t cut_start[2][32];
-    int32_t cut_prefix[2][33];
-    float xmax[2][2][kBM];           // [tile parity][warpgroup][row] partial row maxima
-    float xsum[2][kBM];              // [warpgroup][row] partial row sums
+    int32_t row_t[2][kQT][kBM];      // row tables, double buffered by unit
+    int32_t row_j[2][kQT][kBM];
+    float row_gate[2][kQT][kBM];
+    int32_t cut_start[2][kQT][32];
+    int32_t cut_prefix[2][kQT][33];
     uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
-    uint64_t s_full[2], p_full[2], pv_done[2], xchg[2];
-    uint64_t q_full[2], q_empty[2], rows_free[2];
-    uint64_t o_full, o_empty, sum_xchg, mma_drain;
+    uint64_t s_full[kQT], p_full[kQT], o_full[kQT], o_empty[kQT];
+    uint64_t q_full[2], q_empty, rows_free[2], mma_drain;
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -83,9 +82,9 @@ struct Params {
     int q_rows;  // B*T*h: rows of Q viewed as [B*T*h, 128]
 };
 
-// Keys needed by the unit at window w: 0 .. end-1, end = min((w+1) W, T).
-__device__ __forceinline__ int unit_kv_tiles(const UnitGeom& u, int w) {
-    const int end = min((w + 1) * u.W, u.T);
+// Keys needed by Q tile t of the unit at window w: 0 .. end-1, end = min(w0 + (t+1)W, T).
+__device__ __forceinline__ int tile_kv_tiles(const UnitGeom& u, int w, int t) {
+    const int end = min(w * kQT * u.W + (t + 1) * u.W, u.T);
     return (end + kBN - 1) / kBN;
 }
 
@@ -103,6 +102,7 @@ __device__ __forceinline__ void fail(Smem& sm, const Params& p, uint32_t detail)
     atomicExch(&sm.abort_flag, 1);
     report_error(p.status, GQE_ERR_DEVICE_TIMEOUT, kWhereTc, detail);
 }
+
 
 // tcgen05.wait::ld that also ties the loaded registers, so no use of them can
 // be scheduled before the wait.
@@ -126,6 +126,7 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
                  :
                  : "memory");
 }
+
 
 // ---------------------------------------------------------------- packed fp32 pairs (sm_100 f32x2)
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -195,17 +196,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             mbar_init(&sm.kv_full_v[i], 1);
             mbar_init(&sm.kv_empty_k[i], 1);
             mbar_init(&sm.kv_empty_v[i], 1);
-            mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.p_full[i], 256);
-            mbar_init(&sm.pv_done[i], 1);
-            mbar_init(&sm.xchg[i], 256);
             mbar_init(&sm.q_full[i], 1);
-            mbar_init(&sm.q_empty[i], 1);
             mbar_init(&sm.rows_free[i], 256);
         }
-        mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_empty, 256);
-        mbar_init(&sm.sum_xchg, 256);
+        for (int t = 0; t < kQT; ++t) {
+            mbar_init(&sm.s_full[t], 1);
+            mbar_init(&sm.p_full[t], 128);
+            mbar_init(&sm.o_full[t], 1);
+            mbar_init(&sm.o_empty[t], 128);
+        }
+        mbar_init(&sm.q_empty, 1);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -220,6 +220,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&mapK);
@@ -232,7 +233,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 if (unit < 0 || aborted(sm)) break;
                 int b, q, w;
                 unit_coords(u, unit, b, q, w);
-                const int n = unit_kv_tiles(u, w);
+                const int n = tile_kv_tiles(u, w, kQT - 1);
                 bool ok = true;
                 for (int i = 0; i < n; ++i, ++kv_it) {
                     const int st = kv_it & 1;
@@ -259,68 +260,91 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             }
         }
     } else if (warp == 1) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, kD, false, true);
-            uint32_t kv_it = 0, u_it = 0;
-            auto issue_s = [&](uint32_t qaddr, uint32_t it) {
+            uint32_t kv_it = 0, u_it = 0, c[kQT] = {0, 0};
+            bool ok = true;
+            auto issue_s = [&](int t, uint32_t it) {
+                const uint32_t qaddr = smem_u32(sm.q[t]);
                 const uint32_t kaddr = smem_u32(sm.k[it & 1]);
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
                     const uint64_t adesc = smem_desc(qaddr + off, 16, 1024, kSwizzle128B);
                     const uint64_t bdesc = smem_desc(kaddr + off, 16, 1024, kSwizzle128B);
-                    umma_ss(tmem + kColS + (it & 1) * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + kColS + t * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&sm.s_full[it & 1]);
-                umma_commit(&sm.kv_empty_k[it & 1]);
+                umma_commit(&sm.s_full[t]);
             };
-            // O += P(it) V(it), after both softmax warpgroups released P(it).
-            auto issue_pv = [&](uint32_t it, bool first) -> bool {
-                const int sb = it & 1;
-                if (!mbar_wait(&sm.p_full[sb], (it >> 1) & 1)) return false;
-                if (first && !mbar_wait(&sm.o_empty, (u_it & 1) ^ 1)) return false;
-                if (!mbar_wait(&sm.kv_full_v[sb], (it >> 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t vaddr = smem_u32(sm.v[sb]);
+            auto issue_pv = [&](int t, uint32_t it, bool first) {
+                const uint32_t vaddr = smem_u32(sm.v[it & 1]);
                 for (int kk = 0; kk < kBN / 16; ++kk) {
                     const uint64_t bdesc = smem_desc(vaddr + kk * 2048, kHalf, 1024, kSwizzle128B);
-                    umma_ts(tmem + kColO, tmem + kColP + sb * 64 + kk * 8, bdesc, idesc_pv,
+                    umma_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + kk * 8, bdesc, idesc_pv,
                             (first && kk == 0) ? 0u : 1u);
                 }
-                umma_commit(&sm.kv_empty_v[sb]);
-                umma_commit(&sm.pv_done[sb]);
-                return true;
             };
-            bool ok = true;
+            auto wait_k = [&](uint32_t it) { return mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1); };
+            auto wait_v = [&](uint32_t it) { return mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1); };
             for (int64_t j = 0; ok; ++j, ++u_it) {
                 const int64_t unit = cta_unit(j, n_units);
                 if (unit < 0 || aborted(sm)) break;
                 int b, q, w;
                 unit_coords(u, unit, b, q, w);
-                const int n = unit_kv_tiles(u, w);
+                const int n0 = tile_kv_tiles(u, w, 0), n1 = tile_kv_tiles(u, w, 1);
                 const int qs = u_it & 1;
                 if (!mbar_wait(&sm.q_full[qs], (u_it >> 1) & 1)) { fail(sm, p, 10); break; }
                 tc_fence_after();
-                const uint32_t qaddr = smem_u32(sm.q[qs]);
-                for (int i = 0; i < n; ++i) {
+                if (!wait_k(kv_it)) { fail(sm, p, 11); break; }
+                tc_fence_after();
+                issue_s(0, kv_it);
+                issue_s(1, kv_it);
+                umma_commit(&sm.kv_empty_k[kv_it & 1]);
+                if (n1 == 1) umma_commit(&sm.q_empty);
+                for (int i = 0; i < n1; ++i) {
                     const uint32_t it = kv_it + i;
-                    if (!mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1)) { fail(sm, p, 11); ok = false; break; }
+                    if (i < n0) {
+                        ok = mbar_wait(&sm.p_full[0], (c[0] + i) & 1);
+                        if (ok && i == 0) ok = mbar_wait(&sm.o_empty[0], (u_it & 1) ^ 1);
+                        if (ok) ok = wait_v(it);
+                        if (!ok) { fail(sm, p, 12); break; }
+                        tc_fence_after();
+                        issue_pv(0, it, i == 0);
+                        if (i == n0 - 1) umma_commit(&sm.o_full[0]);
+                        if (i + 1 < n0) {
+                            if (!wait_k(it + 1)) { fail(sm, p, 13); ok = false; break; }
+                            tc_fence_after();
+                            issue_s(0, it + 1);
+                        }
+                    }
+                    ok = mbar_wait(&sm.p_full[1], (c[1] + i) & 1);
+                    if (ok && i == 0) ok = mbar_wait(&sm.o_empty[1], (u_it & 1) ^ 1);
+                    if (ok) ok = wait_v(it);
+                    if (!ok) { fail(sm, p, 14); break; }
                     tc_fence_after();
-                    issue_s(qaddr, it);
-                    if (i == n - 1) umma_commit(&sm.q_empty[qs]);
-                    if (i >= 1 && !issue_pv(it - 1, i == 1)) { fail(sm, p, 12); ok = false; break; }
+                    issue_pv(1, it, i == 0);
+                    umma_commit(&sm.kv_empty_v[it & 1]);
+                    if (i == n1 - 1) umma_commit(&sm.o_full[1]);
+                    if (i + 1 < n1) {
+                        if (!wait_k(it + 1)) { fail(sm, p, 15); ok = false; break; }
+                        tc_fence_after();
+                        issue_s(1, it + 1);
+                        umma_commit(&sm.kv_empty_k[(it + 1) & 1]);
+                        if (i + 1 == n1 - 1) umma_commit(&sm.q_empty);
+                    }
                 }
-                if (!ok) break;
-                if (!issue_pv(kv_it + n - 1, n == 1)) { fail(sm, p, 13); break; }
-                umma_commit(&sm.o_full);
-                kv_it += n;
+                kv_it += n1;
+                c[0] += n0;
+                c[1] += n1;
             }
             // Drain: all issued MMAs complete before TMEM is released.
             umma_commit(&sm.mma_drain);
             mbar_wait(&sm.mma_drain, 0);
         }
     } else if (warp == 2) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
         // ------------------------------------------------------------ row tables + Q gather
         uint32_t u_it = 0;
         int64_t armed = -1;  // last unit whose Q loads were issued
@@ -331,89 +355,95 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             int b, q, w;
             unit_coords(u, unit, b, q, w);
             const int rs = u_it & 1;
-            const uint32_t par = ((u_it >> 1) & 1) ^ 1;
-            // Row table and Q tile are double buffered: this unit's are built
-            // while the previous unit computes.
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_free[rs], par))) {
+            // The row tables are double buffered: build this unit's while the
+            // previous unit still computes, then wait for its Q tiles to be free.
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_free[rs], ((u_it >> 1) & 1) ^ 1))) {
                 if (lane == 0) fail(sm, p, 20);
                 break;
             }
-            const int w0 = w * u.W;
-            // 1. per-head slices of the window in the packed position lists
-            if (lane < u.hpg) {
-                const int jh = q * u.hpg + lane;
-                int32_t a0 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0);
-                int32_t a1 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0 + u.W);
-                if (a0 < 0 || a1 < a0 || a1 > total) {  // malformed lists: report, use none
-                    report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 41);
-                    a0 = a1 = 0;
+            for (int t = 0; t < kQT; ++t) {
+                const int w0 = (w * kQT + t) * u.W;  // first position of this tile's half-window
+                // 1. per-head slices of the half-window in the packed position lists
+                if (lane < u.hpg) {
+                    const int jh = q * u.hpg + lane;
+                    int32_t a0 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0);
+                    int32_t a1 = list_cut(u, p.head_offsets, p.head_chunk_offsets, b, jh, w0 + u.W);
+                    if (a0 < 0 || a1 < a0 || a1 > total) {  // malformed lists: report, use none
+                        report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 41);
+                        a0 = a1 = 0;
+                    }
+                    sm.cut_start[rs][t][lane] = a0;
+                    sm.cut_prefix[rs][t][lane + 1] = a1 - a0;
                 }
-                sm.cut_start[rs][lane] = a0;
-                sm.cut_prefix[rs][lane + 1] = a1 - a0;
-            }
-            __syncwarp();
-            if (lane == 0) {
-                int acc = 0;
-                sm.cut_prefix[rs][0] = 0;
-                for (int jj = 0; jj < u.hpg; ++jj) {
-                    acc = min(acc + sm.cut_prefix[rs][jj + 1], kBM);
-                    sm.cut_prefix[rs][jj + 1] = acc;
-                }
-            }
-            __syncwarp();
-            const int nrows = sm.cut_prefix[rs][u.hpg];
-            // 2. row table: position, head and gate of each routed row.  Each
-            // lane's 4 rows issue their loads together (two dependent rounds:
-            // head_pos, then the token's k (idx, gate) pairs).
-            int tt[kBM / 32], jh[kBM / 32];
-#pragma unroll
-            for (int i = 0; i < kBM / 32; ++i) {
-                const int r = lane + 32 * i;
-                tt[i] = -1;
-                jh[i] = 0;
-                if (r < nrows) {
-                    int jj = 0;
-                    while (sm.cut_prefix[rs][jj + 1] <= r) ++jj;
-                    jh[i] = q * u.hpg + jj;
-                    tt[i] = p.head_pos[sm.cut_start[rs][jj] + (r - sm.cut_prefix[rs][jj])];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < kBM / 32; ++i) {
-                const int r = lane + 32 * i;
-                float gv = 0.f;
-                if (tt[i] >= 0) {
-                    if (tt[i] < w0 || tt[i] >= min(w0 + u.W, u.T)) {  // outside the window: report, drop
-                        report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 40);
-                        tt[i] = -1;
-                    } else {
-                        const int64_t sel = (((int64_t)b * u.T + tt[i]) * u.g + q) * u.k;
-                        int sj[4];
-                        float sg[4];
-#pragma unroll
-                        for (int s2 = 0; s2 < 4; ++s2) {
-                            if (s2 < u.k) {
-                                sj[s2] = p.idx[sel + s2];
-                                sg[s2] = p.gate[sel + s2];
-                            }
-                        }
-#pragma unroll
-                        for (int s2 = 0; s2 < 4; ++s2)
-                            if (s2 < u.k && sj[s2] == jh[i]) gv = sg[s2];
+                __syncwarp();
+                if (lane == 0) {
+                    int acc = 0;
+                    sm.cut_prefix[rs][t][0] = 0;
+                    for (int jj = 0; jj < u.hpg; ++jj) {
+                        acc = min(acc + sm.cut_prefix[rs][t][jj + 1], kBM);
+                        sm.cut_prefix[rs][t][jj + 1] = acc;
                     }
                 }
-                sm.row_t[rs][r] = tt[i];
-                sm.row_j[rs][r] = jh[i];
-                sm.row_gate[rs][r] = gv;
-                // pull the row into L2 while the previous unit still computes
-                if (tt[i] >= 0) {
-                    const __nv_bfloat16* row = p.Q + (((int64_t)b * u.T + tt[i]) * u.h + jh[i]) * kD;
-                    prefetch_l2(row);
-                    prefetch_l2(row + 64);
+                __syncwarp();
+                const int nrows = sm.cut_prefix[rs][t][u.hpg];
+                // 2. row table: position, head and gate of each routed row.  Each
+                // lane's 4 rows issue their loads together (two dependent rounds:
+                // head_pos, then the token's k (idx, gate) pairs).
+                int tt[kBM / 32], jh[kBM / 32];
+#pragma unroll
+                for (int i = 0; i < kBM / 32; ++i) {
+                    const int r = lane + 32 * i;
+                    tt[i] = -1;
+                    jh[i] = 0;
+                    if (r < nrows) {
+                        int jj = 0;
+                        while (sm.cut_prefix[rs][t][jj + 1] <= r) ++jj;
+                        jh[i] = q * u.hpg + jj;
+                        tt[i] = p.head_pos[sm.cut_start[rs][t][jj] + (r - sm.cut_prefix[rs][t][jj])];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kBM / 32; ++i) {
+                    const int r = lane + 32 * i;
+                    float gv = 0.f;
+                    if (tt[i] >= 0) {
+                        if (tt[i] < w0 || tt[i] >= min(w0 + u.W, u.T)) {  // outside the window: report, drop
+                            report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereTc, 40);
+                            tt[i] = -1;
+                        } else {
+                            const int64_t sel = (((int64_t)b * u.T + tt[i]) * u.g + q) * u.k;
+                            int sj[4];
+                            float sg[4];
+#pragma unroll
+                            for (int s2 = 0; s2 < 4; ++s2) {
+                                if (s2 < u.k) {
+                                    sj[s2] = p.idx[sel + s2];
+                                    sg[s2] = p.gate[sel + s2];
+                                }
+                            }
+#pragma unroll
+                            for (int s2 = 0; s2 < 4; ++s2)
+                                if (s2 < u.k && sj[s2] == jh[i]) gv = sg[s2];
+                        }
+                    }
+                    sm.row_t[rs][t][r] = tt[i];
+                    sm.row_j[rs][t][r] = jh[i];
+                    sm.row_gate[rs][t][r] = gv;
                 }
             }
             __syncwarp();
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_empty[rs], par))) {
+            // Pull the unit's Q rows into L2 while the previous unit still computes.
+            for (int t = 0; t < kQT; ++t) {
+                for (int r = lane; r < kBM; r += 32) {
+                    const int tr = sm.row_t[rs][t][r];
+                    if (tr >= 0) {
+                        const __nv_bfloat16* row = p.Q + (((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][t][r]) * kD;
+                        prefetch_l2(row);
+                        prefetch_l2(row + 64);
+                    }
+                }
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_empty, (u_it & 1) ^ 1))) {
                 if (lane == 0) fail(sm, p, 21);
                 break;
             }
@@ -423,166 +453,162 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             // 128-byte swizzle follows the shared-memory address, so each row
             // gets its own chunk permutation.  Padding rows name an
             // out-of-range row, which the TMA zero-fills.
-            if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[rs], kTileBytes);
+            if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[rs], kQT * kTileBytes);
             __syncwarp();
             {
-                const int r0 = lane * 4;  // four rows per lane
-                int row[4];
+                const int t = lane >> 4;            // 16 lanes per tile
+                const int r0 = (lane & 15) * 8;     // 8 rows per lane: two gather4 groups
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tr = sm.row_t[rs][r0 + e];
-                    row[e] = (tr >= 0) ? (int)(((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][r0 + e]) : p.q_rows;
+                for (int gq = 0; gq < 2; ++gq) {
+                    int row[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r0 + gq * 4 + e;
+                        const int tr = sm.row_t[rs][t][r];
+                        row[e] = (tr >= 0) ? (int)(((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][t][r]) : p.q_rows;
+                    }
+                    uint8_t* dst = sm.q[t] + (r0 + gq * 4) * 128;
+                    tma_gather4_2d(&mapQ, &sm.q_full[rs], dst, 0, row[0], row[1], row[2], row[3]);
+                    tma_gather4_2d(&mapQ, &sm.q_full[rs], dst + kHalf, 64, row[0], row[1], row[2], row[3]);
                 }
-                uint8_t* dst = sm.q[rs] + r0 * 128;
-                tma_gather4_2d(&mapQ, &sm.q_full[rs], dst, 0, row[0], row[1], row[2], row[3]);
-                tma_gather4_2d(&mapQ, &sm.q_full[rs], dst + kHalf, 64, row[0], row[1], row[2], row[3]);
             }
             armed = u_it;
         }
         // Drain: the last issued Q loads land before the CTA may exit.
         if (armed >= 0) mbar_wait(&sm.q_full[armed & 1], (armed >> 1) & 1);
     } else if (warp == 3) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
         // ------------------------------------------------------------ zero fill of unselected slots
-        // The unit's window [w0, w0 + W) x heads of group q: slots whose head the
-        // token did not select are written as zeros.  Each lane owns up to 4 of
-        // the window's tokens and loads their k selections at once (one round
-        // of loads per window, not one per slot); the warp then zeroes the
-        // unselected 256-byte slots, 16 lanes per slot.
+        // The unit's window [w0, w0 + 2W) x heads of group q, one W-position half
+        // at a time: slots whose head the token did not select are written as
+        // zeros.  Each lane owns up to 4 of the half's tokens and loads their k
+        // selections at once; the warp then zeroes the unselected 256-byte
+        // slots, 16 lanes per slot.
         const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
         for (int64_t j = 0;; ++j) {
             const int64_t unit = cta_unit(j, n_units);
             if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
-            const int w0 = w * u.W;
-            const int nt = min(w0 + u.W, u.T) - w0;  // tokens in the window, <= 128
-            int sj[kBM / 32][4];
+            for (int half = 0; half < kQT; ++half) {
+                const int w0 = (w * kQT + half) * u.W;
+                const int nt = min(w0 + u.W, u.T) - w0;  // tokens in the half, <= 128
+                if (nt <= 0) break;
+                int sj[kBM / 32][4];
 #pragma unroll
-            for (int i = 0; i < kBM / 32; ++i) {
-                const int tt = lane + 32 * i;
-                const int64_t sel = (((int64_t)b * u.T + w0 + tt) * u.g + q) * u.k;
+                for (int i = 0; i < kBM / 32; ++i) {
+                    const int tt = lane + 32 * i;
+                    const int64_t sel = (((int64_t)b * u.T + w0 + tt) * u.g + q) * u.k;
 #pragma unroll
-                for (int s = 0; s < 4; ++s) sj[i][s] = (tt < nt && s < u.k) ? p.idx[sel + s] : -1;
-            }
-            uint32_t unsel[kBM / 32];
-            bool any = false;
-#pragma unroll
-            for (int i = 0; i < kBM / 32; ++i) {
-                uint32_t m = 0;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int a = sj[i][s] - q * u.hpg;  // head within the group
-                    if (a >= 0 && a < u.hpg) m |= 1u << a;
+                    for (int s = 0; s < 4; ++s) sj[i][s] = (tt < nt && s < u.k) ? p.idx[sel + s] : -1;
                 }
-                unsel[i] = (lane + 32 * i < nt) ? (~m & group_mask) : 0u;
-                any |= unsel[i] != 0u;
-            }
-            if (!__any_sync(0xffffffffu, any)) continue;
-            for (int tt = 0; tt < nt; ++tt) {
-                uint32_t un = __shfl_sync(0xffffffffu, unsel[0], tt & 31);
+                uint32_t unsel[kBM / 32];
+                bool any = false;
 #pragma unroll
-                for (int i = 1; i < kBM / 32; ++i) {
-                    const uint32_t v = __shfl_sync(0xffffffffu, unsel[i], tt & 31);
-                    if ((tt >> 5) == i) un = v;
+                for (int i = 0; i < kBM / 32; ++i) {
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const int a = sj[i][s] - q * u.hpg;  // head within the group
+                        if (a >= 0 && a < u.hpg) m |= 1u << a;
+                    }
+                    unsel[i] = (lane + 32 * i < nt) ? (~m & group_mask) : 0u;
+                    any |= unsel[i] != 0u;
                 }
-                __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + w0 + tt) * u.h + q * u.hpg) * kD;
-                while (un != 0u) {
-                    // two slots per pass: the lowest set bit for lanes 0-15, the next for 16-31
-                    const int a0 = __ffs(un) - 1;
-                    un &= un - 1u;
-                    const int a1 = (un != 0u) ? __ffs(un) - 1 : -1;
-                    if (a1 >= 0) un &= un - 1u;
-                    const int a = (lane < 16) ? a0 : a1;
-                    if (a >= 0) reinterpret_cast<uint4*>(orow + (int64_t)a * kD)[lane & 15] = make_uint4(0, 0, 0, 0);
+                if (!__any_sync(0xffffffffu, any)) continue;
+                for (int tt = 0; tt < nt; ++tt) {
+                    uint32_t un = __shfl_sync(0xffffffffu, unsel[0], tt & 31);
+#pragma unroll
+                    for (int i = 1; i < kBM / 32; ++i) {
+                        const uint32_t v = __shfl_sync(0xffffffffu, unsel[i], tt & 31);
+                        if ((tt >> 5) == i) un = v;
+                    }
+                    __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + w0 + tt) * u.h + q * u.hpg) * kD;
+                    while (un != 0u) {
+                        // two slots per pass: the lowest set bit for lanes 0-15, the next for 16-31
+                        const int a0 = __ffs(un) - 1;
+                        un &= un - 1u;
+                        const int a1 = (un != 0u) ? __ffs(un) - 1 : -1;
+                        if (a1 >= 0) un &= un - 1u;
+                        const int a = (lane < 16) ? a0 : a1;
+                        if (a >= 0) reinterpret_cast<uint4*>(orow + (int64_t)a * kD)[lane & 15] = make_uint4(0, 0, 0, 0);
+                    }
                 }
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax + epilogue
-        const int wg = (warp - 4) >> 2;    // key-column half of this warpgroup
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        // ------------------------------------------------------------ softmax + epilogue (tile t)
+        const int t = (warp - 4) >> 2;     // Q tile of this warpgroup
         const int wq = warp & 3;           // TMEM lane quarter of this warp
         const int r = wq * 32 + lane;      // routed row owned by this thread
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t o_addr = tmem + lane_off + kColO + wg * 64;
+        const uint32_t s_addr = tmem + lane_off + kColS + t * 128;
+        const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
         uint32_t ctile = 0, u_it = 0;
         for (int64_t j = 0;; ++j, ++u_it) {
             const int64_t unit = cta_unit(j, n_units);
             if (unit < 0 || aborted(sm)) break;
             int b, q, w;
             unit_coords(u, unit, b, q, w);
-            const int n = unit_kv_tiles(u, w);
+            const int n = tile_kv_tiles(u, w, t);
             const int rs = u_it & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[rs], (u_it >> 1) & 1))) {
                 if (lane == 0) fail(sm, p, 30);
                 break;
             }
-            const int t_row = sm.row_t[rs][r];
+            const int t_row = sm.row_t[rs][t][r];
             const int t_eff = (t_row >= 0) ? t_row : INT_MAX;  // padding rows: unmasked, output dropped
-            const int lo = w * u.W;                           // first position of the window
+            const int lo = (w * kQT + t) * u.W;               // first position of the tile
             float m = -INFINITY, l = 0.f;
             bool ok = true;
             for (int i = 0; i < n; ++i, ++ctile) {
-                const int sb = ctile & 1;
-                const uint32_t ph = (ctile >> 1) & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], ph))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], ctile & 1))) {
                     if (lane == 0) fail(sm, p, 31);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t s[2][32];
-                const uint32_t s_addr = tmem + lane_off + kColS + sb * 128 + wg * 64;
-                tmem_ld32(s_addr, s[0]);
-                tmem_ld32(s_addr + 32, s[1]);
+                uint32_t s[4][32];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) tmem_ld32(s_addr + cb * 32, s[cb]);
                 ld_wait_bind(s[0]);
                 ld_bind(s[1]);
-                const int kv0 = i * kBN + wg * 64;  // key index of this half's first column
-                const bool need_mask = i * kBN + kBN - 1 > lo;
+                ld_bind(s[2]);
+                ld_bind(s[3]);
+                const int kv0 = i * kBN;
+                const bool need_mask = kv0 + kBN - 1 > lo;
                 if (need_mask) {
 #pragma unroll
-                    for (int cb = 0; cb < 2; ++cb)
+                    for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             if (kv0 + cb * 32 + e > t_eff) s[cb][e] = __float_as_uint(-INFINITY);
                 }
-                // partial row max of the raw scores, then the exchange with the other half
-                float mq[2];
+                // row max of the raw scores: four independent 3-input max chains
+                float mq[4];
 #pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
+                for (int cb = 0; cb < 4; ++cb) {
                     float a0 = __uint_as_float(s[cb][0]);
 #pragma unroll
                     for (int e = 1; e < 31; e += 2)
                         a0 = fmax3(a0, __uint_as_float(s[cb][e]), __uint_as_float(s[cb][e + 1]));
                     mq[cb] = fmaxf(a0, __uint_as_float(s[cb][31]));
                 }
-                sm.xmax[sb][wg][r] = fmaxf(mq[0], mq[1]);
-                mbar_arrive(&sm.xchg[sb]);
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.xchg[sb], ph))) {
-                    if (lane == 0) fail(sm, p, 32);
-                    ok = false;
-                    break;
-                }
-                const float mx = fmaxf(sm.xmax[sb][0][r], sm.xmax[sb][1][r]) * p.scale_log2;
-                // Lazy rescaling (identical decision in both halves): keep the running
-                // max unless it grows by more than the threshold.
+                const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
+                // Lazy rescaling: keep the running max unless it grows by more than the threshold.
                 float m_use = m;
                 bool rescale = false;
                 if (mx > m + kRescaleThreshold || m == -INFINITY) {
                     m_use = mx;
                     rescale = (i > 0);
                 }
+                // S_t of this tile is complete, so O_t already holds P.V of every
+                // earlier tile (the commit that signalled s_full covers them).
                 if (__any_sync(0xffffffffu, rescale)) {
-                    // O must hold P.V of every earlier tile before it is rescaled.
-                    const uint32_t prev = ctile - 1;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[prev & 1], (prev >> 1) & 1))) {
-                        if (lane == 0) fail(sm, p, 33);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
                     const float alpha = rescale ? fast_exp2(m - m_use) : 1.0f;
 #pragma unroll 1
-                    for (int cb = 0; cb < 2; ++cb) {
+                    for (int cb = 0; cb < 4; ++cb) {
                         uint32_t o[32];
                         tmem_ld32(o_addr + cb * 32, o);
                         ld_wait_bind(o);
@@ -593,60 +619,72 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     }
                     l *= alpha;
                 }
-                // P buffer sb was last read by P.V(ctile-2), issued before S(ctile):
-                // the commit that signalled s_full covers it, so the buffer is free.
                 // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
                 // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
                 const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);
                 const uint64_t NM2 = pk2(-m_use, -m_use);
-                const uint32_t pa = tmem + lane_off + kColP + sb * 64 + wg * 32;
                 uint64_t sum2[4] = {0, 0, 0, 0};
+                if (need_mask) {
 #pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    uint32_t pk[16];
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint64_t x2 =
-                            ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2);
-                        float x0, x1, p0, p1;
-                        up2(x2, x0, x1);
-                        if (e < kPolyPairs && !need_mask) {
-                            up2(exp2_poly2(pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p0, p1);
-                        } else {
-                            p0 = fast_exp2(x0);
-                            p1 = fast_exp2(x1);
+                        for (int e = 0; e < 16; ++e) {
+                            float x0, x1;
+                            up2(ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2),
+                                x0, x1);
+                            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                            sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
+                            pk[e] = pack_bf16x2(p0, p1);
                         }
-                        sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
-                        pk[e] = pack_bf16x2(p0, p1);
+                        tmem_st16(s_addr + cb * 16, pk);
                     }
-                    tmem_st16(pa + cb * 16, pk);
+                } else {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t x2 =
+                                ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2);
+                            float p0, p1;
+                            if (e < kPolyPairs) {
+                                float x0, x1;
+                                up2(x2, x0, x1);
+                                up2(exp2_poly2(pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p0, p1);
+                            } else {
+                                float x0, x1;
+                                up2(x2, x0, x1);
+                                p0 = fast_exp2(x0);
+                                p1 = fast_exp2(x1);
+                            }
+                            sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
+                            pk[e] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(s_addr + cb * 16, pk);
+                    }
                 }
-                float sa, sb2;
-                up2(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])), sa, sb2);
-                l += sa + sb2;
+                float sa, sb;
+                up2(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])), sa, sb);
+                const float rowsum = sa + sb;
+                l += rowsum;
                 m = m_use;
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sm.p_full[sb]);
+                mbar_arrive(&sm.p_full[t]);
             }
             if (!ok) break;
-            // Epilogue: O / l * gate -> bf16 half row of O[b, t, j, :].  The row sum
-            // is the sum of the two halves' partial sums.
-            sm.xsum[wg][r] = l;
-            mbar_arrive(&sm.sum_xchg);
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.sum_xchg, u_it & 1)) ||
-                !__all_sync(0xffffffffu, mbar_wait(&sm.o_full, u_it & 1))) {
-                if (lane == 0) fail(sm, p, 35);
+            // Epilogue: O_t / l * gate -> bf16 row of O[b, t, j, :].
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], u_it & 1))) {
+                if (lane == 0) fail(sm, p, 34);
                 break;
             }
             tc_fence_after();
-            const float lt = sm.xsum[0][r] + sm.xsum[1][r];
-            const int j_row = sm.row_j[rs][r];
-            const float f = (t_row >= 0) ? sm.row_gate[rs][r] / lt : 0.f;
-            __nv_bfloat16* orow =
-                p.O + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD + wg * 64;
+            const int j_row = sm.row_j[rs][t][r];
+            const float f = (t_row >= 0) ? sm.row_gate[rs][t][r] / l : 0.f;
+            __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD;
 #pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
+            for (int cb = 0; cb < 4; ++cb) {
                 uint32_t o[32];
                 tmem_ld32(o_addr + cb * 32, o);
                 ld_wait_bind(o);
@@ -664,7 +702,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 }
             }
             tc_fence_before();
-            mbar_arrive(&sm.o_empty);
+            mbar_arrive(&sm.o_empty[t]);
             mbar_arrive(&sm.rows_free[rs]);
         }
     }
@@ -685,16 +723,27 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     if (s.k > 4 || s.h / s.g > 32) return cudaErrorNotSupported;
     UnitGeom u;
     u.B = s.B; u.T = s.T; u.h = s.h; u.g = s.g; u.k = s.k; u.hpg = s.h / s.g;
-    u.W = 32 * (4 / s.k);  // k*W <= 128 rows per unit, W a multiple of the 32-token chunk
-    u.nwin = (s.T + u.W - 1) / u.W;
+    u.W = 32 * (4 / s.k);  // k*W <= 128 rows per tile, W a multiple of the 32-token chunk
+    u.nwin = (s.T + kQT * u.W - 1) / (kQT * u.W);
     u.nchunk = gqe_chunk_count(s.T);
 
-    CUtensorMap mapK, mapV, mapQ;
+    // The setmaxnreg split needs exactly kRegsLaunch registers per thread at launch.
+    static int regs_checked = 0;
+    if (regs_checked == 0) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel);
+        if (e != cudaSuccess) return e;
+        regs_checked = (fa.numRegs == kRegsLaunch) ? 1 : -1;
+    }
+    if (regs_checked != 1) return cudaErrorNotSupported;
+
+    CUtensorMap mapK, mapV;
     const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
     const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kBN, 1};
     if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    CUtensorMap mapQ;
     const int64_t q_rows = (int64_t)s.B * s.T * s.h;
     if (q_rows >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
     {
