@@ -215,8 +215,14 @@ class Runner:
         self.attend()
 
     def launches_per_step(self):
-        route = 4  # router + compaction count / scan / scatter
-        return route + (2 if self.w.decode else 1)
+        # router (+ a separate count pass unless the tensor-core router fuses the
+        # counts: bf16, h % 8 == 0, h <= 256, d_model % 8 == 0, h/g <= 64, T % 32 == 0)
+        # + one scan-and-scatter pass; then one prefill or two decode kernels
+        w = self.w
+        fused = (w.dtype == "bf16" and w.h % 8 == 0 and w.h <= 256 and w.d_model % 8 == 0
+                 and w.h // w.g <= 64 and w.T % 32 == 0)
+        route = 2 if fused else 3
+        return route + (2 if w.decode else 1)
 
     def work(self):
         """(work units per step, unit string, scale to the unit)."""

@@ -102,6 +102,9 @@ struct RouteArgs {
 cudaError_t launch_route(const RouteArgs& a);
 bool router_tc_supported(const gqe_shape* s);
 cudaError_t launch_router_tc(const RouteArgs& a);  // a1+a2 on tensor cores (bf16)
+// True when launch_router_tc also writes RouteArgs::counts (T a multiple of
+// the 32-token chunk), so the separate count pass is skipped.
+bool router_tc_fuses_counts(const gqe_shape* s);
 
 // Library-held scratch for gqe_route_static: per-(b, head, chunk) counts,
 // at most kRouteStaticScratchBytes.  Resolves the calling thread's current

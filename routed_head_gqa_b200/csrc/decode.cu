@@ -161,53 +161,65 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T
 }
 
 // Merge the chunk partials of each (b, group, routed row), apply the gate,
-// write O[b, j, :]; zero the unselected heads.  One block per sequence.
+// write O[b, j, :]; zero the unselected heads.  One warp per (b, head j):
+// lanes hold the chunks' (max, sum) pairs, so the merged max and row sum are
+// warp reductions, and the weighted rows of the chunks are read with
+// independent loads.
+constexpr int kCombineWarps = 8;
 template <typename T, int D>
-__global__ void decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lengths,
-                                      const int32_t* __restrict__ idx, const float* __restrict__ gate,
-                                      int Lmax, int h, int g, int k, int nchunk_max, T* __restrict__ O) {
+__global__ void __launch_bounds__(32 * kCombineWarps)
+decode_combine_kernel(const float* __restrict__ part, const int32_t* __restrict__ lengths,
+                      const int32_t* __restrict__ idx, const float* __restrict__ gate, int Lmax, int h, int g,
+                      int k, int nchunk_max, T* __restrict__ O) {
     constexpr int DPL = (D + 31) / 32;
+    constexpr int kRec = PartRec<D>::kFloats;
     const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.y * kCombineWarps + (threadIdx.x >> 5);
+    if (j >= h) return;
+    const int hpg = h / g, grp = j / hpg;
+    T* o = O + ((int64_t)b * h + j) * D;
+    // the routed row of head j in this sequence, if any (first match, as the router never repeats a head)
+    int r = -1;
+    for (int rr = k - 1; rr >= 0; --rr)
+        if (idx[((int64_t)b * g + grp) * k + rr] == j) r = rr;
+    if (r < 0) {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e)
+            if (e * 32 + lane < D) o[e * 32 + lane] = Elem<T>::from_f(0.f);
+        return;
+    }
     const int L = min(max(lengths[b], 1), Lmax);
     const int nc = (L + kDecodeChunk - 1) / kDecodeChunk;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const int hpg = h / g;
-    // Routed rows.
-    for (int pr = warp; pr < g * k; pr += nwarps) {
-        const int grp = pr / k, r = pr % k;
-        const int64_t sel = ((int64_t)b * g + grp) * k + r;
-        const int j = idx[sel];
-        if (j < grp * hpg || j >= (grp + 1) * hpg) continue;  // out of group: skip
-        const float gv = gate[sel];
-        float M = -INFINITY;
-        for (int c = 0; c < nc; ++c)
-            M = fmaxf(M, part[((((int64_t)b * nchunk_max + c) * g + grp) * k + r) * PartRec<D>::kFloats + D]);
-        float Ls = 0.f, acc[DPL];
+    const int64_t stride = (int64_t)g * k * kRec;  // from chunk c to chunk c+1
+    const float* rec0 = part + (((int64_t)b * nchunk_max * g + grp) * k + r) * kRec;
+    float M = -INFINITY;
+    for (int c = lane; c < nc; c += 32) M = fmaxf(M, rec0[c * stride + D]);
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-        for (int c = 0; c < nc; ++c) {
-            const float* rec = part + ((((int64_t)b * nchunk_max + c) * g + grp) * k + r) * PartRec<D>::kFloats;
-            const float w = fast_exp2(rec[D] - M);
-            Ls = fmaf(rec[D + 1], w, Ls);
+    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+    float Ls = 0.f, acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    for (int c0 = 0; c0 < nc; c0 += 32) {
+        const int c = c0 + lane;
+        const float wl = (c < nc) ? fast_exp2(rec0[c * stride + D] - M) : 0.f;
+        Ls = (c < nc) ? fmaf(rec0[c * stride + D + 1], wl, Ls) : Ls;
+        const int n = min(32, nc - c0);
+#pragma unroll 4
+        for (int i = 0; i < n; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+            const float* rec = rec0 + (c0 + i) * stride;
 #pragma unroll
             for (int e = 0; e < DPL; ++e)
                 if (e * 32 + lane < D) acc[e] = fmaf(rec[e * 32 + lane], w, acc[e]);
         }
-        const float f = gv / Ls;
-        T* o = O + ((int64_t)b * h + j) * D;
+    }
 #pragma unroll
-        for (int e = 0; e < DPL; ++e)
-            if (e * 32 + lane < D) o[e * 32 + lane] = Elem<T>::from_f(acc[e] * f);
-    }
-    // Unselected heads.
-    for (int j = warp; j < h; j += nwarps) {
-        const int grp = j / hpg;
-        bool hit = false;
-        for (int r = 0; r < k; ++r) hit |= (idx[((int64_t)b * g + grp) * k + r] == j);
-        if (hit) continue;
-        T* o = O + ((int64_t)b * h + j) * D;
-        for (int e = lane; e < D; e += 32) o[e] = Elem<T>::from_f(0.f);
-    }
+    for (int d = 16; d > 0; d >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, d);
+    const float f = gate[((int64_t)b * g + grp) * k + r] / Ls;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e)
+        if (e * 32 + lane < D) o[e * 32 + lane] = Elem<T>::from_f(acc[e] * f);
 }
 
 template <typename T, int D, int KR>
@@ -220,8 +232,9 @@ cudaError_t launch_typed(const DecodeArgs& a) {
         nchunk_max, a.partials);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    decode_combine_kernel<T, D><<<s.B, 256, 0, a.stream>>>(a.partials, a.lengths, a.idx, a.gate, a.Lmax, s.h,
-                                                          s.g, s.k, nchunk_max, (T*)a.O);
+    dim3 cgrid(s.B, (s.h + kCombineWarps - 1) / kCombineWarps);
+    decode_combine_kernel<T, D><<<cgrid, 32 * kCombineWarps, 0, a.stream>>>(
+        a.partials, a.lengths, a.idx, a.gate, a.Lmax, s.h, s.g, s.k, nchunk_max, (T*)a.O);
     return cudaGetLastError();
 }
 

@@ -109,8 +109,10 @@ router_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __r
     }
 }
 
-// Compaction pass 1/3: per (b, chunk of 32 tokens, head) the number of tokens
-// routed to the head.  One warp per (b, chunk, group); lane = token.
+// Compaction pass 1: per (b, chunk of 32 tokens, head) the number of tokens
+// routed to the head.  One warp per (b, chunk, group); lane = token.  The
+// tensor-core router computes the same counts in its epilogue when T is a
+// multiple of the chunk; this pass serves the other inputs.
 __global__ void compact_count_kernel(const int32_t* __restrict__ idx, int T, int h, int g, int k,
                                      int nchunk, int32_t* __restrict__ counts) {
     const int c = blockIdx.x, b = blockIdx.y;
@@ -130,62 +132,67 @@ __global__ void compact_count_kernel(const int32_t* __restrict__ idx, int T, int
     }
 }
 
-// Compaction pass 2/3: per batch, exclusive prefix sum over (head, chunk) in
-// head-major order -> absolute head_pos offsets.  One block per batch.
-__global__ void compact_scan_kernel(const int32_t* __restrict__ counts, int B, int T, int h, int g,
-                                    int k, int nchunk, int32_t* __restrict__ head_offsets,
-                                    int32_t* __restrict__ head_chunk_offsets) {
-    __shared__ int32_t warp_sums[32];
-    __shared__ int32_t carry;
-    const int b = blockIdx.x;
-    const int n = h * nchunk;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t base = (int64_t)b * T * g * k;
-    if (threadIdx.x == 0) carry = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-        const int i = i0 + threadIdx.x;
-        const int v = (i < n) ? counts[(int64_t)b * n + i] : 0;
-        int incl = v;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += y;
-        }
-        if (lane == 31) warp_sums[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int nw = blockDim.x >> 5;
-            int ws = (lane < nw) ? warp_sums[lane] : 0;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, ws, d);
-                if (lane >= d) ws += y;
-            }
-            if (lane < nw) warp_sums[lane] = ws;  // inclusive over warps
-        }
-        __syncthreads();
-        const int warp_prefix = (warp > 0) ? warp_sums[warp - 1] : 0;
-        const int excl = carry + warp_prefix + incl - v;
-        if (i < n) {
-            const int32_t off = (int32_t)(base + excl);
-            head_chunk_offsets[(int64_t)b * n + i] = off;
-            if (i % nchunk == 0) head_offsets[(int64_t)b * h + i / nchunk] = off;
-        }
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = excl + v;
-        __syncthreads();
-    }
-    if (b == B - 1 && threadIdx.x == 0) head_offsets[(int64_t)B * h] = (int32_t)((int64_t)B * T * g * k);
-}
-
-// Compaction pass 3/3: write positions.  Same tiling as pass 1; a lane's rank
-// within its head's chunk is the popcount of the ballot below it.
-__global__ void compact_scatter_kernel(const int32_t* __restrict__ idx, int T, int h, int g, int k,
-                                       int nchunk, const int32_t* __restrict__ head_chunk_offsets,
-                                       int32_t* __restrict__ head_pos) {
+// Compaction pass 2: write positions, with the offsets each block needs.
+// Block (chunk c, batch b) first derives, from the batch's counts, the
+// head-major exclusive prefix of every (head, c): the sum of all earlier
+// heads' totals plus head j's counts in chunks before c (one warp per head,
+// lanes striding over chunks; then one warp scans the head totals).  The
+// counts of a batch are a few KB, so every block re-reading them costs less
+// than a separate scan launch.  Then it scatters as pass 1 counted: a lane's
+// rank within its head's chunk is the popcount of the ballot below it.
+__global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int B, int T, int h, int g, int k,
+                                            int nchunk, const int32_t* __restrict__ counts,
+                                            int32_t* __restrict__ head_offsets,
+                                            int32_t* __restrict__ head_chunk_offsets,
+                                            int32_t* __restrict__ head_pos) {
+    extern __shared__ int32_t sh[];  // [h] head totals -> head bases, [h] prefix within head
+    int32_t* total = sh;
+    int32_t* before = sh + h;
     const int c = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int32_t* cnt = counts + (int64_t)b * h * nchunk;
+    for (int j = warp; j < h; j += nwarps) {
+        int tot = 0, pre = 0;
+        for (int cc = lane; cc < nchunk; cc += 32) {
+            const int v = cnt[(int64_t)j * nchunk + cc];
+            tot += v;
+            if (cc < c) pre += v;
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) {
+            tot += __shfl_xor_sync(0xffffffffu, tot, d);
+            pre += __shfl_xor_sync(0xffffffffu, pre, d);
+        }
+        if (lane == 0) {
+            total[j] = tot;
+            before[j] = pre;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int j0 = 0; j0 < h; j0 += 32) {
+            const int j = j0 + lane;
+            const int v = (j < h) ? total[j] : 0;
+            int incl = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            if (j < h) total[j] = carry + incl - v;  // exclusive: head j's base within the batch
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncthreads();
+    const int64_t base = (int64_t)b * T * g * k;  // every batch holds exactly T*g*k entries
+    for (int j = threadIdx.x; j < h; j += blockDim.x) {
+        const int32_t off = (int32_t)(base + total[j] + before[j]);
+        head_chunk_offsets[((int64_t)b * h + j) * nchunk + c] = off;
+        if (c == 0) head_offsets[(int64_t)b * h + j] = off;
+    }
+    if (b == B - 1 && c == 0 && threadIdx.x == 0) head_offsets[(int64_t)B * h] = (int32_t)((int64_t)B * T * g * k);
+
     const int hpg = h / g;
     const int t = c * kChunk + lane;
     const unsigned below = (1u << lane) - 1u;
@@ -197,10 +204,7 @@ __global__ void compact_scatter_kernel(const int32_t* __restrict__ idx, int T, i
             bool hit = false;
             for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
             const unsigned ball = __ballot_sync(0xffffffffu, hit);
-            if (hit) {
-                const int32_t off = head_chunk_offsets[((int64_t)b * h + j) * nchunk + c];
-                head_pos[off + __popc(ball & below)] = t;
-            }
+            if (hit) head_pos[base + total[j] + before[j] + __popc(ball & below)] = t;
         }
     }
 }
@@ -236,11 +240,11 @@ cudaError_t launch_route(const RouteArgs& a) {
     const int nchunk = gqe_chunk_count(s.T);
     const int cwarps = s.g < 8 ? s.g : 8;
     dim3 cgrid(nchunk, s.B);
-    compact_count_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk, a.counts);
-    compact_scan_kernel<<<s.B, 1024, 0, a.stream>>>(a.counts, s.B, s.T, s.h, s.g, s.k, nchunk,
-                                                   a.head_offsets, a.head_chunk_offsets);
-    compact_scatter_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk,
-                                                                a.head_chunk_offsets, a.head_pos);
+    if (!(router_tc_supported(a.s) && router_tc_fuses_counts(a.s)))
+        compact_count_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk, a.counts);
+    const int swarps = 8;  // warps of the scan: one head per warp and round
+    compact_scan_scatter_kernel<<<cgrid, 32 * swarps, 2 * s.h * sizeof(int32_t), a.stream>>>(
+        a.idx, s.B, s.T, s.h, s.g, s.k, nchunk, a.counts, a.head_offsets, a.head_chunk_offsets, a.head_pos);
     return cudaGetLastError();
 }
 
