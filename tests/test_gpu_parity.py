@@ -29,6 +29,14 @@ SMALL_BF16 = [
     C("bf16_T33", B=2, T=33, d_model=64, h=8, g=2, d_h=128, k=2, seed=19),
     C("bf16_T129", B=1, T=129, d_model=64, h=8, g=2, d_h=128, k=1, seed=20),
     C("bf16_skew", B=1, T=520, d_model=96, h=16, g=8, d_h=128, k=1, head0_bias=1.0, seed=21),
+    # Router and compaction shapes: d_model split over 4-CTA clusters (8 k-blocks,
+    # 2 token tiles); 64, 128 and 256 heads (one, two and four 64-head MMA blocks;
+    # a head scan over several 32-head rounds); T not a multiple of 32 (counts from
+    # the separate pass).
+    C("bf16_route_ks4", B=1, T=256, d_model=512, h=32, g=8, d_h=128, k=2, seed=22),
+    C("bf16_h64", B=2, T=96, d_model=256, h=64, g=8, d_h=128, k=2, seed=23),
+    C("bf16_h128", B=1, T=64, d_model=128, h=128, g=16, d_h=128, k=1, seed=24),
+    C("bf16_h256_T40", B=1, T=40, d_model=128, h=256, g=32, d_h=128, k=3, seed=25),
 ]
 SMALL_F32 = [
     W["tiny_f32"],
