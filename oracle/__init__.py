@@ -93,7 +93,11 @@ class Oracle:
         lib.oracle_compact.argtypes = [i32, i32, i32, i32, i32, P, P, P]
         lib.oracle_attn_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, i32]
         lib.oracle_decode.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32]
-        for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode):
+        lib.oracle_shared_rows.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
+        lib.oracle_group_slots_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, P,
+                                                i32]
+        for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
+                  lib.oracle_shared_rows, lib.oracle_group_slots_rows):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -159,6 +163,52 @@ class Oracle:
             raise ValueError(f"oracle_attn_rows failed ({rc})")
         return out
 
+    def shared_rows(self, Qs, K, V, kv_group: int, rows=None, n_threads=None):
+        """Shared-head output (float64 [n_rows, d_h]) for Qs [B, T, d_h] (or
+        [B, T, 1, d_h]) attending causally to KV group kv_group of K/V [B, T, g, d_h]."""
+        qa, dt = _as_input(Qs)
+        ka, dk = _as_input(K)
+        va, dv = _as_input(V)
+        if not (dt == dk == dv):
+            raise TypeError("Qs, K, V must share a dtype")
+        B, T, g, d_h = ka.shape
+        qa = qa.reshape(B, T, d_h)
+        if rows is None:
+            rows = np.arange(B * T, dtype=np.int64)
+        ra = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+        out = np.empty((ra.shape[0], d_h), np.float64)
+        rc = self.lib.oracle_shared_rows(B, T, g, d_h, dt, int(kv_group), _ptr(qa), _ptr(ka), _ptr(va),
+                                         ra.shape[0], _ptr(ra), _ptr(out), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_shared_rows failed ({rc})")
+        return out
+
+    def group_slots_rows(self, Q, K, V, idx, gate, rows=None, n_threads=None):
+        """Per-group output slots for token rows b*T + t: (cat float64
+        [n_rows, g, k, d_h], the selected heads' ungated outputs in selection
+        order; wsum float64 [n_rows, g, d_h], their gate-weighted sum)."""
+        qa, dt = _as_input(Q)
+        ka, dk = _as_input(K)
+        va, dv = _as_input(V)
+        if not (dt == dk == dv):
+            raise TypeError("Q, K, V must share a dtype")
+        B, T, h, d_h = qa.shape
+        g = ka.shape[2]
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        ga = np.ascontiguousarray(gate, dtype=np.float64)
+        k = ia.shape[-1]
+        if rows is None:
+            rows = np.arange(B * T, dtype=np.int64)
+        ra = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+        cat = np.empty((ra.shape[0], g, k, d_h), np.float64)
+        wsum = np.empty((ra.shape[0], g, d_h), np.float64)
+        rc = self.lib.oracle_group_slots_rows(B, T, h, g, d_h, k, dt, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ia),
+                                              _ptr(ga), ra.shape[0], _ptr(ra), _ptr(cat), _ptr(wsum),
+                                              _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_group_slots_rows failed ({rc})")
+        return cat, wsum
+
     def attn(self, Q, K, V, idx, gate, n_threads=None):
         """Full GQE output O [B, T, h, d_h] (float64)."""
         B, T, h, d_h = tuple(Q.shape)
@@ -214,3 +264,11 @@ def attn(*a, **kw):
 
 def decode(*a, **kw):
     return default().decode(*a, **kw)
+
+
+def shared_rows(*a, **kw):
+    return default().shared_rows(*a, **kw)
+
+
+def group_slots_rows(*a, **kw):
+    return default().group_slots_rows(*a, **kw)

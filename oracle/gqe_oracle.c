@@ -35,6 +35,14 @@
  *  - Decode.  One new query per sequence at position L_b - 1 against a cache
  *    holding keys 0 .. L_b - 1 of that sequence (the KV cache of the GQA
  *    pages, which stays dense under GQE).
+ *  - Output construction (same GQE page, "Construction de la Sortie"): per
+ *    group, the outputs of the k selected experts are concatenated (here in
+ *    selection order, ungated), a weighted sum of those outputs with the
+ *    renormalised router probabilities forms one more slot, and one extra
+ *    attention head is computed for every token whatever the routing (the
+ *    shared head).  The page names no KV head for the shared head; the reading
+ *    used here: its own query rows attend, causally, to one KV group chosen by
+ *    the caller.
  */
 #include <math.h>
 #include <stdint.h>
@@ -281,6 +289,89 @@ int oracle_decode(int B, int Lmax, int h, int g, int d_h, int k, int dtype,
         }
         free(scores);
         free(o);
+    }
+    return err;
+}
+
+/*
+ * Shared head: one query head computed for every token, attending causally to
+ * KV group kv_group.
+ * Qs [B, T, d_h], K/V [B, T, g, d_h] (dtype); rows [n_rows]: b*T + t
+ * Os_rows [n_rows, d_h] out (double)
+ */
+int oracle_shared_rows(int B, int T, int g, int d_h, int dtype, int kv_group,
+                       const void* Qs, const void* K, const void* V,
+                       int64_t n_rows, const int64_t* rows, double* Os_rows, int n_threads) {
+    if (B < 0 || T < 1 || g < 1 || d_h < 1 || kv_group < 0 || kv_group >= g) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * T) return 1;
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)T);
+        if (!scores) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n_rows; ++r) {
+                const int64_t bt = rows[r];
+                const int64_t b = bt / T, t = bt % T;
+                const size_t kv_base = ((size_t)b * T * g + kv_group) * d_h;
+                attend_one(Qs, (size_t)bt * d_h, K, V, kv_base, (size_t)g * d_h, t + 1, d_h, dtype,
+                           scores, Os_rows + (size_t)r * d_h);
+            }
+        }
+        free(scores);
+    }
+    return err;
+}
+
+/*
+ * Group slots of the layer output for a list of token rows.
+ * Q [B, T, h, d_h], K/V [B, T, g, d_h] (dtype); idx/gate [B, T, g, k]
+ * cat_rows  [n_rows, g, k, d_h] out (double): the attention output of the
+ *           selected head idx[b,t,q,r] in slot (q, r), not gated
+ * wsum_rows [n_rows, g, d_h] out (double): sum_r gate[b,t,q,r] * cat(q, r)
+ */
+int oracle_group_slots_rows(int B, int T, int h, int g, int d_h, int k, int dtype,
+                            const void* Q, const void* K, const void* V,
+                            const int32_t* idx, const double* gate,
+                            int64_t n_rows, const int64_t* rows, double* cat_rows,
+                            double* wsum_rows, int n_threads) {
+    if (B < 0 || T < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * T) return 1;
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)T);
+        if (!scores) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n_rows; ++r) {
+                const int64_t bt = rows[r];
+                const int64_t b = bt / T, t = bt % T;
+                for (int q = 0; q < g; ++q) {
+                    double* ws = wsum_rows + ((size_t)r * g + q) * d_h;
+                    for (int d = 0; d < d_h; ++d) ws[d] = 0.0;
+                    for (int s = 0; s < k; ++s) {
+                        const size_t sel = ((size_t)bt * g + q) * k + s;
+                        const int j = idx[sel];
+                        double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;
+                        const size_t kv_base = ((size_t)b * T * g + q) * d_h;
+                        attend_one(Q, ((size_t)bt * h + j) * d_h, K, V, kv_base, (size_t)g * d_h, t + 1,
+                                   d_h, dtype, scores, slot);
+                        for (int d = 0; d < d_h; ++d) ws[d] += gate[sel] * slot[d];
+                    }
+                }
+            }
+        }
+        free(scores);
     }
     return err;
 }

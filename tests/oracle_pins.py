@@ -371,8 +371,78 @@ def check_active_heads_golden(o):
     assert (nonzero == routed).all(), f"nonzero head slots per token {set(nonzero.ravel())} != {routed}"
 
 
+# --------------------------------------------------------------------------
+# Output construction: shared head and per-group slots
+# --------------------------------------------------------------------------
+
+def check_shared_head_closed_forms(o):
+    """The shared head attends causally to the chosen KV group only."""
+    B, T, g, d = 2, 7, 3, 8
+    kv = 2  # not group 0: the other groups' V differ, so a wrong group fails
+    Qs = _f32((B, T, d), 70)
+    V = _f32((B, T, g, d), 71)
+    Vd = V.astype(np.float64)
+    # K = 0: uniform weights over s <= t -> running mean of the group's V
+    Os = o.shared_rows(Qs, np.zeros((B, T, g, d), np.float32), V, kv).reshape(B, T, d)
+    run_mean = np.cumsum(Vd[:, :, kv], axis=1) / np.arange(1, T + 1)[None, :, None]
+    assert np.allclose(Os, run_mean, atol=1e-13), "shared head, K = 0"
+    # T = 1: the token's own V row
+    O1 = o.shared_rows(Qs[:, :1], _f32((B, 1, g, d), 72), V[:, :1], kv).reshape(B, d)
+    assert np.allclose(O1, Vd[:, 0, kv], atol=1e-15), "shared head, T = 1"
+    # one dominant key at s* = 3 in the chosen group: rows t >= 3 return V[s*]
+    Qd = np.zeros((B, T, d), np.float32)
+    Qd[..., 1] = 30.0
+    Kd = np.zeros((B, T, g, d), np.float32)
+    Kd[:, 3, kv, 1] = 30.0
+    Od = o.shared_rows(Qd, Kd, V, kv).reshape(B, T, d)
+    for t in range(T):
+        want = Vd[:, 3, kv] if t >= 3 else run_mean[:, t]
+        assert np.allclose(Od[:, t], want, atol=1e-12), f"shared head, dominant key t={t}"
+
+
+def check_group_slots(o):
+    """Each head's query dominates one key, so its attention output is exactly
+    that key's V row (the other weights underflow to zero in double); the
+    concatenated slots must follow the selection order and the weighted sum
+    must pair each slot with its own gate."""
+    B, T, h, g, d, k = 1, 4, 4, 2, 4, 2
+    hpg = h // g
+    key_of_head = [3, 1, 0, 2]
+    K = np.zeros((B, T, g, d), np.float32)
+    for s in range(T):
+        K[0, s, :, s] = 40.0
+    Q = np.zeros((B, T, h, d), np.float32)
+    for j in range(h):
+        Q[0, :, j, key_of_head[j]] = 40.0
+    V = _f32((B, T, g, d), 73)
+    Vd = V.astype(np.float64)
+    idx = np.zeros((B, T, g, k), np.int32)
+    gate = np.zeros((B, T, g, k), np.float64)
+    for t in range(T):
+        for q_ in range(g):
+            order = [q_ * hpg + 1, q_ * hpg] if (t + q_) % 2 == 0 else [q_ * hpg, q_ * hpg + 1]
+            idx[0, t, q_] = order
+            gate[0, t, q_] = [0.7, 0.3] if t % 2 == 0 else [0.6, 0.4]
+    t = T - 1  # every key visible
+    cat, wsum = o.group_slots_rows(Q, K, V, idx, gate, rows=[t])
+    for q_ in range(g):
+        want_w = np.zeros(d)
+        for r in range(k):
+            j = idx[0, t, q_, r]
+            want = Vd[0, key_of_head[j], q_]
+            assert np.allclose(cat[0, q_, r], want, atol=1e-12), f"slot (q={q_}, r={r})"
+            want_w += gate[0, t, q_, r] * want
+        assert np.allclose(wsum[0, q_], want_w, atol=1e-12), f"weighted sum q={q_}"
+    # T = 1: every selected head sees only its own token
+    cat1, wsum1 = o.group_slots_rows(Q[:, :1], K[:, :1], V[:, :1], idx[:, :1], gate[:, :1], rows=[0])
+    for q_ in range(g):
+        assert np.allclose(cat1[0, q_], Vd[0, 0, q_][None, :], atol=1e-15)
+        assert np.allclose(wsum1[0, q_], Vd[0, 0, q_] * gate[0, 0, q_].sum(), atol=1e-15)
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
+    check_shared_head_closed_forms, check_group_slots,
 ]

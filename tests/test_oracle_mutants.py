@@ -29,6 +29,14 @@ MUTANTS = [
     ("unselected_heads_not_zero", "for (int i = 0; i < h * d_h; ++i) out[i] = 0.0;", "for (int i = 0; i < h * d_h; ++i) out[i] = 1e-3;"),
     ("transposed_qk_index", "load_elem(K, kr + d, dtype)", "load_elem(K, kv_base + (size_t)d * kv_row_stride + (size_t)s % (size_t)d_h, dtype)"),
     ("compact_strided_group", "const int q = j / hpg;", "const int q = j % g;"),
+    ("shared_head_group_0", "const size_t kv_base = ((size_t)b * T * g + kv_group) * d_h;",
+     "const size_t kv_base = ((size_t)b * T * g + 0) * d_h;"),
+    ("shared_head_sees_all_keys", "(size_t)g * d_h, t + 1, d_h, dtype,\n                           scores, Os_rows",
+     "(size_t)g * d_h, T, d_h, dtype,\n                           scores, Os_rows"),
+    ("weighted_sum_ungated", "for (int d = 0; d < d_h; ++d) ws[d] += gate[sel] * slot[d];",
+     "for (int d = 0; d < d_h; ++d) ws[d] += slot[d];"),
+    ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
+     "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
 
 _CHILD = r"""
