@@ -315,6 +315,72 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
     return res
 
 
+def time_output_construction(w, steps, warmup, peaks, peak_kind):
+    """The GQE output construction on the workload's shapes, each call timed
+    alone with CUDA events (L2 flushed before each call, outside the events):
+    the always-active shared head (one dense causal head over KV group 0, on
+    the routed prefill's tensor-core kernel) and the per-group slots
+    (concatenated expert outputs + gate-weighted sum, HBM-bound)."""
+    from routed_head_gqa_b200 import metrics
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    r = Runner(w, dev)
+    g = r.g
+    r.step()
+    Qs = gqe_synth.make_shared_query(w).to(dev)
+    Os = torch.empty((w.B, w.T, w.d_h), dtype=w.torch_dtype, device=dev)
+    cat = torch.empty((w.B, w.T, w.g, w.k, w.d_h), dtype=w.torch_dtype, device=dev)
+    wsum = torch.empty((w.B, w.T, w.g, w.d_h), dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def shared():
+        g.gqe_attn_shared_head(r.shape, Qs, r.d["K"], r.d["V"], 0, Os, r.buf.workspace)
+
+    def slots():
+        g.gqe_group_slots(r.shape, r.buf.O, r.buf.idx, r.buf.gate, cat, wsum)
+
+    def timed(fn):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+    sh_ms = timed(shared)
+    sl_ms = timed(slots)
+    st = r.buf.status()
+    if st != 0:
+        raise RuntimeError(f"device status {g.gqe_status_string(st)} in the output construction")
+    sh_flops = 4.0 * w.d_h * w.B * w.T * (w.T + 1) / 2  # one head, causal
+    el = 2 if w.dtype == "bf16" else 4
+    rows = w.B * w.T * w.g * w.k
+    sl_bytes = float(rows * w.d_h * el * 2 + w.B * w.T * w.g * w.d_h * el + rows * 8)  # O rows in, cat + wsum out
+    sh_tf = sh_flops / (sh_ms * 1e-3) * 1e-12
+    sl_gbs = sl_bytes / (sl_ms * 1e-3) * 1e-9
+    del r, flush
+    torch.cuda.empty_cache()
+    return {
+        "shared_head": {"ms": sh_ms, "value": sh_tf, "unit": "TFLOP/s", "flops": sh_flops,
+                        "roofline": {"bound": "tensor", "achieved": round(sh_tf, 1), "peak": peaks["bf16_tflops"],
+                                     "unit": "TFLOP/s", "frac": round(sh_tf / peaks["bf16_tflops"], 4),
+                                     "peak_source": f"bf16_tflops burst ({peak_kind})",
+                                     "kernel": "gqe_attn_shared_head (prefill_tc_kernel, identity routing)"}},
+        "group_slots": {"ms": sl_ms, "value": sl_gbs, "unit": "GB/s", "bytes": sl_bytes,
+                        "roofline": {"bound": "hbm", "achieved": round(sl_gbs, 1), "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": round(sl_gbs / peaks["hbm_gbs"], 4),
+                                     "peak_source": f"hbm_gbs ({peak_kind})",
+                                     "kernel": "gqe_group_slots (group_slots_kernel)"}},
+        "shape": w.describe(),
+    }
+
+
 def time_e2e(r, steps, ws, work, scale, unit):
     """Same metric through the public API with host buffers: every step copies
     its inputs from pinned host memory to the device and the output back."""
@@ -475,6 +541,9 @@ def main():
             secondary[name] = {"value": r2["value"], "unit": r2["unit"], "ms_per_step": r2["ms_per_step"],
                                "attn_ms": r2["attn_ms"], "route_ms": r2["route_ms"], "roofline": r2["roofline"],
                                "shape": sw.describe()}
+    output_construction = None
+    if not args.no_secondary and args.workload == PRIMARY:
+        output_construction = time_output_construction(w, max(5, args.steps // 2), 3, peaks, peak_kind)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)
@@ -493,6 +562,8 @@ def main():
         }
         if secondary:
             line["workloads"] = secondary
+        if output_construction:
+            line["output_construction"] = output_construction
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist

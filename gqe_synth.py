@@ -141,6 +141,14 @@ def make_inputs(w: Workload):
     return out
 
 
+def make_shared_query(w: Workload):
+    """Query rows of the always-active shared head, Qs [B, T, d_h]: N(0, 1) in
+    the workload's dtype, from their own seeded generator (seed + 7919), so the
+    other inputs are unchanged."""
+    gen = torch.Generator().manual_seed(w.seed + 7919)
+    return _normal((w.B, w.T, w.d_h), gen).to(w.torch_dtype)
+
+
 def sample_rows(w: Workload, n: int, seed: int = 1234):
     """A seeded sample of n flattened token rows (b*T + t) that always includes
     the last position of every sequence and the first position of batch 0."""

@@ -182,6 +182,57 @@ gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cach
                            const int32_t* idx, const float* gate, void* O, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/*
+ * gqe_attn_shared_head -- the always-active shared head of the GQE layer.
+ *
+ * One extra attention head computed for every token whatever the routing
+ * (gist.science summary, "Construction de la Sortie", "Tete Partagee
+ * Toujours Active").  The page does not say which KV head it attends to; this
+ * library's reading: its own query rows attend causally to KV group kv_group
+ * of the layer's dense K/V:
+ *   Os[b,t,:] = sum_{s <= t} softmax_s(Qs[b,t,:] . K[b,s,kv_group,:] / sqrt(d_h)) V[b,s,kv_group,:]
+ *
+ *   s            the layer's shape (B, T, g, d_h, dtype are used; h and k
+ *                only in the shape checks)
+ *   Qs [B, T, d_h]                     device, dtype
+ *   K/V [B, T, g, d_h]                 device, dtype (the routed prefill's K/V)
+ *   kv_group     0 <= kv_group < g, else GQE_ERR_INVALID_ARGUMENT
+ *   Os [B, T, d_h]                     device, dtype, out
+ *   workspace    at least gqe_workspace_bytes(s, 0) bytes; the call writes
+ *                identity routing tables of the one head into it, so calls
+ *                sharing a workspace must be ordered on one stream
+ * Implemented cases: as gqe_attn_prefill (bf16 with d_h = 128 on the tensor
+ * cores, the same kernel as the routed heads; fp32 with d_h in {32, 64, 128}).
+ */
+gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* K, const void* V, int kv_group,
+                                void* Os, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_group_slots -- the per-group output slots of the GQE layer.
+ *
+ * Per group, the outputs of the k selected experts are concatenated and a
+ * weighted sum of them with the renormalised router probabilities forms one
+ * more slot (gist.science summary, "Construction de la Sortie": "Concatenation
+ * Forte", "Somme Ponderee Renormalisee").  Both are built from the gated
+ * output of gqe_attn_prefill (or gqe_attn_decode with T = 1):
+ *   O_cat[b,t,q,r,:] = O[b,t,idx[b,t,q,r],:] / gate[b,t,q,r]   (the expert's
+ *                      ungated output, in selection order; 0 if the gate
+ *                      underflowed to 0)
+ *   O_wsum[b,t,q,:]  = sum_r O[b,t,idx[b,t,q,r],:] = sum_r gate * o
+ * A selection outside its group (not produced by gqe_route) contributes 0.
+ *
+ *   O [B, T, h, d_h]                   device, dtype (gated routed output)
+ *   idx, gate [B, T, g, k]             device, as written by gqe_route
+ *   O_cat [B, T, g, k, d_h]            device, dtype, out, or NULL
+ *   O_wsum [B, T, g, d_h]              device, dtype, out, or NULL
+ * At least one output must be non-NULL; O, O_cat and O_wsum 16-byte aligned
+ * (else GQE_ERR_INVALID_ARGUMENT).  d_h in {32, 64, 128}; bf16 or fp32.
+ * In bf16, O_cat carries the rounding of O and of the division (relative
+ * error about 2^-8).
+ */
+gqe_status gqe_group_slots(const gqe_shape* s, const void* O, const int32_t* idx, const float* gate, void* O_cat,
+                           void* O_wsum, void* stream);
+
 /* Synchronise `stream`, read the workspace status word, reset it to zero and
  * return it (GQE_OK when no kernel reported a failure). */
 gqe_status gqe_get_device_status(void* workspace, void* stream);

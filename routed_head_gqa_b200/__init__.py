@@ -27,7 +27,8 @@ GQE_F32 = 0
 GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
-            "gqe_attn_prefill", "gqe_attn_decode", "gqe_get_device_status", "gqe_status_string"]
+            "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_shared_head", "gqe_group_slots",
+            "gqe_get_device_status", "gqe_status_string"]
 
 
 class GqeShape(ctypes.Structure):
@@ -65,11 +66,13 @@ def _load():
     lib.gqe_route_static.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.gqe_attn_prefill.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_shared_head.argtypes = [S, _P, _P, _P, _I, _P, _P, _SZ, _P]
+    lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
-              "gqe_get_device_status"):
+              "gqe_attn_shared_head", "gqe_group_slots", "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -161,6 +164,17 @@ def gqe_attn_decode(shape, q, K_cache, V_cache, Lmax, lengths, idx, gate, O, wor
     _check("gqe_attn_decode", _lib.gqe_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache),
                                                    int(Lmax), _ptr(lengths), _ptr(idx), _ptr(gate), _ptr(O),
                                                    _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def gqe_attn_shared_head(shape, Qs, K, V, kv_group, Os, workspace, stream=None) -> None:
+    _check("gqe_attn_shared_head", _lib.gqe_attn_shared_head(ctypes.byref(shape), _ptr(Qs), _ptr(K), _ptr(V),
+                                                             int(kv_group), _ptr(Os), _ptr(workspace),
+                                                             _nbytes(workspace), _stream(stream)))
+
+
+def gqe_group_slots(shape, O, idx, gate, O_cat, O_wsum, stream=None) -> None:
+    _check("gqe_group_slots", _lib.gqe_group_slots(ctypes.byref(shape), _ptr(O), _ptr(idx), _ptr(gate),
+                                                   _ptr(O_cat), _ptr(O_wsum), _stream(stream)))
 
 
 def gqe_get_device_status(workspace, stream=None) -> int:

@@ -21,7 +21,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", os.path.join(os.path.dirname(PKG), "include")]
 
-LIB_SOURCES = ["gqe_api.cu", "router.cu", "router_tc.cu", "prefill_simt.cu", "prefill_tc.cu", "decode.cu"]
+LIB_SOURCES = ["gqe_api.cu", "router.cu", "router_tc.cu", "prefill_simt.cu", "prefill_tc.cu", "decode.cu",
+               "output.cu"]
 SELFTEST_SOURCES = ["selftest.cu"]
 
 

@@ -125,7 +125,34 @@ struct PrefillArgs {
     void* O;
     void* status;
     cudaStream_t stream;
+    // K/V layout [B, T, kv_g, d_h]; the shape's group q reads KV group kv_q0 + q.
+    // A routed prefill has kv_g = g, kv_q0 = 0; the shared head runs as one
+    // group of one head over a chosen KV group of the caller's K/V.
+    int kv_g;
+    int kv_q0;
 };
+// Output construction (output.cu).
+struct GroupSlotsArgs {
+    const gqe_shape* s;
+    const void* O;       // [B, T, h, d_h] gated routed output
+    const int32_t* idx;  // [B, T, g, k]
+    const float* gate;   // [B, T, g, k]
+    void* cat;           // [B, T, g, k, d_h] or null
+    void* wsum;          // [B, T, g, d_h] or null
+    cudaStream_t stream;
+};
+cudaError_t launch_group_slots(const GroupSlotsArgs& a);
+// Identity routing of one head (every position, gate 1) for the shared head.
+struct IdentityTables {
+    int32_t* idx;
+    float* gate;
+    int32_t* head_offsets;
+    int32_t* head_pos;
+    int32_t* head_chunk_offsets;
+};
+size_t shared_tables_bytes(int B, int T);
+cudaError_t launch_identity_tables(int B, int T, void* tables, IdentityTables* out, cudaStream_t stream);
+
 cudaError_t launch_prefill_simt(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a);
 

@@ -49,6 +49,8 @@ int gqe_chunk_count(int T) { return T <= 0 ? 0 : (T + kChunk - 1) / kChunk; }
 size_t gqe_workspace_bytes(const gqe_shape* s, int Lmax) {
     if (check_shape(s) == GQE_ERR_INVALID_ARGUMENT || Lmax < 0) return 0;
     size_t need = kStatusBytes + route_scratch_bytes(s);
+    const size_t shared = kStatusBytes + shared_tables_bytes(s->B, s->T);
+    if (shared > need) need = shared;
     if (Lmax > 0) {
         const size_t dec = kStatusBytes + align256(decode_partials_bytes(s, Lmax));
         if (dec > need) need = dec;
@@ -141,6 +143,8 @@ gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, co
     a.O = O;
     a.status = workspace;
     a.stream = (cudaStream_t)stream;
+    a.kv_g = s->g;
+    a.kv_q0 = 0;
     if (s->dtype == GQE_BF16) {
         if (s->d_h != 128) return GQE_ERR_UNSUPPORTED;
         return from_cuda(launch_prefill_tc(a));
@@ -148,6 +152,63 @@ gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, co
     if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
     if (s->h / s->g > 64) return GQE_ERR_UNSUPPORTED;
     return from_cuda(launch_prefill_simt(a));
+}
+
+gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* K, const void* V, int kv_group,
+                                void* Os, void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!Qs || !K || !V || !Os) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(Qs) || !aligned16(K) || !aligned16(V) || !aligned16(Os)) return GQE_ERR_INVALID_ARGUMENT;
+    if (kv_group < 0 || kv_group >= s->g) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->dtype == GQE_BF16 ? s->d_h != 128 : (s->d_h != 32 && s->d_h != 64 && s->d_h != 128))
+        return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + shared_tables_bytes(s->B, s->T));
+    if (st != GQE_OK) return st;
+    // One group of one head, selected by every token with gate 1.
+    gqe_shape one = *s;
+    one.h = 1;
+    one.g = 1;
+    one.k = 1;
+    IdentityTables tab;
+    cudaError_t err = launch_identity_tables(s->B, s->T, static_cast<char*>(workspace) + kStatusBytes, &tab,
+                                             (cudaStream_t)stream);
+    if (err != cudaSuccess) return GQE_ERR_CUDA;
+    PrefillArgs a;
+    a.s = &one;
+    a.Q = Qs;
+    a.K = K;
+    a.V = V;
+    a.idx = tab.idx;
+    a.gate = tab.gate;
+    a.head_offsets = tab.head_offsets;
+    a.head_pos = tab.head_pos;
+    a.head_chunk_offsets = tab.head_chunk_offsets;
+    a.O = Os;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    a.kv_g = s->g;
+    a.kv_q0 = kv_group;
+    return from_cuda(s->dtype == GQE_BF16 ? launch_prefill_tc(a) : launch_prefill_simt(a));
+}
+
+gqe_status gqe_group_slots(const gqe_shape* s, const void* O, const int32_t* idx, const float* gate, void* O_cat,
+                           void* O_wsum, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!O || !idx || !gate || (!O_cat && !O_wsum)) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(O) || (O_cat && !aligned16(O_cat)) || (O_wsum && !aligned16(O_wsum)))
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+    GroupSlotsArgs a;
+    a.s = s;
+    a.O = O;
+    a.idx = idx;
+    a.gate = gate;
+    a.cat = O_cat;
+    a.wsum = O_wsum;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_group_slots(a));
 }
 
 gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cache,

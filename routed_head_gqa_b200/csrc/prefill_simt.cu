@@ -21,7 +21,7 @@ prefill_simt_kernel(UnitGeom u, const float* __restrict__ Q, const float* __rest
                     const float* __restrict__ V, const int32_t* __restrict__ idx,
                     const float* __restrict__ gate, const int32_t* __restrict__ head_offsets,
                     const int32_t* __restrict__ head_pos, const int32_t* __restrict__ head_chunk_offsets,
-                    float* __restrict__ O, void* status) {
+                    float* __restrict__ O, void* status, int kv_g, int kv_q0) {
     constexpr int d_h = DPL * 32;
     __shared__ int32_t s_start[64], s_prefix[65];
     __shared__ int32_t rows_t[kMaxRowsSimt];
@@ -102,10 +102,10 @@ prefill_simt_kernel(UnitGeom u, const float* __restrict__ Q, const float* __rest
             acc[e] = 0.f;
         }
         float m = -INFINITY, l = 0.f;
-        const float* kb = K + ((int64_t)b * u.T * u.g + q) * d_h;
-        const float* vb = V + ((int64_t)b * u.T * u.g + q) * d_h;
+        const float* kb = K + ((int64_t)b * u.T * kv_g + kv_q0 + q) * d_h;
+        const float* vb = V + ((int64_t)b * u.T * kv_g + kv_q0 + q) * d_h;
         for (int s = 0; s <= t; ++s) {
-            const float* kr = kb + (int64_t)s * u.g * d_h;
+            const float* kr = kb + (int64_t)s * kv_g * d_h;
             float p = 0.f;
 #pragma unroll
             for (int e = 0; e < DPL; ++e) p = fmaf(qv[e], kr[e * 32 + lane], p);
@@ -115,7 +115,7 @@ prefill_simt_kernel(UnitGeom u, const float* __restrict__ Q, const float* __rest
             const float corr = exp2f(m - m_new);
             const float e_p = exp2f(p - m_new);
             l = l * corr + e_p;
-            const float* vr = vb + (int64_t)s * u.g * d_h;
+            const float* vr = vb + (int64_t)s * kv_g * d_h;
 #pragma unroll
             for (int e = 0; e < DPL; ++e) acc[e] = fmaf(e_p, vr[e * 32 + lane], acc[e] * corr);
             m = m_new;
@@ -140,7 +140,7 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a) {
 #define GQE_SIMT_LAUNCH(DPL)                                                                        \
     prefill_simt_kernel<DPL><<<blocks, kSimtThreads, 0, a.stream>>>(                              \
         u, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.idx, a.gate, a.head_offsets, \
-        a.head_pos, a.head_chunk_offsets, (float*)a.O, a.status)
+        a.head_pos, a.head_chunk_offsets, (float*)a.O, a.status, a.kv_g, a.kv_q0)
     switch (s.d_h) {
         case 32: GQE_SIMT_LAUNCH(1); break;
         case 64: GQE_SIMT_LAUNCH(2); break;

@@ -80,6 +80,7 @@ struct Params {
     uint32_t* status;
     float scale_log2;
     int q_rows;  // B*T*h: rows of Q viewed as [B*T*h, 128]
+    int kv_q0;   // KV group of the unit's group 0 in the K/V tensor maps
 };
 
 // Keys needed by Q tile t of the unit at window w: 0 .. end-1, end = min(w0 + (t+1)W, T).
@@ -240,13 +241,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     const uint32_t par = ((kv_it >> 1) & 1) ^ 1;
                     if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(sm, p, 1); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_k[st], kTileBytes);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, q, i * kBN, b);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, q, i * kBN, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, p.kv_q0 + q, i * kBN, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, p.kv_q0 + q, i * kBN, b);
                     k_pending = true;
                     if (!mbar_wait(&sm.kv_empty_v[st], par)) { fail(sm, p, 2); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_v[st], kTileBytes);
-                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, q, i * kBN, b);
-                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, q, i * kBN, b);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, p.kv_q0 + q, i * kBN, b);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, p.kv_q0 + q, i * kBN, b);
                     k_pending = false;
                 }
                 if (!ok) break;
@@ -738,8 +739,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     if (regs_checked != 1) return cudaErrorNotSupported;
 
     CUtensorMap mapK, mapV;
-    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
-    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)a.kv_g, (uint64_t)s.T, (uint64_t)s.B};
+    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)a.kv_g * kD * 2, (uint64_t)s.T * a.kv_g * kD * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kBN, 1};
     if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
@@ -765,6 +766,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     p.status = (uint32_t*)a.status;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     p.q_rows = (int)q_rows;
+    p.kv_q0 = a.kv_q0;
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);

@@ -101,6 +101,30 @@ def test_null_and_misaligned_pointers_rejected():
                                   1 << 30, None) == 1
 
 
+def test_output_construction_validation():
+    import routed_head_gqa_b200 as g
+
+    s = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_BF16)
+    fake = 0x10000
+    big = 1 << 30
+    # shared head: kv_group outside [0, g), null query, too small a workspace
+    for kv in (-1, 8):
+        assert g._lib.gqe_attn_shared_head(ctypes.byref(s), fake, fake, fake, kv, fake, fake, big, None) == 1
+    assert g._lib.gqe_attn_shared_head(ctypes.byref(s), None, fake, fake, 0, fake, fake, big, None) == 1
+    assert g._lib.gqe_attn_shared_head(ctypes.byref(s), fake, fake, fake, 0, fake, fake, 256, None) == 1
+    # the workspace of gqe_workspace_bytes covers the shared head's identity tables
+    assert g.gqe_workspace_bytes(s, 0) >= 256 + 3 * 2 * 64 * 4 + 3 * 4 + 2 * 2 * 4
+    # bf16 needs d_h = 128, as the routed prefill
+    s64 = g.make_shape(2, 64, 128, 32, 8, 64, 2, g.GQE_BF16)
+    assert g._lib.gqe_attn_shared_head(ctypes.byref(s64), fake, fake, fake, 0, fake, fake, big, None) == 2
+    # group slots: at least one output, supported d_h
+    assert g._lib.gqe_group_slots(ctypes.byref(s), fake, fake, fake, None, None, None) == 1
+    assert g._lib.gqe_group_slots(ctypes.byref(s), None, fake, fake, fake, fake, None) == 1
+    assert g._lib.gqe_group_slots(ctypes.byref(s), fake, fake, fake, fake + 8, None, None) == 1
+    s96 = g.make_shape(2, 64, 128, 32, 8, 96, 2, g.GQE_BF16)
+    assert g._lib.gqe_group_slots(ctypes.byref(s96), fake, fake, fake, fake, None, None) == 2
+
+
 def test_unsupported_cases_report_unsupported():
     import routed_head_gqa_b200 as g
 
