@@ -9,7 +9,8 @@ input, with inputs resident in HBM:
   decode workload:   gqe_route on the new tokens + gqe_attn_decode
 Metric: active-head TFLOP/s for prefill (4*d_h*(t+1) per routed row), KV-cache
 GB/s for decode (2*g*d_h*L_b bf16 elements per sequence).  The L2 is flushed
-(256 MB memset) before every timed step, outside the step's CUDA events.
+before every timed step, outside the step's CUDA events: a 256 MB buffer is
+written, then read back, so the step starts with clean, unrelated lines in L2.
 
 With N > 1 (torchrun) every rank runs an independent replica on its own batch
 (the path has no exchange step); value = all ranks' work / the slowest rank's time.
@@ -45,8 +46,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "52eb0dd68639c989", "bytes_per_launch": 104635904 + 31958016,
+        "sha": "76741b759b980fd7", "bytes_per_launch": 105262080 + 29858816,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
+    ("decode_partial_kernel", "gqe_decode"): {
+        "sha": "265f8d71d70cc0c8", "bytes_per_launch": 2270542956,
+        "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch of the partial kernel: "
+                "dram__bytes.sum.per_second x duration (profiles/decode_partial_kernel_gqe_decode.md)"},
 }
 
 
@@ -128,6 +133,15 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(mhz)}
+
+
+def l2_flush(buf):
+    """Evict the L2 between timed steps: write a 256 MB buffer (twice the L2),
+    then read it back, so that the L2 is left holding clean lines of an
+    unrelated buffer and the timed kernels do not pay for writing the flush's
+    dirty lines back to HBM."""
+    buf.zero_()
+    buf.view(torch.int32).max()
 
 
 # ---------------------------------------------------------------------------
@@ -247,7 +261,7 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
         assert metrics.prefill_active_flops_from_routing(r.buf.idx, w.d_h) == int(work)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(warmup):
-        flush.zero_()
+        l2_flush(flush)
         r.step()
     torch.cuda.synchronize()
     st = r.buf.status()
@@ -263,7 +277,7 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
     barrier(ws)
     torch.cuda.synchronize()
     for i in range(steps):
-        flush.zero_()
+        l2_flush(flush)
         e0, e1, e2 = ev[i]
         e0.record()
         r.route()
@@ -341,12 +355,12 @@ def time_output_construction(w, steps, warmup, peaks, peak_kind):
 
     def timed(fn):
         for _ in range(warmup):
-            flush.zero_()
+            l2_flush(flush)
             fn()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
         for a, b in ev:
-            flush.zero_()
+            l2_flush(flush)
             a.record()
             fn()
             b.record()
@@ -555,7 +569,8 @@ def main():
             "data": "synthetic (seeded, gqe_synth recipe)",
             "config": {"workload": w.name, "shape": w.describe(), "per_gpu_batch": w.B,
                        "global_batch": w.B * ws, "parallelism": f"replicas x{ws} (no exchange step)",
-                       "l2": "flushed (256 MB memset) before every timed step, outside the step events",
+                       "l2": "flushed before every timed step, outside the step events: 256 MB written, "
+                             "then read back (clean lines, no write-back charged to the step)",
                        "attn_ms": res["attn_ms"], "route_ms": res["route_ms"]},
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"],
             "gpu_launches": res["gpu_launches"],

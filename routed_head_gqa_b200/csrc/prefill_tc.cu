@@ -219,6 +219,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // Launched as a programmatic dependent of the compaction: the set-up above
+    // overlaps its tail; nothing it writes is read before this wait.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
@@ -776,8 +779,17 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    prefill_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel, mapK, mapV, mapQ, p);
 }
 
 }  // namespace gqe

@@ -148,6 +148,10 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
     extern __shared__ int32_t sh[];  // [h] head totals -> head bases, [h] prefix within head
     int32_t* total = sh;
     int32_t* before = sh + h;
+    // Launched as a programmatic dependent of the router: wait for its grid,
+    // then let the prefill that follows start its set-up.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int c = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const int32_t* cnt = counts + (int64_t)b * h * nchunk;
@@ -243,8 +247,22 @@ cudaError_t launch_route(const RouteArgs& a) {
     if (!(router_tc_supported(a.s) && router_tc_fuses_counts(a.s)))
         compact_count_kernel<<<cgrid, 32 * cwarps, 0, a.stream>>>(a.idx, s.T, s.h, s.g, s.k, nchunk, a.counts);
     const int swarps = 8;  // warps of the scan: one head per warp and round
-    compact_scan_scatter_kernel<<<cgrid, 32 * swarps, 2 * s.h * sizeof(int32_t), a.stream>>>(
-        a.idx, s.B, s.T, s.h, s.g, s.k, nchunk, a.counts, a.head_offsets, a.head_chunk_offsets, a.head_pos);
+    // Programmatic dependent launch: this grid is scheduled while the router
+    // finishes and waits (griddepcontrol.wait) for it before reading.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = cgrid;
+    cfg.blockDim = dim3(32 * swarps);
+    cfg.dynamicSmemBytes = 2 * s.h * sizeof(int32_t);
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e2 = cudaLaunchKernelEx(&cfg, compact_scan_scatter_kernel, (const int32_t*)a.idx, s.B, s.T, s.h,
+                                        s.g, s.k, nchunk, (const int32_t*)a.counts, a.head_offsets,
+                                        a.head_chunk_offsets, a.head_pos);
+    if (e2 != cudaSuccess) return e2;
     return cudaGetLastError();
 }
 

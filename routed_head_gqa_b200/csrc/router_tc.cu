@@ -77,7 +77,7 @@ __device__ __forceinline__ float ld_peer(uint32_t addr) {
     return v;
 }
 
-template <int NB, int KS>
+template <int NB, int KS, int KMAX>
 __global__ void __launch_bounds__(128)
 router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
                  const float* __restrict__ bias, int64_t BT, int d_model, int h, int g, int k, int T,
@@ -95,6 +95,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
     const int nk = (d_model + kTK - 1) / kTK;
     const int kb0 = (int)((int64_t)nk * rank / KS);
     const int nkl = (int)((int64_t)nk * (rank + 1) / KS) - kb0;  // >= 1: the host keeps KS <= nk
+    // Each tile starts its walk over the slice at a different block, so that the
+    // CTAs in flight read different column ranges of their token rows instead of
+    // all hitting the same offset of every 8 KB-strided row at once.
+    const int rot = (int)(((blockIdx.x / KS) * 7) % nkl);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -121,7 +125,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         for (int i = 0; i < nkl; ++i) {
             const int s = i % S;
             if (!mbar_wait(&sm.empty[s], ((i / S) & 1) ^ 1)) { sm.failed = 1; break; }
-            const int kb = kb0 + i;
+            const int kb = kb0 + (i + rot) % nkl;
             mbar_arrive_expect_tx(&sm.full[s], kXBytes + NB * kWBlock);
             tma_load_2d(&mapX, &sm.full[s], sm.x[s], kb * kTK, (int)tok0);
             for (int nb = 0; nb < NB; ++nb) tma_load_2d(&mapW, &sm.full[s], sm.w[s][nb], nb * 64, kb * kTK);
@@ -150,6 +154,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         umma_commit(&sm.acc_full);
     }
     __syncwarp();
+
+    // The compaction pass may start launching now; it waits for this grid's
+    // completion before reading anything.
+    asm volatile("griddepcontrol.launch_dependents;");
 
     // Epilogue.  The stages are free once the accumulator is complete; the
     // partial logits go through them, one padded row per token
@@ -198,50 +206,62 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         __syncthreads();
     }
     const bool failed = sm.failed != 0;  // final: every writer is before the barrier above
-    if (!failed && tid < kRows) {
-        const int row = (int)rank * kRows + tid;
-        const int64_t tok = tok0 + row;
-        float* lg = lg_base + row * ld;
-        const bool valid = tok < BT;
+    if (!failed) {
+        // Top-k over (row, group) items, rows fastest: the 32 lanes of a warp
+        // take 32 consecutive tokens of one group, which is also one chunk for
+        // the selection counts.
         const int hpg = h / g;
-        if (valid && bias)
-            for (int j = 0; j < h; ++j) lg[j] += bias[j];
-        // chunk of this warp's 32 tokens (counts fused only when T % 32 == 0)
-        const int64_t t_first = tok0 + (int)rank * kRows + warp * 32;
-        const int cb = (int)(t_first / T), cc = (int)((t_first % T) / kChunk);
-        const bool warp_valid = t_first < BT;
-        for (int q = 0; q < g; ++q) {
-            // top-k of the group's logits, equal logits -> lower index
-            const float* lq = lg + q * hpg;
+        const int nitems = kRows * g;  // kRows is a multiple of 32: whole warps per group
+        for (int it = tid; it < nitems; it += 128) {
+            const int q = it / kRows, rloc = it % kRows;
+            const int row = (int)rank * kRows + rloc;
+            const int64_t tok = tok0 + row;
+            const float* lq = lg_base + row * ld + q * hpg;
+            const float* bq = bias ? bias + q * hpg : nullptr;
             uint64_t taken = 0;  // hpg <= 64 on this path
-            if (valid) {
-                float m = 0.f, denom = 0.f;
-                int sel[16];
-                float sel_l[16];
-                for (int s = 0; s < k; ++s) {
-                    int best = -1;
-                    float bv = 0.f;
-                    for (int a = 0; a < hpg; ++a) {
-                        if ((taken >> a) & 1ull) continue;
-                        const float v = lq[a];
-                        if (best < 0 || v > bv) {
-                            best = a;
-                            bv = v;
+            if (tok < BT) {
+                // top-k of the group's logits (+ bias), equal logits -> lower index
+                int sel[KMAX];
+                float sl[KMAX];
+#pragma unroll
+                for (int s = 0; s < KMAX; ++s) {
+                    sel[s] = 0;
+                    sl[s] = 0.f;
+                    if (s < k) {
+                        int best = -1;
+                        float bv = 0.f;
+                        for (int a = 0; a < hpg; ++a) {
+                            if ((taken >> a) & 1ull) continue;
+                            const float v = bq ? lq[a] + bq[a] : lq[a];
+                            if (best < 0 || v > bv) {
+                                best = a;
+                                bv = v;
+                            }
                         }
+                        taken |= 1ull << best;
+                        sel[s] = best;
+                        sl[s] = bv;
                     }
-                    taken |= 1ull << best;
-                    sel[s] = best;
-                    sel_l[s] = bv;
-                    if (s == 0) m = bv;
-                    denom += expf(bv - m);
                 }
+                const float m = sl[0];
+                float denom = 0.f;
+#pragma unroll
+                for (int s = 0; s < KMAX; ++s)
+                    if (s < k) {
+                        sl[s] = expf(sl[s] - m);
+                        denom += sl[s];
+                    }
                 const int64_t o = (tok * g + q) * k;
-                for (int s = 0; s < k; ++s) {
-                    idx[o + s] = q * hpg + sel[s];
-                    gate[o + s] = expf(sel_l[s] - m) / denom;
-                }
+#pragma unroll
+                for (int s = 0; s < KMAX; ++s)
+                    if (s < k) {
+                        idx[o + s] = q * hpg + sel[s];
+                        gate[o + s] = sl[s] / denom;
+                    }
             }
-            if (counts != nullptr && warp_valid) {
+            const int64_t t_first = tok0 + (int)rank * kRows + (rloc - lane);  // the warp's first token
+            if (counts != nullptr && t_first < BT) {
+                const int cb = (int)(t_first / T), cc = (int)((t_first % T) / kChunk);
                 for (int a = 0; a < hpg; ++a) {
                     const unsigned ball = __ballot_sync(0xffffffffu, (taken >> a) & 1ull);
                     if (lane == 0) counts[((int64_t)cb * h + q * hpg + a) * nchunk + cc] = __popc(ball);
@@ -272,7 +292,7 @@ cudaError_t set_smem_once(K kern, size_t smem, std::atomic<uint64_t>& done) {
     return err;
 }
 
-template <int NB, int KS>
+template <int NB, int KS, int KMAX>
 cudaError_t launch_nb(const RouteArgs& a, bool fused_counts) {
     static std::atomic<uint64_t> configured{0};
     const gqe_shape& s = *a.s;
@@ -291,7 +311,7 @@ cudaError_t launch_nb(const RouteArgs& a, bool fused_counts) {
         if (!make_bf16_map(&mapW, a.W_r, 2, dims, strides, box)) return cudaErrorInvalidValue;
     }
     const size_t smem = sizeof(RouterSmem<NB>) + 1024;
-    auto kern = router_tc_kernel<NB, KS>;
+    auto kern = router_tc_kernel<NB, KS, KMAX>;
     cudaError_t err = set_smem_once(kern, smem, configured);
     if (err != cudaSuccess) return err;
     const int64_t tiles = (BT + kTM - 1) / kTM;
@@ -312,7 +332,7 @@ cudaError_t launch_nb(const RouteArgs& a, bool fused_counts) {
                               (uint32_t*)a.status);
 }
 
-template <int NB>
+template <int NB, int KMAX>
 cudaError_t launch_ks(const RouteArgs& a, bool fused_counts) {
     const gqe_shape& s = *a.s;
     const int64_t tiles = ((int64_t)s.B * s.T + kTM - 1) / kTM;
@@ -321,9 +341,9 @@ cudaError_t launch_ks(const RouteArgs& a, bool fused_counts) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // split d_model over a cluster while the grid would leave SMs idle
-    if (tiles * 4 <= sms && nk >= 4) return launch_nb<NB, 4>(a, fused_counts);
-    if (tiles * 2 <= sms && nk >= 2) return launch_nb<NB, 2>(a, fused_counts);
-    return launch_nb<NB, 1>(a, fused_counts);
+    if (tiles * 4 <= sms && nk >= 4) return launch_nb<NB, 4, KMAX>(a, fused_counts);
+    if (tiles * 2 <= sms && nk >= 2) return launch_nb<NB, 2, KMAX>(a, fused_counts);
+    return launch_nb<NB, 1, KMAX>(a, fused_counts);
 }
 
 }  // namespace
@@ -337,9 +357,15 @@ bool router_tc_fuses_counts(const gqe_shape* s) { return s->T % kChunk == 0; }
 cudaError_t launch_router_tc(const RouteArgs& a) {
     const int h = a.s->h;
     const bool fused = router_tc_fuses_counts(a.s);
-    if (h <= 64) return launch_ks<1>(a, fused);
-    if (h <= 128) return launch_ks<2>(a, fused);
-    return launch_ks<4>(a, fused);
+    // selections held in registers: up to 4 (every configuration here), else 16
+    if (a.s->k <= 4) {
+        if (h <= 64) return launch_ks<1, 4>(a, fused);
+        if (h <= 128) return launch_ks<2, 4>(a, fused);
+        return launch_ks<4, 4>(a, fused);
+    }
+    if (h <= 64) return launch_ks<1, 16>(a, fused);
+    if (h <= 128) return launch_ks<2, 16>(a, fused);
+    return launch_ks<4, 16>(a, fused);
 }
 
 }  // namespace gqe
