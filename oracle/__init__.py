@@ -96,8 +96,9 @@ class Oracle:
         lib.oracle_shared_rows.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_group_slots_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, P,
                                                 i32]
+        lib.oracle_qproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
-                  lib.oracle_shared_rows, lib.oracle_group_slots_rows):
+                  lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -209,6 +210,29 @@ class Oracle:
             raise ValueError(f"oracle_group_slots_rows failed ({rc})")
         return cat, wsum
 
+    def qproj_rows(self, x, W_Q, idx, d_h: int, rows=None, n_threads=None):
+        """Routed query projection (float64 [n_rows, g, k, d_h]): the query row of
+        each selected head idx[b,t,q,r] for token rows b*T + t."""
+        xa, dt = _as_input(x)
+        wa, dw = _as_input(W_Q)
+        if dt != dw:
+            raise TypeError("x and W_Q must share a dtype")
+        B, T, d_model = xa.shape
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        g, k = ia.shape[2], ia.shape[3]
+        h = wa.shape[1] // d_h
+        if wa.shape != (d_model, h * d_h):
+            raise ValueError("W_Q must be [d_model, h*d_h]")
+        if rows is None:
+            rows = np.arange(B * T, dtype=np.int64)
+        ra = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+        out = np.empty((ra.shape[0], g, k, d_h), np.float64)
+        rc = self.lib.oracle_qproj_rows(B, T, d_model, h, g, d_h, k, dt, _ptr(xa), _ptr(wa), _ptr(ia),
+                                        ra.shape[0], _ptr(ra), _ptr(out), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_qproj_rows failed ({rc})")
+        return out
+
     def attn(self, Q, K, V, idx, gate, n_threads=None):
         """Full GQE output O [B, T, h, d_h] (float64)."""
         B, T, h, d_h = tuple(Q.shape)
@@ -272,3 +296,7 @@ def shared_rows(*a, **kw):
 
 def group_slots_rows(*a, **kw):
     return default().group_slots_rows(*a, **kw)
+
+
+def qproj_rows(*a, **kw):
+    return default().qproj_rows(*a, **kw)

@@ -43,6 +43,10 @@
  *    shared head).  The page names no KV head for the shared head; the reading
  *    used here: its own query rows attend, causally, to one KV group chosen by
  *    the caller.
+ *  - Routed query projection (same page, "Activation Conditionnelle": the
+ *    query-side computation is conditional on the routing): the query row of
+ *    head j is x . W_Q[:, j*d_h : (j+1)*d_h], computed only for the heads a
+ *    token selected.
  */
 #include <math.h>
 #include <stdint.h>
@@ -374,4 +378,38 @@ int oracle_group_slots_rows(int B, int T, int h, int g, int d_h, int k, int dtyp
         free(scores);
     }
     return err;
+}
+
+/*
+ * Routed query projection for a list of token rows.
+ * x [B, T, d_model], W_Q [d_model, h*d_h] (dtype); idx [B, T, g, k]
+ * Qsel_rows [n_rows, g, k, d_h] out (double): for each selected head
+ *           j = idx[b,t,q,r], sum_i x[b,t,i] * W_Q[i, j*d_h + c]
+ */
+int oracle_qproj_rows(int B, int T, int d_model, int h, int g, int d_h, int k, int dtype,
+                      const void* x, const void* W_Q, const int32_t* idx,
+                      int64_t n_rows, const int64_t* rows, double* Qsel_rows, int n_threads) {
+    if (B < 0 || T < 1 || d_model < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    if (k < 1 || k > h / g) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * T) return 1;
+    const size_t ldw = (size_t)h * d_h;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t bt = rows[r];
+        for (int q = 0; q < g; ++q) {
+            for (int s = 0; s < k; ++s) {
+                const int j = idx[((size_t)bt * g + q) * k + s];
+                double* out = Qsel_rows + (((size_t)r * g + q) * k + s) * d_h;
+                for (int c = 0; c < d_h; ++c) {
+                    double acc = 0.0;
+                    for (int i = 0; i < d_model; ++i)
+                        acc += load_elem(x, (size_t)bt * d_model + i, dtype) *
+                               load_elem(W_Q, (size_t)i * ldw + (size_t)j * d_h + c, dtype);
+                    out[c] = acc;
+                }
+            }
+        }
+    }
+    return 0;
 }

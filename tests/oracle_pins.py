@@ -440,9 +440,47 @@ def check_group_slots(o):
         assert np.allclose(wsum1[0, q_], Vd[0, 0, q_] * gate[0, 0, q_].sum(), atol=1e-15)
 
 
+# --------------------------------------------------------------------------
+# Routed query projection
+# --------------------------------------------------------------------------
+
+def check_qproj(o):
+    """Block-identity W_Q (d_model = h*d_h): each selected head's query row is
+    exactly its own d_h-slice of x; a one-hot x picks one row of W_Q."""
+    B, T, h, g, d, k = 2, 3, 4, 2, 4, 2
+    d_model = h * d
+    x = _f32((B, T, d_model), 80)
+    idx = np.zeros((B, T, g, k), np.int32)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                idx[b, t, q_] = [q_ * 2 + 1, q_ * 2] if (b + t + q_) % 2 else [q_ * 2, q_ * 2 + 1]
+    Wid = np.eye(d_model, dtype=np.float32)
+    Qs = o.qproj_rows(x, Wid, idx, d).reshape(B, T, g, k, d)
+    xd = x.astype(np.float64)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                for r in range(k):
+                    j = idx[b, t, q_, r]
+                    assert np.array_equal(Qs[b, t, q_, r], xd[b, t, j * d:(j + 1) * d]), f"identity W_Q ({b},{t},{q_},{r})"
+    # one-hot x at input i: the query row of head j is row i of W_Q's j-th column block
+    W = _f32((d_model, h * d), 81)
+    i0 = 5
+    x1 = np.zeros((B, T, d_model), np.float32)
+    x1[:, :, i0] = 1.0
+    Q1 = o.qproj_rows(x1, W, idx, d).reshape(B, T, g, k, d)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                for r in range(k):
+                    j = idx[b, t, q_, r]
+                    assert np.array_equal(Q1[b, t, q_, r], W[i0, j * d:(j + 1) * d].astype(np.float64))
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
-    check_shared_head_closed_forms, check_group_slots,
+    check_shared_head_closed_forms, check_group_slots, check_qproj,
 ]

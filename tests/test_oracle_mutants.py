@@ -35,6 +35,10 @@ MUTANTS = [
      "(size_t)g * d_h, T, d_h, dtype,\n                           scores, Os_rows"),
     ("weighted_sum_ungated", "for (int d = 0; d < d_h; ++d) ws[d] += gate[sel] * slot[d];",
      "for (int d = 0; d < d_h; ++d) ws[d] += slot[d];"),
+    ("qproj_head_block_offset", "load_elem(W_Q, (size_t)i * ldw + (size_t)j * d_h + c, dtype);",
+     "load_elem(W_Q, (size_t)i * ldw + (size_t)j + c, dtype);"),
+    ("qproj_transposed_weight", "load_elem(W_Q, (size_t)i * ldw + (size_t)j * d_h + c, dtype);",
+     "load_elem(W_Q, ((size_t)((size_t)j * d_h + c) * d_model + i) % ((size_t)d_model * ldw), dtype);"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
