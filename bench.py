@@ -329,12 +329,13 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
     return res
 
 
-def time_output_construction(w, steps, warmup, peaks, peak_kind):
-    """The GQE output construction on the workload's shapes, each call timed
-    alone with CUDA events (L2 flushed before each call, outside the events):
-    the always-active shared head (one dense causal head over KV group 0, on
-    the routed prefill's tensor-core kernel) and the per-group slots
-    (concatenated expert outputs + gate-weighted sum, HBM-bound)."""
+def time_layer_ops(w, steps, warmup, peaks, peak_kind):
+    """The GQE layer's calls around the routed attention, on the workload's
+    shapes, each timed alone with CUDA events (L2 flushed before each call,
+    outside the events): the routed query projection (a tensor-core grouped
+    GEMM over the routed rows only), the always-active shared head (one dense
+    causal head over KV group 0, on the routed prefill's kernel) and the
+    per-group slots (concatenated expert outputs + gate-weighted sum, HBM-bound)."""
     from routed_head_gqa_b200 import metrics
 
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -343,6 +344,8 @@ def time_output_construction(w, steps, warmup, peaks, peak_kind):
     r.step()
     Qs = gqe_synth.make_shared_query(w).to(dev)
     Os = torch.empty((w.B, w.T, w.d_h), dtype=w.torch_dtype, device=dev)
+    W_Q = gqe_synth.make_qproj_weight(w).to(dev)
+    Qp = torch.empty((w.B, w.T, w.h, w.d_h), dtype=w.torch_dtype, device=dev)
     cat = torch.empty((w.B, w.T, w.g, w.k, w.d_h), dtype=w.torch_dtype, device=dev)
     wsum = torch.empty((w.B, w.T, w.g, w.d_h), dtype=w.torch_dtype, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -352,6 +355,9 @@ def time_output_construction(w, steps, warmup, peaks, peak_kind):
 
     def slots():
         g.gqe_group_slots(r.shape, r.buf.O, r.buf.idx, r.buf.gate, cat, wsum)
+
+    def qproj():
+        g.gqe_routed_qproj(r.shape, r.d["x"], W_Q, r.buf.head_offsets, r.buf.head_pos, Qp, r.buf.workspace)
 
     def timed(fn):
         for _ in range(warmup):
@@ -369,6 +375,7 @@ def time_output_construction(w, steps, warmup, peaks, peak_kind):
 
     sh_ms = timed(shared)
     sl_ms = timed(slots)
+    qp_ms = timed(qproj)
     st = r.buf.status()
     if st != 0:
         raise RuntimeError(f"device status {g.gqe_status_string(st)} in the output construction")
@@ -376,11 +383,18 @@ def time_output_construction(w, steps, warmup, peaks, peak_kind):
     el = 2 if w.dtype == "bf16" else 4
     rows = w.B * w.T * w.g * w.k
     sl_bytes = float(rows * w.d_h * el * 2 + w.B * w.T * w.g * w.d_h * el + rows * 8)  # O rows in, cat + wsum out
+    qp_flops = 2.0 * w.d_model * w.d_h * rows  # routed rows only
+    qp_tf = qp_flops / (qp_ms * 1e-3) * 1e-12
     sh_tf = sh_flops / (sh_ms * 1e-3) * 1e-12
     sl_gbs = sl_bytes / (sl_ms * 1e-3) * 1e-9
     del r, flush
     torch.cuda.empty_cache()
     return {
+        "routed_qproj": {"ms": qp_ms, "value": qp_tf, "unit": "TFLOP/s", "flops": qp_flops,
+                         "roofline": {"bound": "tensor", "achieved": round(qp_tf, 1), "peak": peaks["bf16_tflops"],
+                                      "unit": "TFLOP/s", "frac": round(qp_tf / peaks["bf16_tflops"], 4),
+                                      "peak_source": f"bf16_tflops burst ({peak_kind})",
+                                      "kernel": "gqe_routed_qproj (qproj_kernel)"}},
         "shared_head": {"ms": sh_ms, "value": sh_tf, "unit": "TFLOP/s", "flops": sh_flops,
                         "roofline": {"bound": "tensor", "achieved": round(sh_tf, 1), "peak": peaks["bf16_tflops"],
                                      "unit": "TFLOP/s", "frac": round(sh_tf / peaks["bf16_tflops"], 4),
@@ -555,9 +569,9 @@ def main():
             secondary[name] = {"value": r2["value"], "unit": r2["unit"], "ms_per_step": r2["ms_per_step"],
                                "attn_ms": r2["attn_ms"], "route_ms": r2["route_ms"], "roofline": r2["roofline"],
                                "shape": sw.describe()}
-    output_construction = None
+    layer_ops = None
     if not args.no_secondary and args.workload == PRIMARY:
-        output_construction = time_output_construction(w, max(5, args.steps // 2), 3, peaks, peak_kind)
+        layer_ops = time_layer_ops(w, max(5, args.steps // 2), 3, peaks, peak_kind)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)
@@ -577,8 +591,8 @@ def main():
         }
         if secondary:
             line["workloads"] = secondary
-        if output_construction:
-            line["output_construction"] = output_construction
+        if layer_ops:
+            line["gqe_layer_ops"] = layer_ops
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist

@@ -149,6 +149,14 @@ def make_shared_query(w: Workload):
     return _normal((w.B, w.T, w.d_h), gen).to(w.torch_dtype)
 
 
+def make_qproj_weight(w: Workload):
+    """Query projection W_Q [d_model, h*d_h] ~ N(0, 1/sqrt(d_model)) in the
+    workload's dtype (query rows of unit scale), from its own seeded generator
+    (seed + 104729)."""
+    gen = torch.Generator().manual_seed(w.seed + 104729)
+    return _normal((w.d_model, w.h * w.d_h), gen, std=1.0 / math.sqrt(w.d_model)).to(w.torch_dtype)
+
+
 def sample_rows(w: Workload, n: int, seed: int = 1234):
     """A seeded sample of n flattened token rows (b*T + t) that always includes
     the last position of every sequence and the first position of batch 0."""

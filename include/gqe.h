@@ -183,6 +183,29 @@ gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cach
                            size_t workspace_bytes, void* stream);
 
 /*
+ * gqe_routed_qproj -- query projection for the routed heads only.
+ *
+ * The routing makes the query side conditional while K/V stay dense
+ * (gist.science summary, "Activation Conditionnelle", "Chemin KV Dense"), so
+ * a head's query row is computed only for the tokens that selected it:
+ *   Q[b,t,j,:] = sum_i x[b,t,i] * W_Q[i, j*d_h + c]      for every routed (b, t, j),
+ * accumulated in fp32 on the tensor cores and rounded to bf16.  Rows of Q
+ * whose head was not selected are not written (gqe_attn_prefill never reads
+ * them).
+ *
+ *   x [B, T, d_model]                  device bf16
+ *   W_Q [d_model, h * d_h]             device bf16 (head j's block: columns j*d_h ..)
+ *   head_offsets, head_pos             device, exactly as written by gqe_route
+ *   Q [B, T, h, d_h]                   device bf16, out (routed rows)
+ *   workspace                          status word only (gqe_workspace_bytes)
+ * Implemented cases: bf16, d_h = 128, d_model % 8 == 0; others return
+ * GQE_ERR_UNSUPPORTED.
+ */
+gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* head_offsets,
+                            const int32_t* head_pos, void* Q, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
  * gqe_attn_shared_head -- the always-active shared head of the GQE layer.
  *
  * One extra attention head computed for every token whatever the routing

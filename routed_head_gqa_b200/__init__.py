@@ -27,7 +27,7 @@ GQE_F32 = 0
 GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
-            "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_shared_head", "gqe_group_slots",
+            "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -68,11 +68,12 @@ def _load():
     lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_shared_head.argtypes = [S, _P, _P, _P, _I, _P, _P, _SZ, _P]
     lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
+    lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
-              "gqe_attn_shared_head", "gqe_group_slots", "gqe_get_device_status"):
+              "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -170,6 +171,12 @@ def gqe_attn_shared_head(shape, Qs, K, V, kv_group, Os, workspace, stream=None) 
     _check("gqe_attn_shared_head", _lib.gqe_attn_shared_head(ctypes.byref(shape), _ptr(Qs), _ptr(K), _ptr(V),
                                                              int(kv_group), _ptr(Os), _ptr(workspace),
                                                              _nbytes(workspace), _stream(stream)))
+
+
+def gqe_routed_qproj(shape, x, W_Q, head_offsets, head_pos, Q, workspace, stream=None) -> None:
+    _check("gqe_routed_qproj", _lib.gqe_routed_qproj(ctypes.byref(shape), _ptr(x), _ptr(W_Q), _ptr(head_offsets),
+                                                     _ptr(head_pos), _ptr(Q), _ptr(workspace), _nbytes(workspace),
+                                                     _stream(stream)))
 
 
 def gqe_group_slots(shape, O, idx, gate, O_cat, O_wsum, stream=None) -> None:

@@ -131,6 +131,19 @@ struct PrefillArgs {
     int kv_g;
     int kv_q0;
 };
+// Routed query projection (qproj.cu).
+struct QprojArgs {
+    const gqe_shape* s;
+    const void* x;               // [B, T, d_model] bf16
+    const void* W_Q;             // [d_model, h * 128] bf16
+    const int32_t* head_offsets; // as written by gqe_route
+    const int32_t* head_pos;
+    void* Q;                     // [B, T, h, 128] bf16, routed rows written
+    void* status;
+    cudaStream_t stream;
+};
+cudaError_t launch_qproj(const QprojArgs& a);
+
 // Output construction (output.cu).
 struct GroupSlotsArgs {
     const gqe_shape* s;

@@ -192,6 +192,28 @@ gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* 
     return from_cuda(s->dtype == GQE_BF16 ? launch_prefill_tc(a) : launch_prefill_simt(a));
 }
 
+gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* head_offsets,
+                            const int32_t* head_pos, void* Q, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!x || !W_Q || !head_offsets || !head_pos || !Q) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(W_Q) || !aligned16(Q)) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->dtype != GQE_BF16 || s->d_h != 128 || s->d_model % 8 != 0) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != GQE_OK) return st;
+    QprojArgs a;
+    a.s = s;
+    a.x = x;
+    a.W_Q = W_Q;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.Q = Q;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_qproj(a));
+}
+
 gqe_status gqe_group_slots(const gqe_shape* s, const void* O, const int32_t* idx, const float* gate, void* O_cat,
                            void* O_wsum, void* stream) {
     gqe_status st = check_shape(s);

@@ -125,6 +125,20 @@ def test_output_construction_validation():
     assert g._lib.gqe_group_slots(ctypes.byref(s96), fake, fake, fake, fake, None, None) == 2
 
 
+def test_routed_qproj_validation():
+    import routed_head_gqa_b200 as g
+
+    fake = 0x10000
+    s = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_BF16)
+    assert g._lib.gqe_routed_qproj(ctypes.byref(s), None, fake, fake, fake, fake, fake, 1 << 20, None) == 1
+    assert g._lib.gqe_routed_qproj(ctypes.byref(s), fake, fake + 4, fake, fake, fake, fake, 1 << 20, None) == 1
+    # tensor-core path only: bf16 with d_h = 128
+    s32 = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_F32)
+    assert g._lib.gqe_routed_qproj(ctypes.byref(s32), fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
+    s64 = g.make_shape(2, 64, 128, 32, 8, 64, 2, g.GQE_BF16)
+    assert g._lib.gqe_routed_qproj(ctypes.byref(s64), fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
+
+
 def test_unsupported_cases_report_unsupported():
     import routed_head_gqa_b200 as g
 
