@@ -46,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "76741b759b980fd7", "bytes_per_launch": 105262080 + 29858816,
+        "sha": "42066333828ea0fa", "bytes_per_launch": 105111040 + 29436928,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
         "sha": "265f8d71d70cc0c8", "bytes_per_launch": 2270542956,
@@ -528,6 +528,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layer-ops-only", action="store_true",
+                    help="time only the calls around the routed attention (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -558,6 +560,15 @@ def main():
         gqe_build.build()
     barrier(ws)
     peaks, peak_kind = load_peaks()
+    if args.layer_ops_only:
+        ops = time_layer_ops(w, args.steps, args.warmup, peaks, peak_kind)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "gqe_layer_ops": ops}))
+        if ws > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
     res = time_workload(w, args.steps, args.warmup, ws, rank, peaks, peak_kind, with_clocks=(rank == 0),
                         with_e2e=True)
     secondary = {}

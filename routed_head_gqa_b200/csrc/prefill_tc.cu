@@ -16,7 +16,9 @@
 // Roles (384 threads, one persistent CTA per SM):
 //   warp 0      TMA producer for K/V tiles; owns the TMEM allocation
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V on tcgen05
-//   warp 2      row tables and Q gather (TMA tile::gather4 of routed rows, 128B-swizzled)
+//   warp 2      row tables and Q tiles: one TMA box per head and half when every
+//               token of the half-window selected every head of the group (dense
+//               GQA), TMA tile::gather4 of the routed rows otherwise (128B-swizzled)
 //   warp 3      zero fill of the window's unselected output slots
 //   warps 4-7   softmax + epilogue of Q tile 0 (one row per thread)
 //   warps 8-11  softmax + epilogue of Q tile 1
@@ -184,7 +186,8 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-                  const __grid_constant__ CUtensorMap mapQ, const Params p) {
+                  const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQB,
+                  const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -230,6 +233,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             tma_prefetch_desc(&mapK);
             tma_prefetch_desc(&mapV);
             tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapQB);
             uint32_t kv_it = 0;
             bool k_pending = false;
             for (int64_t j = 0;; ++j) {
@@ -451,27 +455,36 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 if (lane == 0) fail(sm, p, 21);
                 break;
             }
-            // 3. Q gather by TMA: each routed row is one row of Q viewed as
-            // [B*T*h, 128].  One tile::gather4 copy moves four rows' 64-column
-            // halves (box one row high) to rows r..r+3 of a tile half; the
-            // 128-byte swizzle follows the shared-memory address, so each row
-            // gets its own chunk permutation.  Padding rows name an
+            // 3. Q tiles by TMA.  A tile with h/g * W rows holds every position
+            // of its half-window for every head of the group (dense GQA): head
+            // jj's W rows are W consecutive tokens of Q viewed as [B, T, h, 128],
+            // one box per 64-column half.  Any other tile is gathered: each
+            // routed row is one row of Q viewed as [B*T*h, 128], and one
+            // tile::gather4 copy moves four rows' 64-column halves (box one row
+            // high) to rows r..r+3 of a tile half.  Either way the 128-byte
+            // swizzle follows the shared-memory address.  Padding rows name an
             // out-of-range row, which the TMA zero-fills.
             if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[rs], kQT * kTileBytes);
             __syncwarp();
-            {
-                const int t = lane >> 4;            // 16 lanes per tile
-                const int r0 = (lane & 15) * 8;     // 8 rows per lane: two gather4 groups
 #pragma unroll
-                for (int gq = 0; gq < 2; ++gq) {
+            for (int t = 0; t < kQT; ++t) {
+                // full tile of exactly 128 rows: the boxes deliver the 32 KB the
+                // barrier expects (a 96-row full tile, h/g = k = 3, is gathered)
+                if (u.hpg * u.W == kBM && sm.cut_prefix[rs][t][u.hpg] == kBM) {
+                    if (lane < 2 * u.hpg) {
+                        const int jj = lane >> 1, half = lane & 1;
+                        uint8_t* dst = sm.q[t] + jj * u.W * 128 + half * kHalf;
+                        tma_load_4d(&mapQB, &sm.q_full[rs], dst, half * 64, q * u.hpg + jj, (w * kQT + t) * u.W, b);
+                    }
+                } else {
+                    const int r0 = lane * 4;  // four rows per lane
                     int row[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int r = r0 + gq * 4 + e;
-                        const int tr = sm.row_t[rs][t][r];
-                        row[e] = (tr >= 0) ? (int)(((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][t][r]) : p.q_rows;
+                        const int tr = sm.row_t[rs][t][r0 + e];
+                        row[e] = (tr >= 0) ? (int)(((int64_t)b * u.T + tr) * u.h + sm.row_j[rs][t][r0 + e]) : p.q_rows;
                     }
-                    uint8_t* dst = sm.q[t] + (r0 + gq * 4) * 128;
+                    uint8_t* dst = sm.q[t] + r0 * 128;
                     tma_gather4_2d(&mapQ, &sm.q_full[rs], dst, 0, row[0], row[1], row[2], row[3]);
                     tma_gather4_2d(&mapQ, &sm.q_full[rs], dst + kHalf, 64, row[0], row[1], row[2], row[3]);
                 }
@@ -756,6 +769,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
         const uint32_t qbox[2] = {64, 1};
         if (!make_bf16_map(&mapQ, a.Q, 2, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
     }
+    CUtensorMap mapQB;  // Q as [B, T, h, 128]: one head's W consecutive tokens per box
+    {
+        const uint64_t qdims[4] = {(uint64_t)kD, (uint64_t)s.h, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t qstrides[3] = {(uint64_t)kD * 2, (uint64_t)s.h * kD * 2, (uint64_t)s.T * s.h * kD * 2};
+        const uint32_t qbox[4] = {64, 1, (uint32_t)u.W, 1};
+        if (!make_bf16_map(&mapQB, a.Q, 4, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
+    }
 
     Params p;
     p.u = u;
@@ -789,7 +809,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel, mapK, mapV, mapQ, p);
+    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel, mapK, mapV, mapQ, mapQB, p);
 }
 
 }  // namespace gqe
