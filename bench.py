@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
         "sha": "42066333828ea0fa", "bytes_per_launch": 105111040 + 29436928,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
-        "sha": "265f8d71d70cc0c8", "bytes_per_launch": 2270542956,
+        "sha": "7308e784ba49063e", "bytes_per_launch": 2270746301,
         "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch of the partial kernel: "
                 "dram__bytes.sum.per_second x duration (profiles/decode_partial_kernel_gqe_decode.md)"},
 }
