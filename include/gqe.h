@@ -104,7 +104,8 @@ gqe_status gqe_workspace_init(void* workspace, size_t workspace_bytes, void* str
  *                              device int32 out: at [(b*h + j)*nchunk + c] the
  *                              head_pos index of the first entry of (b, j) with
  *                              t >= 32*c
- * Requires h % g == 0, 1 <= k <= h/g, B*T*g*k < 2^31.
+ * Requires B >= 1, T >= 1, h % g == 0, 1 <= k <= h/g, B*T*g*k < 2^31 (any
+ * other shape returns GQE_ERR_INVALID_ARGUMENT, for every entry point).
  */
 gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
                      int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,

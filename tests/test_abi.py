@@ -69,6 +69,7 @@ def test_workspace_bytes():
     ("k", 5, 1),        # k > h/g
     ("k", 0, 1),
     ("T", 0, 1),
+    ("B", 0, 1),        # empty batch: rejected before anything is enqueued
     ("dtype", 7, 1),
 ])
 def test_route_rejects_bad_shapes(field, value, code):
