@@ -97,8 +97,10 @@ class Oracle:
         lib.oracle_group_slots_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, P,
                                                 i32]
         lib.oracle_qproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
+        lib.oracle_decode_paged.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32]
         for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
-                  lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows):
+                  lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows,
+                  lib.oracle_decode_paged):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -233,6 +235,30 @@ class Oracle:
             raise ValueError(f"oracle_qproj_rows failed ({rc})")
         return out
 
+    def decode_paged(self, q, K_pages, V_pages, block_table, lengths, idx, gate, n_threads=None):
+        """Paged GQE decode output O [B, h, d_h] (float64): caches as pages
+        [num_pages, page_size, g, d_h], block_table [B, max_blocks], lengths [B]."""
+        qa, dt = _as_input(q)
+        ka, dk = _as_input(K_pages)
+        va, dv = _as_input(V_pages)
+        if not (dt == dk == dv):
+            raise TypeError("q and the pages must share a dtype")
+        num_pages, page_size, g, d_h = ka.shape
+        B = int(np.asarray(lengths).shape[0])
+        h = qa.shape[-2]
+        ta = np.ascontiguousarray(np.asarray(block_table), dtype=np.int32).reshape(B, -1)
+        ia = np.ascontiguousarray(idx, dtype=np.int32).reshape(B, g, -1)
+        ga = np.ascontiguousarray(gate, dtype=np.float64).reshape(B, g, -1)
+        k = ia.shape[-1]
+        la = np.ascontiguousarray(np.asarray(lengths), dtype=np.int32).reshape(B)
+        out = np.empty((B, h, d_h), np.float64)
+        rc = self.lib.oracle_decode_paged(B, page_size, ta.shape[1], num_pages, h, g, d_h, k, dt, _ptr(qa), _ptr(ka),
+                                          _ptr(va), _ptr(ta), _ptr(la), _ptr(ia), _ptr(ga), _ptr(out),
+                                          _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_decode_paged failed ({rc})")
+        return out
+
     def attn(self, Q, K, V, idx, gate, n_threads=None):
         """Full GQE output O [B, T, h, d_h] (float64)."""
         B, T, h, d_h = tuple(Q.shape)
@@ -300,3 +326,7 @@ def group_slots_rows(*a, **kw):
 
 def qproj_rows(*a, **kw):
     return default().qproj_rows(*a, **kw)
+
+
+def decode_paged(*a, **kw):
+    return default().decode_paged(*a, **kw)

@@ -43,6 +43,10 @@
  *    shared head).  The page names no KV head for the shared head; the reading
  *    used here: its own query rows attend, causally, to one KV group chosen by
  *    the caller.
+ *  - Paged decode.  The same decode with the cache kept in fixed-size pages:
+ *    logical row s of sequence b lives in page block_table[b][s / page_size]
+ *    at row s % page_size (the KV cache stays dense under GQE; only where its
+ *    rows sit in memory changes).
  *  - Routed query projection (same page, "Activation Conditionnelle": the
  *    query-side computation is conditional on the routing): the query row of
  *    head j is x . W_Q[:, j*d_h : (j+1)*d_h], computed only for the heads a
@@ -412,4 +416,77 @@ int oracle_qproj_rows(int B, int T, int d_model, int h, int g, int d_h, int k, i
         }
     }
     return 0;
+}
+
+/*
+ * Paged decode: as oracle_decode, with the caches as pages.
+ * K_pages/V_pages [num_pages, page_size, g, d_h] (dtype); block_table
+ * [B, max_blocks]: page of logical rows [i*page_size, (i+1)*page_size) of
+ * sequence b at [b*max_blocks + i]; lengths[b] <= page_size * max_blocks.
+ * query [B, h, d_h]; idx/gate [B, g, k]; O [B, h, d_h] out (double).
+ */
+int oracle_decode_paged(int B, int page_size, int max_blocks, int num_pages, int h, int g, int d_h, int k,
+                        int dtype, const void* query, const void* K_pages, const void* V_pages,
+                        const int32_t* block_table, const int32_t* lengths, const int32_t* idx,
+                        const double* gate, double* O, int n_threads) {
+    if (B < 0 || page_size < 1 || max_blocks < 1 || num_pages < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1)
+        return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    const int64_t cap = (int64_t)page_size * max_blocks;
+    for (int b = 0; b < B; ++b) {
+        if (lengths[b] < 1 || lengths[b] > cap) return 1;
+        for (int i = 0; i < (lengths[b] + page_size - 1) / page_size; ++i)
+            if (block_table[(size_t)b * max_blocks + i] < 0 || block_table[(size_t)b * max_blocks + i] >= num_pages)
+                return 1;
+    }
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)cap);
+        if (!scores) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1) collapse(2)
+            for (int b = 0; b < B; ++b) {
+                for (int q = 0; q < g; ++q) {
+                    for (int jj = 0; jj < hpg; ++jj)
+                        for (int d = 0; d < d_h; ++d) O[((size_t)b * h + q * hpg + jj) * d_h + d] = 0.0;
+                    const int L = lengths[b];
+                    const double scale = 1.0 / sqrt((double)d_h);
+                    for (int r = 0; r < k; ++r) {
+                        const size_t sel = ((size_t)b * g + q) * k + r;
+                        const int j = idx[sel];
+                        const size_t q_off = ((size_t)b * h + j) * d_h;
+                        /* scores over the logical rows, each read through the block table */
+                        double mx = -INFINITY;
+                        for (int s = 0; s < L; ++s) {
+                            const size_t pg = (size_t)block_table[(size_t)b * max_blocks + s / page_size];
+                            const size_t row = ((pg * page_size + (size_t)(s % page_size)) * g + q) * d_h;
+                            double dot = 0.0;
+                            for (int d = 0; d < d_h; ++d)
+                                dot += load_elem(query, q_off + d, dtype) * load_elem(K_pages, row + d, dtype);
+                            scores[s] = dot * scale;
+                            if (scores[s] > mx) mx = scores[s];
+                        }
+                        double denom = 0.0;
+                        for (int s = 0; s < L; ++s) {
+                            scores[s] = exp(scores[s] - mx);
+                            denom += scores[s];
+                        }
+                        double* out = O + ((size_t)b * h + j) * d_h;
+                        for (int s = 0; s < L; ++s) {
+                            const size_t pg = (size_t)block_table[(size_t)b * max_blocks + s / page_size];
+                            const size_t row = ((pg * page_size + (size_t)(s % page_size)) * g + q) * d_h;
+                            const double w = gate[sel] * scores[s] / denom;
+                            for (int d = 0; d < d_h; ++d) out[d] += w * load_elem(V_pages, row + d, dtype);
+                        }
+                    }
+                }
+            }
+        }
+        free(scores);
+    }
+    return err;
 }

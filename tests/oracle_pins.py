@@ -478,9 +478,70 @@ def check_qproj(o):
                     assert np.array_equal(Q1[b, t, q_, r], W[i0, j * d:(j + 1) * d].astype(np.float64))
 
 
+# --------------------------------------------------------------------------
+# Paged decode
+# --------------------------------------------------------------------------
+
+def check_decode_paged(o):
+    """Pages in a permuted pool: zero keys give the mean of the sequence's first
+    L logical rows; a dominant key at logical position s* returns exactly that
+    row; and the result equals the contiguous decode of the gathered cache."""
+    B, ps, nb, npages, h, g, d, k = 2, 4, 3, 8, 4, 2, 8, 1
+    hpg = h // g
+    bt = np.array([[5, 2, 7], [1, 6, 0]], np.int32)
+    lengths = np.array([10, 5], np.int32)
+    q = _f32((B, h, d), 90)
+    Vp = _f32((npages, ps, g, d), 91)
+    idx = np.array([[[0], [3]], [[1], [2]]], np.int32)  # [B, g, k]: one head per group
+    gate = np.ones((B, g, k), np.float64)
+
+    def logical(P, b, s_):
+        return P[bt[b, s_ // ps], s_ % ps]
+
+    Vd = Vp.astype(np.float64)
+    # zero keys: uniform weights over the L logical rows
+    O0 = o.decode_paged(q, np.zeros_like(Vp), Vp, bt, lengths, idx, gate)
+    for b in range(B):
+        mean = np.mean([logical(Vd, b, s_) for s_ in range(lengths[b])], axis=0)  # [g, d]
+        for q_ in range(g):
+            assert np.allclose(O0[b, idx[b, q_, 0]], mean[q_], atol=1e-13), f"paged K=0 b={b}"
+    # dominant key at logical position s* (order-sensitive)
+    star = [7, 3]
+    Kp = np.zeros_like(Vp)
+    qd = np.zeros_like(q)
+    qd[..., 0] = 30.0
+    for b in range(B):
+        pg, r = bt[b, star[b] // ps], star[b] % ps
+        Kp[pg, r, :, 0] = 30.0
+    Od = o.decode_paged(qd, Kp, Vp, bt, lengths, idx, gate)
+    for b in range(B):
+        for q_ in range(g):
+            assert np.allclose(Od[b, idx[b, q_, 0]], logical(Vd, b, star[b])[q_], atol=1e-12), f"paged s* b={b}"
+    # the gathered cache through the contiguous decode
+    Kp2 = _f32((npages, ps, g, d), 92)
+    Lmax = ps * nb
+    Kc = np.zeros((B, Lmax, g, d), np.float32)
+    Vc = np.zeros((B, Lmax, g, d), np.float32)
+    for b in range(B):
+        for s_ in range(lengths[b]):
+            Kc[b, s_] = logical(Kp2, b, s_)
+            Vc[b, s_] = logical(Vp, b, s_)
+    idx2 = np.array([[[1], [2]], [[0], [3]]], np.int32)
+    gate2 = np.full((B, g, k), 0.75)
+    Op = o.decode_paged(q, Kp2, Vp, bt, lengths, idx2, gate2)
+    Oc = o.decode(q, Kc, Vc, lengths, idx2, gate2)
+    # (the gate enters each weight here and the finished row there: agreement to rounding)
+    assert np.allclose(Op, Oc, rtol=0, atol=1e-12), "paged decode differs from the contiguous decode of the gathered cache"
+    for b in range(B):
+        for j in range(h):
+            if j not in idx2[b].reshape(-1):
+                assert np.all(Op[b, j] == 0.0)
+    _ = hpg
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
-    check_shared_head_closed_forms, check_group_slots, check_qproj,
+    check_shared_head_closed_forms, check_group_slots, check_qproj, check_decode_paged,
 ]

@@ -39,6 +39,10 @@ MUTANTS = [
      "load_elem(W_Q, (size_t)i * ldw + (size_t)j + c, dtype);"),
     ("qproj_transposed_weight", "load_elem(W_Q, (size_t)i * ldw + (size_t)j * d_h + c, dtype);",
      "load_elem(W_Q, ((size_t)((size_t)j * d_h + c) * d_model + i) % ((size_t)d_model * ldw), dtype);"),
+    ("paged_row_offset", "const size_t row = ((pg * page_size + (size_t)(s % page_size)) * g + q) * d_h;",
+     "const size_t row = ((pg * page_size + (size_t)((s + 1) % page_size)) * g + q) * d_h;"),
+    ("paged_block_lookup", "(size_t)block_table[(size_t)b * max_blocks + s / page_size];",
+     "(size_t)block_table[(size_t)b * max_blocks + (s / page_size) % 2];"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
