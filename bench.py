@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
         "sha": "42066333828ea0fa", "bytes_per_launch": 105111040 + 29436928,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
-        "sha": "7308e784ba49063e", "bytes_per_launch": 2270746301,
+        "sha": "38d1f07202b92c94", "bytes_per_launch": 2270814604,
         "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch of the partial kernel: "
                 "dram__bytes.sum.per_second x duration (profiles/decode_partial_kernel_gqe_decode.md)"},
 }
@@ -409,6 +409,52 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
     }
 
 
+def time_paged_decode(w, steps, warmup, peaks, peak_kind, page_size=256):
+    """The decode workload with its caches cut into pages of page_size rows,
+    scattered over the pool in a seeded random order (gqe_attn_decode_paged),
+    timed like the contiguous decode: CUDA events around the decode call, L2
+    flushed before each, outside the events."""
+    from routed_head_gqa_b200 import metrics
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    r = Runner(w, dev)
+    g = r.g
+    r.route()
+    Kp, Vp, bt = gqe_synth.make_paged_cache(r.inp["K_cache"], r.inp["V_cache"], page_size)
+    Kp, Vp, bt = Kp.to(dev), Vp.to(dev), bt.to(dev)
+    del r.d["K_cache"], r.d["V_cache"]
+    O = torch.empty_like(r.buf.O)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def paged():
+        g.gqe_attn_decode_paged(r.shape, r.d["q"], Kp, Vp, page_size, bt, r.d["lengths"], r.buf.idx, r.buf.gate, O,
+                                r.buf.workspace)
+
+    for _ in range(warmup):
+        l2_flush(flush)
+        paged()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        l2_flush(flush)
+        a.record()
+        paged()
+        b.record()
+    torch.cuda.synchronize()
+    st = r.buf.status()
+    if st != 0:
+        raise RuntimeError(f"device status {g.gqe_status_string(st)} in the paged decode")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    nbytes = float(metrics.decode_kv_bytes(r.inp["lengths"], w.g, w.d_h, 2))
+    gbs = nbytes / (ms * 1e-3) * 1e-9
+    del r, Kp, Vp, flush
+    torch.cuda.empty_cache()
+    return {"page_size": page_size, "ms": ms, "value": gbs, "unit": "GB/s",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"hbm_gbs ({peak_kind})",
+                         "kernel": "gqe_attn_decode_paged (decode_partial_kernel paged + decode_combine_kernel)"}}
+
+
 def time_e2e(r, steps, ws, work, scale, unit):
     """Same metric through the public API with host buffers: every step copies
     its inputs from pinned host memory to the device and the output back."""
@@ -580,6 +626,8 @@ def main():
             secondary[name] = {"value": r2["value"], "unit": r2["unit"], "ms_per_step": r2["ms_per_step"],
                                "attn_ms": r2["attn_ms"], "route_ms": r2["route_ms"], "roofline": r2["roofline"],
                                "shape": sw.describe()}
+            if sw.decode:
+                secondary[name]["paged"] = time_paged_decode(sw, max(5, args.steps // 2), 3, peaks, peak_kind)
     layer_ops = None
     if not args.no_secondary and args.workload == PRIMARY:
         layer_ops = time_layer_ops(w, max(5, args.steps // 2), 3, peaks, peak_kind)

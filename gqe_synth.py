@@ -149,6 +149,25 @@ def make_shared_query(w: Workload):
     return _normal((w.B, w.T, w.d_h), gen).to(w.torch_dtype)
 
 
+def make_paged_cache(K_cache, V_cache, page_size: int, seed: int = 4242, spare_pages: int = 3):
+    """Cut contiguous caches [B, Lmax, g, d_h] into pages of page_size rows and
+    scatter them over a pool in a seeded random order (plus a few unused
+    pages).  Returns (K_pages, V_pages [num_pages, page_size, g, d_h],
+    block_table int32 [B, max_blocks]) such that logical row s of sequence b is
+    row s % page_size of page block_table[b, s // page_size]."""
+    B, Lmax, g, d_h = K_cache.shape
+    if Lmax % page_size:
+        raise ValueError("Lmax must be a multiple of page_size")
+    nb = Lmax // page_size
+    num_pages = B * nb + spare_pages
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(seed))[: B * nb]
+    K_pages = torch.zeros((num_pages, page_size, g, d_h), dtype=K_cache.dtype)
+    V_pages = torch.zeros((num_pages, page_size, g, d_h), dtype=V_cache.dtype)
+    K_pages[perm] = K_cache.reshape(B * nb, page_size, g, d_h)
+    V_pages[perm] = V_cache.reshape(B * nb, page_size, g, d_h)
+    return K_pages, V_pages, perm.to(torch.int32).reshape(B, nb)
+
+
 def make_qproj_weight(w: Workload):
     """Query projection W_Q [d_model, h*d_h] ~ N(0, 1/sqrt(d_model)) in the
     workload's dtype (query rows of unit scale), from its own seeded generator

@@ -257,6 +257,30 @@ gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* 
 gqe_status gqe_group_slots(const gqe_shape* s, const void* O, const int32_t* idx, const float* gate, void* O_cat,
                            void* O_wsum, void* stream);
 
+/*
+ * gqe_attn_decode_paged -- gqe_attn_decode with the KV cache in pages.
+ *
+ * The cache stays dense under GQE (gist.science summary, "Chemin KV Dense");
+ * only where its rows sit changes: logical row s of sequence b is row
+ * s % page_size of page block_table[b * max_blocks + s / page_size].  The
+ * result is exactly that of gqe_attn_decode on the gathered cache.
+ *
+ *   K_pages, V_pages [num_pages, page_size, g, d_h]   device, dtype
+ *   page_size        a power of two, 1 .. 65536
+ *   block_table [B, max_blocks]   device int32; entries for rows < lengths[b]
+ *                    must name pages in [0, num_pages) (device-side contract: an
+ *                    entry outside is reported as GQE_ERR_INVALID_ARGUMENT in
+ *                    the status word and read as page 0)
+ *   lengths [B]      device int32, each in [1, page_size * max_blocks]
+ *   q, idx, gate, O  as for gqe_attn_decode
+ *   workspace        at least gqe_workspace_bytes(s, page_size * max_blocks)
+ * Implemented cases: as gqe_attn_decode.
+ */
+gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* K_pages, const void* V_pages,
+                                 int num_pages, int page_size, const int32_t* block_table, int max_blocks,
+                                 const int32_t* lengths, const int32_t* idx, const float* gate, void* O,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, read the workspace status word, reset it to zero and
  * return it (GQE_OK when no kernel reported a failure). */
 gqe_status gqe_get_device_status(void* workspace, void* stream);

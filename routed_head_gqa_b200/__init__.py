@@ -27,7 +27,8 @@ GQE_F32 = 0
 GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
-            "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj",
+            "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
+            "gqe_group_slots", "gqe_routed_qproj",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -69,11 +70,13 @@ def _load():
     lib.gqe_attn_shared_head.argtypes = [S, _P, _P, _P, _I, _P, _P, _SZ, _P]
     lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
     lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_decode_paged.argtypes = [S, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
-              "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_get_device_status"):
+              "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
+              "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -171,6 +174,16 @@ def gqe_attn_shared_head(shape, Qs, K, V, kv_group, Os, workspace, stream=None) 
     _check("gqe_attn_shared_head", _lib.gqe_attn_shared_head(ctypes.byref(shape), _ptr(Qs), _ptr(K), _ptr(V),
                                                              int(kv_group), _ptr(Os), _ptr(workspace),
                                                              _nbytes(workspace), _stream(stream)))
+
+
+def gqe_attn_decode_paged(shape, q, K_pages, V_pages, page_size, block_table, lengths, idx, gate, O, workspace,
+                          stream=None) -> None:
+    num_pages = int(K_pages.shape[0])
+    max_blocks = int(block_table.shape[-1])
+    _check("gqe_attn_decode_paged", _lib.gqe_attn_decode_paged(
+        ctypes.byref(shape), _ptr(q), _ptr(K_pages), _ptr(V_pages), num_pages, int(page_size), _ptr(block_table),
+        max_blocks, _ptr(lengths), _ptr(idx), _ptr(gate), _ptr(O), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)))
 
 
 def gqe_routed_qproj(shape, x, W_Q, head_offsets, head_pos, Q, workspace, stream=None) -> None:

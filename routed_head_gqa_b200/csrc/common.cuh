@@ -182,6 +182,13 @@ struct DecodeArgs {
     float* partials;  // workspace
     void* status;
     cudaStream_t stream;
+    // Paged caches (block_table != null): K_cache/V_cache are [num_pages,
+    // page_size, g, d_h]; logical row s of sequence b is row s % page_size of
+    // page block_table[b * max_blocks + s / page_size]; Lmax = page_size * max_blocks.
+    const int32_t* block_table = nullptr;
+    int max_blocks = 0;
+    int page_shift = 0;  // log2(page_size)
+    int num_pages = 0;
 };
 int decode_chunk_tokens(const gqe_shape* s);
 size_t decode_partials_bytes(const gqe_shape* s, int Lmax);

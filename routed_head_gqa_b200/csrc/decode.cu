@@ -17,17 +17,20 @@ namespace {
 constexpr int kDecodeChunk = 512;   // cache rows per block
 constexpr int kDecodeThreads = 256; // 8 warps; warp w serves groups w, w+8, ...
 constexpr int kDecodeUnroll = 8;    // token steps in flight per lane
+constexpr uint32_t kWhereDecode = 4; // status "where" id of the decode kernels
 
 template <int D>
 struct PartRec {
     static constexpr int kFloats = D + 4;  // acc[D], m, l, pad, pad
 };
 
-template <typename T, int D, int KR>
+template <typename T, int D, int KR, bool PAGED>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
                       const int32_t* __restrict__ lengths, const int32_t* __restrict__ idx, int Lmax,
-                      int h, int g, int k, int nchunk_max, float* __restrict__ part) {
+                      int h, int g, int k, int nchunk_max, float* __restrict__ part,
+                      const int32_t* __restrict__ block_table, int max_blocks, int page_shift, int num_pages,
+                      void* status) {
     constexpr int EPL = 16 / sizeof(T);  // elements per 16-byte vector
     constexpr int LPR = D / EPL;         // lanes per cache row
     constexpr int TPS = 32 / LPR;        // cache rows per warp step
@@ -69,8 +72,25 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T
 #pragma unroll
             for (int e = 0; e < EPL; ++e) acc[r][e] = 0.f;
         }
-        const T* kbase = Kc + (int64_t)b * Lmax * row_stride + (int64_t)grp * D + sub * EPL;
-        const T* vbase = Vc + (int64_t)b * Lmax * row_stride + (int64_t)grp * D + sub * EPL;
+        // Cache row of logical position s: contiguous [B, Lmax] rows, or a row
+        // of a page named by the block table (an entry outside the page pool is
+        // reported and read as page 0, never out of bounds).
+        const int64_t seq_base = PAGED ? 0 : (int64_t)b * Lmax * row_stride;
+        const T* kbase = Kc + seq_base + (int64_t)grp * D + sub * EPL;
+        const T* vbase = Vc + seq_base + (int64_t)grp * D + sub * EPL;
+        const int32_t* bt = PAGED ? block_table + (int64_t)b * max_blocks : nullptr;
+        auto cache_row = [&](int s) -> int64_t {
+            if constexpr (PAGED) {
+                int pg = bt[s >> page_shift];
+                if ((unsigned)pg >= (unsigned)num_pages) {
+                    report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereDecode, (uint32_t)b);
+                    pg = 0;
+                }
+                return ((int64_t)pg << page_shift) + (s & ((1 << page_shift) - 1));
+            } else {
+                return s;  // the sequence's base is in kbase / vbase
+            }
+        };
 
         for (int sb = s0; sb < s1; sb += TPS * kDecodeUnroll) {
             uint4 kv[kDecodeUnroll], vv[kDecodeUnroll];
@@ -80,8 +100,9 @@ decode_partial_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T
                 const int s = sb + u * TPS + slot;
                 valid[u] = s < s1;
                 const int sc = valid[u] ? s : s1 - 1;
-                kv[u] = ld_stream16(kbase + (int64_t)sc * row_stride);
-                vv[u] = ld_stream16(vbase + (int64_t)sc * row_stride);
+                const int64_t row = cache_row(sc);
+                kv[u] = ld_stream16(kbase + row * row_stride);
+                vv[u] = ld_stream16(vbase + row * row_stride);
             }
             float sc_[kDecodeUnroll][KR];
 #pragma unroll
@@ -227,9 +248,14 @@ cudaError_t launch_typed(const DecodeArgs& a) {
     const gqe_shape& s = *a.s;
     const int nchunk_max = (a.Lmax + kDecodeChunk - 1) / kDecodeChunk;
     dim3 grid(nchunk_max, s.B);
-    decode_partial_kernel<T, D, KR><<<grid, kDecodeThreads, 0, a.stream>>>(
-        (const T*)a.q, (const T*)a.K_cache, (const T*)a.V_cache, a.lengths, a.idx, a.Lmax, s.h, s.g, s.k,
-        nchunk_max, a.partials);
+    if (a.block_table != nullptr)
+        decode_partial_kernel<T, D, KR, true><<<grid, kDecodeThreads, 0, a.stream>>>(
+            (const T*)a.q, (const T*)a.K_cache, (const T*)a.V_cache, a.lengths, a.idx, a.Lmax, s.h, s.g, s.k,
+            nchunk_max, a.partials, a.block_table, a.max_blocks, a.page_shift, a.num_pages, a.status);
+    else
+        decode_partial_kernel<T, D, KR, false><<<grid, kDecodeThreads, 0, a.stream>>>(
+            (const T*)a.q, (const T*)a.K_cache, (const T*)a.V_cache, a.lengths, a.idx, a.Lmax, s.h, s.g, s.k,
+            nchunk_max, a.partials, nullptr, 0, 0, 0, a.status);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     dim3 cgrid(s.B, (s.h + kCombineWarps - 1) / kCombineWarps);

@@ -264,6 +264,46 @@ gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cach
     return from_cuda(launch_decode(a));
 }
 
+gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* K_pages, const void* V_pages,
+                                 int num_pages, int page_size, const int32_t* block_table, int max_blocks,
+                                 const int32_t* lengths, const int32_t* idx, const float* gate, void* O,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (s->T != 1 || num_pages < 1 || max_blocks < 1) return GQE_ERR_INVALID_ARGUMENT;
+    if (page_size < 1 || page_size > (1 << 16) || (page_size & (page_size - 1)) != 0) return GQE_ERR_INVALID_ARGUMENT;
+    const int64_t cap = (int64_t)page_size * max_blocks;
+    if (cap >= ((int64_t)1 << 31)) return GQE_ERR_UNSUPPORTED;
+    if (!q || !K_pages || !V_pages || !block_table || !lengths || !idx || !gate || !O) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O)) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+    if (s->k > 8) return GQE_ERR_UNSUPPORTED;
+    if ((int64_t)num_pages * page_size * s->g * s->d_h >= ((int64_t)1 << 40)) return GQE_ERR_UNSUPPORTED;
+    const int Lmax = (int)cap;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + align256(decode_partials_bytes(s, Lmax)));
+    if (st != GQE_OK) return st;
+    DecodeArgs a;
+    a.s = s;
+    a.q = q;
+    a.K_cache = K_pages;
+    a.V_cache = V_pages;
+    a.Lmax = Lmax;
+    a.lengths = lengths;
+    a.idx = idx;
+    a.gate = gate;
+    a.O = O;
+    a.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks;
+    int shift = 0;
+    while ((1 << shift) < page_size) ++shift;
+    a.page_shift = shift;
+    a.num_pages = num_pages;
+    return from_cuda(launch_decode(a));
+}
+
 gqe_status gqe_get_device_status(void* workspace, void* stream) {
     if (!workspace) return GQE_ERR_INVALID_ARGUMENT;
     DeviceStatus host{};

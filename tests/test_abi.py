@@ -140,6 +140,22 @@ def test_routed_qproj_validation():
     assert g._lib.gqe_routed_qproj(ctypes.byref(s64), fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
 
 
+def test_decode_paged_validation():
+    import routed_head_gqa_b200 as g
+
+    fake = 0x10000
+    s1 = g.make_shape(2, 1, 128, 32, 8, 128, 2, g.GQE_BF16)
+    big = 1 << 30
+    call = lambda s, npages, ps, bt, nb: g._lib.gqe_attn_decode_paged(
+        ctypes.byref(s), fake, fake, fake, npages, ps, bt, nb, fake, fake, fake, fake, fake, big, None)
+    assert call(s1, 16, 48, fake, 4) == 1      # page size not a power of two
+    assert call(s1, 16, 0, fake, 4) == 1
+    assert call(s1, 0, 64, fake, 4) == 1       # empty pool
+    assert call(s1, 16, 64, None, 4) == 1      # no block table
+    s2 = g.make_shape(2, 2, 128, 32, 8, 128, 2, g.GQE_BF16)
+    assert call(s2, 16, 64, fake, 4) == 1      # decode: T must be 1
+
+
 def test_unsupported_cases_report_unsupported():
     import routed_head_gqa_b200 as g
 
