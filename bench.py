@@ -46,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "42066333828ea0fa", "bytes_per_launch": 105111040 + 29436928,
+        "sha": "a0a298782a4902f5", "bytes_per_launch": 105195008 + 30063872,
         "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
         "sha": "38d1f07202b92c94", "bytes_per_launch": 2270814604,

@@ -14,6 +14,8 @@ Sources, per function (the same citations are in ``gqe_oracle.c``):
               experts per GQA group, renormalised router probabilities.
   compact  -- the per-(batch, head) packed position lists that the routed
               kernels consume (bookkeeping of the selection made by ``route``).
+  attn_backward, route_backward -- the chain rule through the forward's own
+              steps (attention, gating, renormalised gates, linear router).
   attn_rows, decode -- IBM "Que es la atencion de consultas agrupadas"
               (scaled dot-product attention, 1/sqrt(d_k)), ml-canon "56 GQA /
               MQA" (KV head expansion), freenetmedia.pl "Grouped-Query
@@ -98,9 +100,11 @@ class Oracle:
                                                 i32]
         lib.oracle_qproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_decode_paged.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32]
+        lib.oracle_attn_backward.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P, i32]
+        lib.oracle_route_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, i32]
         for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
                   lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows,
-                  lib.oracle_decode_paged):
+                  lib.oracle_decode_paged, lib.oracle_attn_backward, lib.oracle_route_backward):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = lib_path
@@ -259,6 +263,58 @@ class Oracle:
             raise ValueError(f"oracle_decode_paged failed ({rc})")
         return out
 
+    def attn_backward(self, Q, K, V, idx, gate, dO, n_threads=None):
+        """Backward of the routed attention for output gradient dO [B, T, h, d_h]:
+        returns (dQ [B,T,h,d_h], dK [B,T,g,d_h], dV [B,T,g,d_h], dgate [B,T,g,k]),
+        all float64."""
+        qa, dt = _as_input(Q)
+        ka, dk = _as_input(K)
+        va, dv = _as_input(V)
+        if not (dt == dk == dv):
+            raise TypeError("Q, K and V must share a dtype")
+        B, T, h, d_h = qa.shape
+        g = ka.shape[2]
+        ia = np.ascontiguousarray(idx, dtype=np.int32).reshape(B, T, g, -1)
+        ga = np.ascontiguousarray(gate, dtype=np.float64).reshape(B, T, g, -1)
+        k = ia.shape[-1]
+        da = np.ascontiguousarray(np.asarray(dO, dtype=np.float64)).reshape(B, T, h, d_h)
+        dQ = np.empty((B, T, h, d_h), np.float64)
+        dK = np.empty((B, T, g, d_h), np.float64)
+        dV = np.empty((B, T, g, d_h), np.float64)
+        dgate = np.empty((B, T, g, k), np.float64)
+        rc = self.lib.oracle_attn_backward(B, T, h, g, d_h, k, dt, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ia), _ptr(ga),
+                                           _ptr(da), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dgate), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_attn_backward failed ({rc})")
+        return dQ, dK, dV, dgate
+
+    def route_backward(self, x, W_r, idx, gate, dgate, n_threads=None):
+        """Router backward for gate gradient dgate [..., g, k]: returns
+        (dlogits [..., h], dx [..., d_model], dW_r [d_model, h], dbias [h]),
+        all float64."""
+        xa, dt = _as_input(x)
+        wa, dt2 = _as_input(W_r)
+        if dt != dt2:
+            raise TypeError("x and W_r must share a dtype")
+        lead = xa.shape[:-1]
+        d_model = xa.shape[-1]
+        h = wa.shape[1]
+        BT = int(np.prod(lead)) if lead else 1
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        g, k = ia.shape[-2], ia.shape[-1]
+        ia = ia.reshape(BT, g, k)
+        ga = np.ascontiguousarray(gate, dtype=np.float64).reshape(BT, g, k)
+        dga = np.ascontiguousarray(dgate, dtype=np.float64).reshape(BT, g, k)
+        dl = np.empty((BT, h), np.float64)
+        dx = np.empty((BT, d_model), np.float64)
+        dW = np.empty((d_model, h), np.float64)
+        db = np.empty((h,), np.float64)
+        rc = self.lib.oracle_route_backward(BT, d_model, h, g, k, dt, _ptr(xa), _ptr(wa), _ptr(ia), _ptr(ga),
+                                            _ptr(dga), _ptr(dl), _ptr(dx), _ptr(dW), _ptr(db), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_route_backward failed ({rc})")
+        return dl.reshape(*lead, h), dx.reshape(*lead, d_model), dW, db
+
     def attn(self, Q, K, V, idx, gate, n_threads=None):
         """Full GQE output O [B, T, h, d_h] (float64)."""
         B, T, h, d_h = tuple(Q.shape)
@@ -330,3 +386,11 @@ def qproj_rows(*a, **kw):
 
 def decode_paged(*a, **kw):
     return default().decode_paged(*a, **kw)
+
+
+def attn_backward(*a, **kw):
+    return default().attn_backward(*a, **kw)
+
+
+def route_backward(*a, **kw):
+    return default().route_backward(*a, **kw)

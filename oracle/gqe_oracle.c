@@ -51,6 +51,9 @@
  *    query-side computation is conditional on the routing): the query row of
  *    head j is x . W_Q[:, j*d_h : (j+1)*d_h], computed only for the heads a
  *    token selected.
+ *  - Backward (training; the pages state no formula for it): the gradients of
+ *    the routed attention, of the gates and of the router's logits, x, W_r and
+ *    bias, by the chain rule through the steps above in reverse order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -489,4 +492,183 @@ int oracle_decode_paged(int B, int page_size, int max_blocks, int num_pages, int
         free(scores);
     }
     return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass (training): the chain rule through the forward above.      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Gradients of a loss whose gradient with respect to the layer output O is dO,
+ * taken term by term through the forward's own steps for one routed (b, t, j)
+ * with gate gm, softmax weights p_s over keys s <= t and attention output o:
+ *   O = gm * o                 ->  dgm = dO . o,   do = gm * dO
+ *   o = sum_s p_s v_s          ->  dV[b,s,q] += p_s * do,   dp_s = do . v_s
+ *   p = softmax(z),  z_s = q . k_s / sqrt(d_h)
+ *                              ->  dz_s = p_s * (dp_s - sum_r p_r dp_r)
+ *                              ->  dQ[b,t,j] = sum_s dz_s k_s / sqrt(d_h)
+ *                                  dK[b,s,q] += dz_s q / sqrt(d_h)
+ * An unselected slot of O is the constant 0, so it passes no gradient.
+ *
+ * Q [B,T,h,d_h], K/V [B,T,g,d_h] (dtype); idx/gate [B,T,g,k]; dO [B,T,h,d_h]
+ * Out, double: dQ [B,T,h,d_h] (0 in unselected slots), dK/dV [B,T,g,d_h],
+ *              dgate [B,T,g,k].
+ */
+int oracle_attn_backward(int B, int T, int h, int g, int d_h, int k, int dtype,
+                         const void* Q, const void* K, const void* V,
+                         const int32_t* idx, const double* gate, const double* dO,
+                         double* dQ, double* dK, double* dV, double* dgate, int n_threads) {
+    if (B < 0 || T < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    const double scale = 1.0 / sqrt((double)d_h);
+    const size_t kv_stride = (size_t)g * d_h;
+    int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)T);
+        double* dp = (double*)malloc(sizeof(double) * (size_t)T);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d_h);
+        double* dov = (double*)malloc(sizeof(double) * (size_t)d_h);
+        if (!p || !dp || !o || !dov) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+            /* one (b, group) per iteration: it alone writes dK/dV of that group */
+#pragma omp for schedule(dynamic, 1) collapse(2)
+            for (int b = 0; b < B; ++b) {
+                for (int q = 0; q < g; ++q) {
+                    const size_t kv_base = ((size_t)b * T * g + q) * d_h;
+                    for (int t = 0; t < T; ++t) {
+                        for (int d = 0; d < d_h; ++d) {
+                            dK[kv_base + (size_t)t * kv_stride + d] = 0.0;
+                            dV[kv_base + (size_t)t * kv_stride + d] = 0.0;
+                        }
+                        for (int jj = 0; jj < hpg; ++jj)
+                            for (int d = 0; d < d_h; ++d)
+                                dQ[(((size_t)b * T + t) * h + q * hpg + jj) * d_h + d] = 0.0;
+                    }
+                    for (int t = 0; t < T; ++t) {
+                        for (int s_ = 0; s_ < k; ++s_) {
+                            const size_t sel = (((size_t)b * T + t) * g + q) * k + s_;
+                            const int j = idx[sel];
+                            const size_t q_off = (((size_t)b * T + t) * h + j) * d_h;
+                            /* forward: softmax weights and output */
+                            double mx = -INFINITY;
+                            for (int s = 0; s <= t; ++s) {
+                                double dot = 0.0;
+                                for (int d = 0; d < d_h; ++d)
+                                    dot += load_elem(Q, q_off + d, dtype) *
+                                           load_elem(K, kv_base + (size_t)s * kv_stride + d, dtype);
+                                p[s] = dot * scale;
+                                if (p[s] > mx) mx = p[s];
+                            }
+                            double denom = 0.0;
+                            for (int s = 0; s <= t; ++s) {
+                                p[s] = exp(p[s] - mx);
+                                denom += p[s];
+                            }
+                            for (int s = 0; s <= t; ++s) p[s] /= denom;
+                            for (int d = 0; d < d_h; ++d) o[d] = 0.0;
+                            for (int s = 0; s <= t; ++s)
+                                for (int d = 0; d < d_h; ++d)
+                                    o[d] += p[s] * load_elem(V, kv_base + (size_t)s * kv_stride + d, dtype);
+                            /* O = gate * o */
+                            double dg = 0.0;
+                            for (int d = 0; d < d_h; ++d) dg += dO[q_off + d] * o[d];
+                            dgate[sel] = dg;
+                            for (int d = 0; d < d_h; ++d) dov[d] = gate[sel] * dO[q_off + d];
+                            /* o = sum_s p_s v_s */
+                            double pdp = 0.0;
+                            for (int s = 0; s <= t; ++s) {
+                                const size_t kr = kv_base + (size_t)s * kv_stride;
+                                double acc = 0.0;
+                                for (int d = 0; d < d_h; ++d) {
+                                    dV[kr + d] += p[s] * dov[d];
+                                    acc += dov[d] * load_elem(V, kr + d, dtype);
+                                }
+                                dp[s] = acc;
+                                pdp += p[s] * acc;
+                            }
+                            /* p = softmax(z), z = q . k / sqrt(d_h) */
+                            for (int s = 0; s <= t; ++s) {
+                                const size_t kr = kv_base + (size_t)s * kv_stride;
+                                const double dz = p[s] * (dp[s] - pdp);
+                                for (int d = 0; d < d_h; ++d) {
+                                    dQ[q_off + d] += scale * dz * load_elem(K, kr + d, dtype);
+                                    dK[kr + d] += scale * dz * load_elem(Q, q_off + d, dtype);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+        free(o);
+        free(dov);
+    }
+    return err;
+}
+
+/*
+ * Router backward.  The gates are a softmax over the selected logits
+ * (gate_j = exp(l_j) / sum_{i in S} exp(l_i)), so for j in S
+ *   dl_j = gate_j * (dgate_j - sum_{i in S} gate_i dgate_i)
+ * and dl_j = 0 for an unselected head (the top-k choice is piecewise constant
+ * in the logits; the fp32 rounding of the logits is not differentiated).  Then
+ * l = x . W_r + bias gives dx = dl . W_r^T, dW_r = x^T . dl, dbias = sum dl.
+ *
+ * x [BT, d_model], W_r [d_model, h] (dtype); idx/gate/dgate [BT, g, k]
+ * Out, double: dlogits [BT, h]; dx [BT, d_model], dW [d_model, h] and
+ * dbias [h] (each may be NULL to skip it).
+ */
+int oracle_route_backward(int64_t BT, int d_model, int h, int g, int k, int dtype,
+                          const void* x, const void* W_r, const int32_t* idx,
+                          const double* gate, const double* dgate, double* dlogits,
+                          double* dx, double* dW, double* dbias, int n_threads) {
+    if (BT < 0 || d_model < 1 || h < 1 || g < 1 || h % g != 0) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    for (int64_t i = 0; i < BT * g * k; ++i)
+        if (idx[i] < 0 || idx[i] >= h || idx[i] / hpg != (int)((i / k) % g)) return 1;
+    for (int64_t bt = 0; bt < BT; ++bt) {
+        for (int j = 0; j < h; ++j) dlogits[bt * h + j] = 0.0;
+        for (int q = 0; q < g; ++q) {
+            const size_t base = ((size_t)bt * g + q) * k;
+            double mean = 0.0;
+            for (int s = 0; s < k; ++s) mean += gate[base + s] * dgate[base + s];
+            for (int s = 0; s < k; ++s)
+                dlogits[bt * h + idx[base + s]] = gate[base + s] * (dgate[base + s] - mean);
+        }
+    }
+    if (dx) {
+#pragma omp parallel for num_threads(n_threads > 0 ? n_threads : 1) schedule(static)
+        for (int64_t bt = 0; bt < BT; ++bt)
+            for (int i = 0; i < d_model; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < h; ++j)
+                    acc += dlogits[bt * h + j] * load_elem(W_r, (size_t)i * h + j, dtype);
+                dx[bt * d_model + i] = acc;
+            }
+    }
+    if (dW) {
+#pragma omp parallel for num_threads(n_threads > 0 ? n_threads : 1) schedule(static)
+        for (int i = 0; i < d_model; ++i)
+            for (int j = 0; j < h; ++j) {
+                double acc = 0.0;
+                for (int64_t bt = 0; bt < BT; ++bt)
+                    acc += load_elem(x, (size_t)bt * d_model + i, dtype) * dlogits[bt * h + j];
+                dW[(size_t)i * h + j] = acc;
+            }
+    }
+    if (dbias) {
+        for (int j = 0; j < h; ++j) {
+            double acc = 0.0;
+            for (int64_t bt = 0; bt < BT; ++bt) acc += dlogits[bt * h + j];
+            dbias[j] = acc;
+        }
+    }
+    return 0;
 }

@@ -539,9 +539,157 @@ def check_decode_paged(o):
     _ = hpg
 
 
+# --------------------------------------------------------------------------
+# Backward (training)
+# --------------------------------------------------------------------------
+
+def _gate_mask(idx, gate, h):
+    """[B, T, h] with gate_j in selected slots and 0 elsewhere."""
+    B, T, g, k = idx.shape
+    m = np.zeros((B, T, h))
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                for s in range(k):
+                    m[b, t, idx[b, t, q_, s]] = gate[b, t, q_, s]
+    return m
+
+
+def check_backward_sdpa_autograd(o):
+    """dQ, dK, dV, dgate = torch autograd (fp64) of sum(dO * mask * SDPA(causal, GQA)),
+    mask = gate in selected slots, 0 elsewhere: a library routine's own backward."""
+    for (B, T, h, g, d, k, seed) in [(2, 13, 8, 2, 8, 2, 600), (1, 17, 6, 3, 4, 1, 601), (1, 9, 4, 1, 8, 4, 602)]:
+        Q = _f32((B, T, h, d), seed)
+        K = _f32((B, T, g, d), seed + 1)
+        V = _f32((B, T, g, d), seed + 2)
+        idx, gate = _random_routing(B, T, h, g, k, seed + 3)
+        dO = _rng(seed + 4).standard_normal((B, T, h, d))
+        dQ, dK, dV, dgate = o.attn_backward(Q, K, V, idx, gate, dO)
+        q = torch.from_numpy(Q.astype(np.float64)).transpose(1, 2).requires_grad_()
+        kk = torch.from_numpy(K.astype(np.float64)).transpose(1, 2).requires_grad_()
+        vv = torch.from_numpy(V.astype(np.float64)).transpose(1, 2).requires_grad_()
+        full = F.scaled_dot_product_attention(q, kk, vv, is_causal=True, enable_gqa=True).transpose(1, 2)
+        m = torch.from_numpy(_gate_mask(idx, gate, h))[..., None]
+        (full * m * torch.from_numpy(dO)).sum().backward()
+        for name, got, want in (("dQ", dQ, q.grad.transpose(1, 2)), ("dK", dK, kk.grad.transpose(1, 2)),
+                                ("dV", dV, vv.grad.transpose(1, 2))):
+            err = np.abs(got - want.numpy()).max()
+            assert err < 1e-12, f"{name} vs autograd: {err}"
+        fo = full.detach().numpy()
+        for b in range(B):
+            for t in range(T):
+                for q_ in range(g):
+                    for s in range(k):
+                        j = idx[b, t, q_, s]
+                        want = float(np.dot(dO[b, t, j], fo[b, t, j]))
+                        assert abs(dgate[b, t, q_, s] - want) < 1e-12, "dgate vs SDPA output"
+
+
+def _central(f, a, i, eps):
+    """Central difference of f along element i of the fp32 array a, dividing by
+    the step actually taken after rounding to fp32."""
+    x0 = a.flat[i]
+    ap, am = a.copy(), a.copy()
+    ap.flat[i] = np.float32(x0 + eps)
+    am.flat[i] = np.float32(x0 - eps)
+    return (f(ap) - f(am)) / (float(ap.flat[i]) - float(am.flat[i]))
+
+
+def check_backward_finite_differences(o):
+    """Gradients of L = sum(dO * O) against central differences of the forward
+    oracle, for Q, K, V, the gates, and (through the router) x, W_r and bias.
+    Two routings: every head of a group selected (k = h/g), and 2 of 3."""
+    for (B, T, h, g, d, k, d_model, seed) in [(1, 6, 4, 2, 4, 2, 5, 610), (1, 5, 6, 2, 4, 2, 5, 670)]:
+        _fd_case(o, B, T, h, g, d, k, d_model, seed)
+
+
+def _fd_case(o, B, T, h, g, d, k, d_model, seed):
+    Q = _f32((B, T, h, d), seed)
+    K = _f32((B, T, g, d), seed + 1)
+    V = _f32((B, T, g, d), seed + 2)
+    dO = _rng(seed + 3).standard_normal((B, T, h, d))
+    x = _f32((B, T, d_model), seed + 4)
+    W = _f32((d_model, h), seed + 5, 0.7)
+    bias = _f32((h,), seed + 6, 0.3)
+    idx, gate, _, margin = o.route(x, W, h, g, k, bias=bias)
+    assert margin.min() > 0.05 or k == h // g, "test inputs must keep the selection away from ties"
+    dQ, dK, dV, dgate = o.attn_backward(Q, K, V, idx, gate, dO)
+    eps = 1e-3
+    tol = 2e-6
+    for name, arr, grad in (("Q", Q, dQ), ("K", K, dK), ("V", V, dV)):
+        def loss(a, name=name):
+            args = {"Q": Q, "K": K, "V": V}
+            args[name] = a
+            return float((o.attn(args["Q"], args["K"], args["V"], idx, gate) * dO).sum())
+        for i in range(arr.size):
+            fd = _central(loss, arr, i, eps)
+            assert abs(fd - grad.flat[i]) < tol * (1 + abs(fd)), f"d{name}[{i}]: fd {fd} vs {grad.flat[i]}"
+    for i in range(gate.size):  # O is linear in each gate
+        gp, gm = gate.copy(), gate.copy()
+        gp.flat[i] += 0.5
+        gm.flat[i] -= 0.5
+        fd = float(((o.attn(Q, K, V, idx, gp) - o.attn(Q, K, V, idx, gm)) * dO).sum())
+        assert abs(fd - dgate.flat[i]) < 1e-10 * (1 + abs(fd)), f"dgate[{i}]"
+    dl, dx, dW, db = o.route_backward(x, W, idx, gate, dgate)
+
+    def layer(xx, WW, bb):
+        i2, g2, _, _ = o.route(xx, WW, h, g, k, bias=bb)
+        assert np.array_equal(i2, idx), "a finite-difference step changed the selection"
+        return float((o.attn(Q, K, V, i2, g2) * dO).sum())
+    eps_r, tol_r = 1e-2, 2e-4  # the router's fp32 logits add rounding noise to each difference
+    for name, arr, grad in (("x", x, dx), ("W_r", W, dW), ("bias", bias, db)):
+        def loss(a, name=name):
+            args = {"x": x, "W_r": W, "bias": bias}
+            args[name] = a
+            return layer(args["x"], args["W_r"], args["bias"])
+        for i in range(arr.size):
+            fd = _central(loss, arr, i, eps_r)
+            assert abs(fd - grad.flat[i]) < tol_r * (1 + abs(fd)), f"d{name}[{i}]: fd {fd} vs {grad.flat[i]}"
+
+
+def check_backward_invariants(o):
+    """Softmax shift invariance: each attention row's score gradients sum to 0,
+    so sum_s dK[b,s,q] = 0, and each group's logit gradients sum to 0.  Closed
+    forms with K = 0 (uniform weights): dQ = 0 and
+    dV[b,s,q] = sum_{t>=s} sum_{j in S(t,q)} gate_j dO[b,t,j] / (t+1).
+    With one head per group (g = h) the gate is 1 and the logit gradient 0."""
+    B, T, h, g, d, k = 2, 10, 6, 2, 8, 2
+    Q = _f32((B, T, h, d), 620)
+    K = _f32((B, T, g, d), 621)
+    V = _f32((B, T, g, d), 622)
+    idx, gate = _random_routing(B, T, h, g, k, 623)
+    dO = _rng(624).standard_normal((B, T, h, d))
+    dQ, dK, dV, dgate = o.attn_backward(Q, K, V, idx, gate, dO)
+    assert np.abs(dK.sum(axis=1)).max() < 1e-12, "sum_s dK != 0"
+    sel = _gate_mask(idx, gate, h) > 0
+    assert np.all(dQ[~sel] == 0.0), "dQ of an unselected slot"
+    x = _f32((B, T, 7), 625)
+    W = _f32((7, h), 626)
+    dl, _, _, _ = o.route_backward(x, W, idx, gate, dgate)
+    assert np.abs(dl.reshape(B, T, g, h // g).sum(axis=-1)).max() < 1e-12, "sum of a group's dlogits != 0"
+    assert np.all(dl[~sel] == 0.0), "dlogit of an unselected head"
+    dQ0, _, dV0, dg0 = o.attn_backward(Q, np.zeros_like(K), V, idx, gate, dO)
+    assert np.abs(dQ0).max() < 1e-13, "dQ with K = 0"
+    want = np.zeros_like(dV0)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                for s in range(k):
+                    j = idx[b, t, q_, s]
+                    want[b, : t + 1, q_] += gate[b, t, q_, s] * dO[b, t, j] / (t + 1)
+                    assert abs(dg0[b, t, q_, s] - np.dot(dO[b, t, j], V[b, : t + 1, q_].astype(np.float64).mean(0))) < 1e-12
+    assert np.abs(dV0 - want).max() < 1e-12, "dV with K = 0"
+    i1 = np.broadcast_to(np.arange(h, dtype=np.int32).reshape(1, 1, h, 1), (B, T, h, 1)).copy()
+    g1 = np.ones((B, T, h, 1))
+    _, _, _, dg1 = o.attn_backward(Q, np.repeat(K, 3, axis=2), np.repeat(V, 3, axis=2), i1, g1, dO)
+    dl1, _, _, _ = o.route_backward(x, W, i1, g1, dg1)
+    assert np.all(dl1 == 0.0), "one head per group: the logit gradient must be 0"
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
     check_shared_head_closed_forms, check_group_slots, check_qproj, check_decode_paged,
+    check_backward_sdpa_autograd, check_backward_finite_differences, check_backward_invariants,
 ]

@@ -43,6 +43,19 @@ MUTANTS = [
      "const size_t row = ((pg * page_size + (size_t)((s + 1) % page_size)) * g + q) * d_h;"),
     ("paged_block_lookup", "(size_t)block_table[(size_t)b * max_blocks + s / page_size];",
      "(size_t)block_table[(size_t)b * max_blocks + (s / page_size) % 2];"),
+    ("bwd_drops_softmax_mean", "const double dz = p[s] * (dp[s] - pdp);", "const double dz = p[s] * dp[s];"),
+    ("bwd_output_grad_ungated", "dov[d] = gate[sel] * dO[q_off + d];", "dov[d] = dO[q_off + d];"),
+    ("bwd_dk_from_key", "dK[kr + d] += scale * dz * load_elem(Q, q_off + d, dtype);",
+     "dK[kr + d] += scale * dz * load_elem(K, kr + d, dtype);"),
+    ("bwd_dq_unscaled", "dQ[q_off + d] += scale * dz * load_elem(K, kr + d, dtype);",
+     "dQ[q_off + d] += dz * load_elem(K, kr + d, dtype);"),
+    ("bwd_dv_uniform_weights", "dV[kr + d] += p[s] * dov[d];", "dV[kr + d] += dov[d] / (double)(t + 1);"),
+    ("router_bwd_drops_mean", "gate[base + s] * (dgate[base + s] - mean);", "gate[base + s] * dgate[base + s];"),
+    ("router_bwd_dx_transposed", "acc += dlogits[bt * h + j] * load_elem(W_r, (size_t)i * h + j, dtype);",
+     "acc += dlogits[bt * h + j] * load_elem(W_r, ((size_t)j * d_model + i) % ((size_t)d_model * h), dtype);"),
+    ("router_bwd_dw_wrong_head", "acc += load_elem(x, (size_t)bt * d_model + i, dtype) * dlogits[bt * h + j];",
+     "acc += load_elem(x, (size_t)bt * d_model + i, dtype) * dlogits[bt * h + (j + 1) % h];"),
+    ("router_bwd_dbias_halved", "dbias[j] = acc;", "dbias[j] = 0.5 * acc;"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
