@@ -80,7 +80,7 @@ print("FAILED:" + ",".join(failed))
 def test_mutant_is_caught(tmp_path, name, old, new):
     src = open(oracle.SOURCE).read()
     assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
-    mutated = src.replace(old, new)
+    mutated = src.replace(old, new, 1)  # one planted mistake, at the anchor's first occurrence
     c_path = tmp_path / "mutant.c"
     c_path.write_text(mutated)
     lib = str(tmp_path / "libmutant.so")
