@@ -409,6 +409,60 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
     }
 
 
+FP32_LANES_PER_SM = 128  # B200: 4 sub-partitions x 32 fp32 FMA lanes
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+
+
+def time_backward(w, steps, warmup, peaks, peak_kind):
+    """The routed attention's backward (gqe_attn_prefill_backward) on the
+    workload's shapes, after one forward step, timed alone with CUDA events (L2
+    flushed before each call, outside the events).  Algorithmic FLOPs: the
+    five contractions of an attention backward over the visible (row, key)
+    pairs of the routed rows, 2.5x the forward's 4*d_h per pair.  The kernels
+    run on the fp32 CUDA cores, so the roofline is the fp32 FMA peak (148 SMs x
+    128 lanes x 2 FLOP x the 1965 MHz SM clock), with the fraction of the bf16
+    tensor peak given beside it."""
+    from routed_head_gqa_b200 import metrics
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    r = Runner(w, dev)
+    r.step()
+    dO = gqe_synth.make_output_grad(w).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def fn():
+        r.buf.backward(r.d["Q"], r.d["K"], r.d["V"], dO)
+
+    for _ in range(warmup):
+        l2_flush(flush)
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        l2_flush(flush)
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    st = r.buf.backward_status()
+    if st != 0:
+        raise RuntimeError(f"device status {r.g.gqe_status_string(st)} in the backward")
+    flops = 2.5 * metrics.prefill_active_flops(w.B, w.T, w.g, w.k, w.d_h)
+    tf = flops / (ms * 1e-3) * 1e-12
+    alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 * 1e-12
+    del r, flush
+    torch.cuda.empty_cache()
+    return {"ms": ms, "value": tf, "unit": "TFLOP/s", "flops": flops, "launches": 3,
+            "roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(tf / alu_peak, 4),
+                         "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz (derived)",
+                         "frac_of_bf16_tensor": round(tf / peaks["bf16_tflops"], 4),
+                         "kernel": "gqe_attn_prefill_backward (bwd_dq_kernel + bwd_rows_kernel + bwd_dkdv_kernel)"},
+            "shape": w.describe()}
+
+
 def time_paged_decode(w, steps, warmup, peaks, peak_kind, page_size=256):
     """The decode workload with its caches cut into pages of page_size rows,
     scattered over the pool in a seeded random order (gqe_attn_decode_paged),
@@ -576,6 +630,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layer-ops-only", action="store_true",
                     help="time only the calls around the routed attention (for profiling)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the routed attention's backward (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -606,6 +662,15 @@ def main():
         gqe_build.build()
     barrier(ws)
     peaks, peak_kind = load_peaks()
+    if args.backward_only:
+        bw = time_backward(w, args.steps, args.warmup, peaks, peak_kind)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "gqe_backward": bw}))
+        if ws > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
     if args.layer_ops_only:
         ops = time_layer_ops(w, args.steps, args.warmup, peaks, peak_kind)
         if rank == 0:
@@ -631,6 +696,7 @@ def main():
     layer_ops = None
     if not args.no_secondary and args.workload == PRIMARY:
         layer_ops = time_layer_ops(w, max(5, args.steps // 2), 3, peaks, peak_kind)
+        layer_ops["backward"] = time_backward(w, 3, 3, peaks, peak_kind)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)

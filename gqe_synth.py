@@ -176,6 +176,14 @@ def make_qproj_weight(w: Workload):
     return _normal((w.d_model, w.h * w.d_h), gen, std=1.0 / math.sqrt(w.d_model)).to(w.torch_dtype)
 
 
+def make_output_grad(w: Workload):
+    """Incoming gradient dO [B,T,h,d_h] ~ N(0,1) in the workload's dtype (a
+    stand-in for the gradient a training step would bring back), from its own
+    seeded generator (seed + 31337)."""
+    gen = torch.Generator().manual_seed(w.seed + 31337)
+    return _normal((w.B, w.T, w.h, w.d_h), gen).to(w.torch_dtype)
+
+
 def sample_rows(w: Workload, n: int, seed: int = 1234):
     """A seeded sample of n flattened token rows (b*T + t) that always includes
     the last position of every sequence and the first position of batch 0."""

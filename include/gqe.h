@@ -281,6 +281,44 @@ gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* 
                                  const int32_t* lengths, const int32_t* idx, const float* gate, void* O,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gqe_attn_prefill_backward -- gradients of the routed attention and of the
+ * gates, for training.
+ *
+ * The pages state no backward; this is the chain rule through
+ * gqe_attn_prefill and the renormalised gates of gqe_route (gist.science
+ * summary, "Architecture et Routage", "Somme Ponderee Renormalisee"; IBM "Que
+ * es la atencion de consultas agrupadas" for the attention).  For a routed
+ * (b,t,j) with gate gm, attention output o (O = gm * o), incoming gradient
+ * dO, D = dO . O and p_s the attention weights over keys s <= t:
+ *   dQ[b,t,j]    = sum_s p_s (gm dO . v_s - D) k_s / sqrt(d_h)
+ *   dK[b,s,q]   += p_s (gm dO . v_s - D) q / sqrt(d_h),  dV[b,s,q] += p_s gm dO
+ *   dlogits[b,t,j] = D_j - gm_j sum_{i in S(b,t,q)} D_i   (0 when j is not in S)
+ * dlogits is the gradient with respect to the router logits through the
+ * renormalised gates (the top-k choice itself has no gradient).
+ *
+ *   Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets
+ *                        as passed to gqe_attn_prefill (device)
+ *   dO [B,T,h,d_h]       device, dtype: gradient of the loss with respect to O
+ *                        (o is recomputed in fp32, so the forward's output is
+ *                        not an input)
+ *   dQ [B,T,h,d_h]       device float32 out (0 in unselected slots)
+ *   dK, dV [B,T,g,d_h]   device float32 out
+ *   dlogits [B,T,h]      device float32 out
+ *   workspace            at least gqe_attn_backward_workspace_bytes(s) bytes,
+ *                        256-byte aligned; its first 256 bytes are the status word
+ * Implemented cases: bf16 or fp32, d_h in {32, 64, 128}, k <= 16, h <= 256,
+ * B*h <= 65535; others return GQE_ERR_UNSUPPORTED.  All of Q, K, V, dO, dQ,
+ * dK, dV must be 16-byte aligned.  An index outside its group, or a
+ * position outside [0, T), is reported in the status word and skipped.
+ */
+size_t gqe_attn_backward_workspace_bytes(const gqe_shape* s);
+gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                     const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                     const int32_t* head_pos, const int32_t* head_chunk_offsets, const void* dO,
+                                     float* dQ, float* dK, float* dV, float* dlogits, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, read the workspace status word, reset it to zero and
  * return it (GQE_OK when no kernel reported a failure). */
 gqe_status gqe_get_device_status(void* workspace, void* stream);

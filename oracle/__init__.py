@@ -100,7 +100,8 @@ class Oracle:
                                                 i32]
         lib.oracle_qproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_decode_paged.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32]
-        lib.oracle_attn_backward.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P, i32]
+        lib.oracle_attn_backward.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P,
+                                             i32]
         lib.oracle_route_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, i32]
         for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
                   lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows,
@@ -263,10 +264,12 @@ class Oracle:
             raise ValueError(f"oracle_decode_paged failed ({rc})")
         return out
 
-    def attn_backward(self, Q, K, V, idx, gate, dO, n_threads=None):
+    def attn_backward(self, Q, K, V, idx, gate, dO, t_min=0, n_threads=None):
         """Backward of the routed attention for output gradient dO [B, T, h, d_h]:
         returns (dQ [B,T,h,d_h], dK [B,T,g,d_h], dV [B,T,g,d_h], dgate [B,T,g,k]),
-        all float64."""
+        all float64.  With t_min > 0 only query rows t >= t_min contribute: key
+        rows s >= t_min of dK/dV and query rows t >= t_min of dQ/dgate are then
+        exact (earlier key rows hold a partial sum, earlier query rows 0)."""
         qa, dt = _as_input(Q)
         ka, dk = _as_input(K)
         va, dv = _as_input(V)
@@ -282,7 +285,7 @@ class Oracle:
         dK = np.empty((B, T, g, d_h), np.float64)
         dV = np.empty((B, T, g, d_h), np.float64)
         dgate = np.empty((B, T, g, k), np.float64)
-        rc = self.lib.oracle_attn_backward(B, T, h, g, d_h, k, dt, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ia), _ptr(ga),
+        rc = self.lib.oracle_attn_backward(B, T, h, g, d_h, k, dt, int(t_min), _ptr(qa), _ptr(ka), _ptr(va), _ptr(ia), _ptr(ga),
                                            _ptr(da), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dgate), _threads(n_threads))
         if rc:
             raise ValueError(f"oracle_attn_backward failed ({rc})")

@@ -513,14 +513,18 @@ int oracle_decode_paged(int B, int page_size, int max_blocks, int num_pages, int
  * Q [B,T,h,d_h], K/V [B,T,g,d_h] (dtype); idx/gate [B,T,g,k]; dO [B,T,h,d_h]
  * Out, double: dQ [B,T,h,d_h] (0 in unselected slots), dK/dV [B,T,g,d_h],
  *              dgate [B,T,g,k].
+ * t_min: only query rows t >= t_min contribute (0: all).  Key rows s >= t_min
+ * of dK/dV and query rows t >= t_min of dQ/dgate are then the full result's,
+ * since no earlier query row sees a later key; earlier key rows hold only the
+ * later query rows' share, and earlier rows of dQ/dgate are 0.
  */
-int oracle_attn_backward(int B, int T, int h, int g, int d_h, int k, int dtype,
+int oracle_attn_backward(int B, int T, int h, int g, int d_h, int k, int dtype, int t_min,
                          const void* Q, const void* K, const void* V,
                          const int32_t* idx, const double* gate, const double* dO,
                          double* dQ, double* dK, double* dV, double* dgate, int n_threads) {
     if (B < 0 || T < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
     const int hpg = h / g;
-    if (k < 1 || k > hpg) return 1;
+    if (k < 1 || k > hpg || t_min < 0) return 1;
     const double scale = 1.0 / sqrt((double)d_h);
     const size_t kv_stride = (size_t)g * d_h;
     int err = 0;
@@ -551,6 +555,10 @@ int oracle_attn_backward(int B, int T, int h, int g, int d_h, int k, int dtype,
                     for (int t = 0; t < T; ++t) {
                         for (int s_ = 0; s_ < k; ++s_) {
                             const size_t sel = (((size_t)b * T + t) * g + q) * k + s_;
+                            if (t < t_min) {
+                                dgate[sel] = 0.0;
+                                continue;
+                            }
                             const int j = idx[sel];
                             const size_t q_off = (((size_t)b * T + t) * h + j) * d_h;
                             /* forward: softmax weights and output */

@@ -28,7 +28,7 @@ GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
-            "gqe_group_slots", "gqe_routed_qproj",
+            "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_backward_workspace_bytes", "gqe_attn_prefill_backward",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -71,12 +71,15 @@ def _load():
     lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
     lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode_paged.argtypes = [S, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_backward_workspace_bytes.argtypes = [S]
+    lib.gqe_attn_backward_workspace_bytes.restype = _SZ
+    lib.gqe_attn_prefill_backward.argtypes = [S] + [_P] * 14 + [_SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
-              "gqe_get_device_status"):
+              "gqe_attn_prefill_backward", "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -164,6 +167,19 @@ def gqe_attn_prefill(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chu
                                                      _nbytes(workspace), _stream(stream)))
 
 
+def gqe_attn_backward_workspace_bytes(shape) -> int:
+    return int(_lib.gqe_attn_backward_workspace_bytes(ctypes.byref(shape)))
+
+
+def gqe_attn_prefill_backward(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, dO, dQ, dK, dV,
+                              dlogits, workspace, stream=None) -> None:
+    _check("gqe_attn_prefill_backward",
+           _lib.gqe_attn_prefill_backward(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(gate),
+                                          _ptr(head_offsets), _ptr(head_pos), _ptr(head_chunk_offsets),
+                                          _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dlogits), _ptr(workspace),
+                                          _nbytes(workspace), _stream(stream)))
+
+
 def gqe_attn_decode(shape, q, K_cache, V_cache, Lmax, lengths, idx, gate, O, workspace, stream=None) -> None:
     _check("gqe_attn_decode", _lib.gqe_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache),
                                                    int(Lmax), _ptr(lengths), _ptr(idx), _ptr(gate), _ptr(O),
@@ -234,6 +250,26 @@ class Buffers:
     def decode(self, q, K_cache, V_cache, lengths, stream=None):
         gqe_attn_decode(self.shape, q, K_cache, V_cache, K_cache.shape[1], lengths, self.idx, self.gate, self.O,
                         self.workspace, stream)
+
+    def backward(self, Q, K, V, dO, stream=None):
+        """Gradients of the routed attention for output gradient dO (the routing
+        of the last `route`): returns (dQ, dK, dV, dlogits), float32 tensors
+        owned by this object and overwritten by the next call."""
+        sh = self.shape
+        if getattr(self, "_bwd", None) is None:
+            dev = self.idx.device
+            f32 = dict(dtype=torch.float32, device=dev)
+            nbytes = gqe_attn_backward_workspace_bytes(sh)
+            self._bwd = (torch.empty((sh.B, sh.T, sh.h, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.g, sh.d_h), **f32),
+                         torch.empty((sh.B, sh.T, sh.g, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.h), **f32),
+                         torch.zeros(nbytes, dtype=torch.uint8, device=dev))
+        dQ, dK, dV, dl, ws = self._bwd
+        gqe_attn_prefill_backward(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
+                                  self.head_chunk_offsets, dO, dQ, dK, dV, dl, ws, stream)
+        return dQ, dK, dV, dl
+
+    def backward_status(self, stream=None) -> int:
+        return gqe_get_device_status(self._bwd[4], stream)
 
     def status(self, stream=None) -> int:
         return gqe_get_device_status(self.workspace, stream)

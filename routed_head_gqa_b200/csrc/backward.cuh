@@ -1,0 +1,32 @@
+// backward.cuh -- launcher of the routed attention's backward pass.
+#pragma once
+
+#include "common.cuh"
+
+namespace gqe {
+
+struct AttnBwdArgs {
+    const gqe_shape* s;
+    const void* Q;  // [B,T,h,d_h]
+    const void* K;  // [B,T,g,d_h]
+    const void* V;
+    const void* dO;  // gradient of the loss with respect to the output O [B,T,h,d_h]
+    const int32_t* idx;
+    const float* gate;
+    const int32_t* head_offsets;
+    const int32_t* head_pos;
+    const int32_t* head_chunk_offsets;
+    float* dQ;       // [B,T,h,d_h]
+    float* dK;       // [B,T,g,d_h]
+    float* dV;       // [B,T,g,d_h]
+    float* dlogits;  // [B,T,h]
+    void* scratch;   // attn_backward_scratch_bytes(s) bytes, 256-byte aligned
+    void* status;
+    cudaStream_t stream;
+};
+
+// Per-(b,t,j) scratch of the backward: gate, D = dO.O and the row's log2-sum-exp.
+size_t attn_backward_scratch_bytes(const gqe_shape* s);
+cudaError_t launch_attn_backward(const AttnBwdArgs& a);
+
+}  // namespace gqe

@@ -2,6 +2,7 @@
 // host, then kernel launches on the caller's stream.  See include/gqe.h.
 #include <cstring>
 
+#include "backward.cuh"
 #include "common.cuh"
 
 using namespace gqe;
@@ -302,6 +303,49 @@ gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* 
     a.page_shift = shift;
     a.num_pages = num_pages;
     return from_cuda(launch_decode(a));
+}
+
+size_t gqe_attn_backward_workspace_bytes(const gqe_shape* s) {
+    if (check_shape(s) == GQE_ERR_INVALID_ARGUMENT) return 0;
+    return kStatusBytes + attn_backward_scratch_bytes(s);
+}
+
+gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                     const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                     const int32_t* head_pos, const int32_t* head_chunk_offsets, const void* dO,
+                                     float* dQ, float* dK, float* dV, float* dlogits, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!Q || !K || !V || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets || !dO || !dQ || !dK ||
+        !dV || !dlogits)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dK) ||
+        !aligned16(dV))
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (s->d_h != 32 && s->d_h != 64 && s->d_h != 128) return GQE_ERR_UNSUPPORTED;
+    if ((int64_t)s->B * s->h > 65535 || s->B > 65535 || s->g > 65535) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + attn_backward_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    AttnBwdArgs a;
+    a.s = s;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.dO = dO;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dlogits = dlogits;
+    a.scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_attn_backward(a));
 }
 
 gqe_status gqe_get_device_status(void* workspace, void* stream) {

@@ -153,3 +153,18 @@ def decode_parity(w):
     keep = ~excl.reshape(-1)
     err = float(np.abs(got[keep] - want[keep]).max(initial=0.0))
     return err, int(keep.sum()), int(excl.sum())
+
+
+def oracle_tables(w, idx_o, dev="cuda"):
+    """Routing tables of the oracle's selection, for feeding the oracle's
+    routing to a GPU kernel: (idx int32, head_offsets, head_pos,
+    head_chunk_offsets) device tensors, the lists from oracle.compact and the
+    per-32-position chunk starts found by search in each ascending list."""
+    offs, pos = oracle.compact(idx_o, w.h, w.g, w.k)
+    nchunk = (w.T + 31) // 32
+    chunk = np.empty(w.B * w.h * nchunk, np.int32)
+    for bj in range(w.B * w.h):
+        lst = pos[offs[bj]:offs[bj + 1]]
+        chunk[bj * nchunk:(bj + 1) * nchunk] = offs[bj] + np.searchsorted(lst, 32 * np.arange(nchunk), side="left")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    return t(idx_o), t(offs), t(pos), t(chunk)

@@ -679,6 +679,11 @@ def check_backward_invariants(o):
                     want[b, : t + 1, q_] += gate[b, t, q_, s] * dO[b, t, j] / (t + 1)
                     assert abs(dg0[b, t, q_, s] - np.dot(dO[b, t, j], V[b, : t + 1, q_].astype(np.float64).mean(0))) < 1e-12
     assert np.abs(dV0 - want).max() < 1e-12, "dV with K = 0"
+    # a suffix of query rows: the later key rows of dK/dV and the later query rows are exact
+    tq, tk, tv, tg = o.attn_backward(Q, K, V, idx, gate, dO, t_min=6)
+    for name, got, want in (("dK", tk, dK), ("dV", tv, dV), ("dQ", tq, dQ), ("dgate", tg, dgate)):
+        assert np.array_equal(got[:, 6:], want[:, 6:]), f"t_min: {name} rows past t_min"
+    assert np.all(tq[:, :6] == 0.0) and np.all(tg[:, :6] == 0.0), "t_min: query rows before t_min"
     i1 = np.broadcast_to(np.arange(h, dtype=np.int32).reshape(1, 1, h, 1), (B, T, h, 1)).copy()
     g1 = np.ones((B, T, h, 1))
     _, _, _, dg1 = o.attn_backward(Q, np.repeat(K, 3, axis=2), np.repeat(V, 3, axis=2), i1, g1, dO)

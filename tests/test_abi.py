@@ -156,6 +156,26 @@ def test_decode_paged_validation():
     assert call(s2, 16, 64, fake, 4) == 1      # decode: T must be 1
 
 
+def test_attn_backward_validation():
+    import routed_head_gqa_b200 as g
+
+    fake = 0x10000
+    s = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_BF16)
+    need = g.gqe_attn_backward_workspace_bytes(s)
+    assert need == 256 + 3 * 2 * 64 * 8 * 4
+    call = lambda s, dQ, ws_bytes: g._lib.gqe_attn_prefill_backward(
+        ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, dQ, fake, fake, fake, fake,
+        ws_bytes, None)
+    assert call(s, None, need) == 1             # no dQ
+    assert call(s, fake + 8, need) == 1         # misaligned dQ
+    assert call(s, fake, need - 1) == 1         # workspace too small
+    s96 = g.make_shape(2, 64, 128, 8, 2, 96, 2, g.GQE_BF16)
+    assert call(s96, fake, 1 << 30) == 2        # d_h 96 not implemented
+    bad = g.make_shape(2, 64, 128, 8, 3, 128, 2, g.GQE_BF16)
+    assert call(bad, fake, 1 << 30) == 1        # h % g != 0
+    assert g.gqe_attn_backward_workspace_bytes(bad) == 0
+
+
 def test_unsupported_cases_report_unsupported():
     import routed_head_gqa_b200 as g
 
