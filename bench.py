@@ -431,27 +431,39 @@ def time_backward(w, steps, warmup, peaks, peak_kind):
     dO = gqe_synth.make_output_grad(w).to(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    def fn():
+    def attn():
         r.buf.backward(r.d["Q"], r.d["K"], r.d["V"], dO)
 
-    for _ in range(warmup):
-        l2_flush(flush)
-        fn()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    torch.cuda.synchronize()
-    for a, b in ev:
-        l2_flush(flush)
-        a.record()
-        fn()
-        b.record()
-    torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    def router():
+        r.buf.route_backward(r.d["x"], r.d["W_r"], r.buf._bwd[3])
+
+    def timed(fn):
+        for _ in range(warmup):
+            l2_flush(flush)
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            l2_flush(flush)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+    ms = timed(attn)
+    rms = timed(router)
     st = r.buf.backward_status()
     if st != 0:
         raise RuntimeError(f"device status {r.g.gqe_status_string(st)} in the backward")
     flops = 2.5 * metrics.prefill_active_flops(w.B, w.T, w.g, w.k, w.d_h)
     tf = flops / (ms * 1e-3) * 1e-12
     alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 * 1e-12
+    el = 2 if w.dtype == "bf16" else 4
+    BT = w.B * w.T
+    # x read once per 32 heads and dx written (fp32); dlogits read twice; W_r, dW_r, dbias are small
+    r_bytes = float(BT * w.d_model * (el * -(-w.h // 32) + 4) + 2 * BT * w.h * 4 + w.d_model * w.h * (el + 4))
+    r_gbs = r_bytes / (rms * 1e-3) * 1e-9
     del r, flush
     torch.cuda.empty_cache()
     return {"ms": ms, "value": tf, "unit": "TFLOP/s", "flops": flops, "launches": 3,
@@ -460,6 +472,11 @@ def time_backward(w, steps, warmup, peaks, peak_kind):
                          "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz (derived)",
                          "frac_of_bf16_tensor": round(tf / peaks["bf16_tflops"], 4),
                          "kernel": "gqe_attn_prefill_backward (bwd_dq_kernel + bwd_rows_kernel + bwd_dkdv_kernel)"},
+            "router": {"ms": rms, "value": r_gbs, "unit": "GB/s", "bytes": r_bytes, "launches": 4,
+                       "roofline": {"bound": "hbm", "achieved": round(r_gbs, 1), "peak": peaks["hbm_gbs"],
+                                    "unit": "GB/s", "frac": round(r_gbs / peaks["hbm_gbs"], 4),
+                                    "peak_source": f"hbm_gbs ({peak_kind})",
+                                    "kernel": "gqe_route_backward (dx, dW_r partials + reduce, dbias)"}},
             "shape": w.describe()}
 
 

@@ -305,19 +305,40 @@ gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* 
  *   dQ [B,T,h,d_h]       device float32 out (0 in unselected slots)
  *   dK, dV [B,T,g,d_h]   device float32 out
  *   dlogits [B,T,h]      device float32 out
- *   workspace            at least gqe_attn_backward_workspace_bytes(s) bytes,
+ *   workspace            at least gqe_backward_workspace_bytes(s) bytes,
  *                        256-byte aligned; its first 256 bytes are the status word
  * Implemented cases: bf16 or fp32, d_h in {32, 64, 128}, k <= 16, h <= 256,
  * B*h <= 65535; others return GQE_ERR_UNSUPPORTED.  All of Q, K, V, dO, dQ,
  * dK, dV must be 16-byte aligned.  An index outside its group, or a
  * position outside [0, T), is reported in the status word and skipped.
  */
-size_t gqe_attn_backward_workspace_bytes(const gqe_shape* s);
+/* Bytes of device workspace for gqe_attn_prefill_backward and
+ * gqe_route_backward on shape *s (0 for an invalid shape). */
+size_t gqe_backward_workspace_bytes(const gqe_shape* s);
 gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const void* K, const void* V,
                                      const int32_t* idx, const float* gate, const int32_t* head_offsets,
                                      const int32_t* head_pos, const int32_t* head_chunk_offsets, const void* dO,
                                      float* dQ, float* dK, float* dV, float* dlogits, void* workspace,
                                      size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_route_backward -- gradients of the linear router from the logit
+ * gradients (for training; the chain rule through the router of gqe_route,
+ * l = x . W_r + bias, gist.science summary, "Architecture et Routage"):
+ *   dx = dlogits . W_r^T,   dW_r = x^T . dlogits,   dbias = sum over tokens of dlogits
+ *
+ *   x [B*T, d_model], W_r [d_model, h]   device, dtype (as passed to gqe_route)
+ *   dlogits [B*T, h]     device float32 (from gqe_attn_prefill_backward)
+ *   dx [B*T, d_model]    device float32 out
+ *   dW_r [d_model, h]    device float32 out (summed over token ranges in a
+ *                        fixed order: the result is reproducible)
+ *   dbias [h]            device float32 out, or NULL to skip it
+ *   workspace            at least gqe_backward_workspace_bytes(s) bytes
+ * Implemented cases: bf16 or fp32, B*T <= 1048560; others return
+ * GQE_ERR_UNSUPPORTED.
+ */
+gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r, const float* dlogits, float* dx,
+                              float* dW_r, float* dbias, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, read the workspace status word, reset it to zero and
  * return it (GQE_OK when no kernel reported a failure). */

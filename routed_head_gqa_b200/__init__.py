@@ -28,7 +28,8 @@ GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
-            "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_backward_workspace_bytes", "gqe_attn_prefill_backward",
+            "gqe_group_slots", "gqe_routed_qproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
+            "gqe_route_backward",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -71,15 +72,16 @@ def _load():
     lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
     lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode_paged.argtypes = [S, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
-    lib.gqe_attn_backward_workspace_bytes.argtypes = [S]
-    lib.gqe_attn_backward_workspace_bytes.restype = _SZ
+    lib.gqe_backward_workspace_bytes.argtypes = [S]
+    lib.gqe_backward_workspace_bytes.restype = _SZ
     lib.gqe_attn_prefill_backward.argtypes = [S] + [_P] * 14 + [_SZ, _P]
+    lib.gqe_route_backward.argtypes = [S] + [_P] * 7 + [_SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
-              "gqe_attn_prefill_backward", "gqe_get_device_status"):
+              "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -167,8 +169,8 @@ def gqe_attn_prefill(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chu
                                                      _nbytes(workspace), _stream(stream)))
 
 
-def gqe_attn_backward_workspace_bytes(shape) -> int:
-    return int(_lib.gqe_attn_backward_workspace_bytes(ctypes.byref(shape)))
+def gqe_backward_workspace_bytes(shape) -> int:
+    return int(_lib.gqe_backward_workspace_bytes(ctypes.byref(shape)))
 
 
 def gqe_attn_prefill_backward(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, dO, dQ, dK, dV,
@@ -178,6 +180,12 @@ def gqe_attn_prefill_backward(shape, Q, K, V, idx, gate, head_offsets, head_pos,
                                           _ptr(head_offsets), _ptr(head_pos), _ptr(head_chunk_offsets),
                                           _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dlogits), _ptr(workspace),
                                           _nbytes(workspace), _stream(stream)))
+
+
+def gqe_route_backward(shape, x, W_r, dlogits, dx, dW_r, dbias, workspace, stream=None) -> None:
+    _check("gqe_route_backward",
+           _lib.gqe_route_backward(ctypes.byref(shape), _ptr(x), _ptr(W_r), _ptr(dlogits), _ptr(dx), _ptr(dW_r),
+                                   _ptr(dbias), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def gqe_attn_decode(shape, q, K_cache, V_cache, Lmax, lengths, idx, gate, O, workspace, stream=None) -> None:
@@ -259,7 +267,7 @@ class Buffers:
         if getattr(self, "_bwd", None) is None:
             dev = self.idx.device
             f32 = dict(dtype=torch.float32, device=dev)
-            nbytes = gqe_attn_backward_workspace_bytes(sh)
+            nbytes = gqe_backward_workspace_bytes(sh)
             self._bwd = (torch.empty((sh.B, sh.T, sh.h, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.g, sh.d_h), **f32),
                          torch.empty((sh.B, sh.T, sh.g, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.h), **f32),
                          torch.zeros(nbytes, dtype=torch.uint8, device=dev))
@@ -267,6 +275,21 @@ class Buffers:
         gqe_attn_prefill_backward(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
                                   self.head_chunk_offsets, dO, dQ, dK, dV, dl, ws, stream)
         return dQ, dK, dV, dl
+
+    def route_backward(self, x, W_r, dlogits, stream=None):
+        """Router gradients (dx, dW_r, dbias) from the logit gradients, float32
+        tensors owned by this object (uses the backward workspace)."""
+        sh = self.shape
+        if getattr(self, "_rbwd", None) is None:
+            dev = self.idx.device
+            f32 = dict(dtype=torch.float32, device=dev)
+            self._rbwd = (torch.empty((sh.B, sh.T, sh.d_model), **f32), torch.empty((sh.d_model, sh.h), **f32),
+                          torch.empty((sh.h,), **f32))
+        if getattr(self, "_bwd", None) is None:
+            raise RuntimeError("route_backward follows backward (it reuses its workspace)")
+        dx, dW, db = self._rbwd
+        gqe_route_backward(sh, x, W_r, dlogits, dx, dW, db, self._bwd[4], stream)
+        return dx, dW, db
 
     def backward_status(self, stream=None) -> int:
         return gqe_get_device_status(self._bwd[4], stream)

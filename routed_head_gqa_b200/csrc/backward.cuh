@@ -29,4 +29,20 @@ struct AttnBwdArgs {
 size_t attn_backward_scratch_bytes(const gqe_shape* s);
 cudaError_t launch_attn_backward(const AttnBwdArgs& a);
 
+struct RouteBwdArgs {
+    const gqe_shape* s;
+    const void* x;          // [B*T, d_model]
+    const void* W_r;        // [d_model, h]
+    const float* dlogits;   // [B*T, h]
+    float* dx;              // [B*T, d_model]
+    float* dW;              // [d_model, h]
+    float* dbias;           // [h] or null
+    void* scratch;          // route_backward_scratch_bytes(s) bytes
+    cudaStream_t stream;
+};
+
+// Partial sums of dW_r over token ranges (reduced in a fixed order).
+size_t route_backward_scratch_bytes(const gqe_shape* s);
+cudaError_t launch_route_backward(const RouteBwdArgs& a);
+
 }  // namespace gqe

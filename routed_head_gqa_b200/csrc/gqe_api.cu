@@ -305,9 +305,31 @@ gqe_status gqe_attn_decode_paged(const gqe_shape* s, const void* q, const void* 
     return from_cuda(launch_decode(a));
 }
 
-size_t gqe_attn_backward_workspace_bytes(const gqe_shape* s) {
+size_t gqe_backward_workspace_bytes(const gqe_shape* s) {
     if (check_shape(s) == GQE_ERR_INVALID_ARGUMENT) return 0;
-    return kStatusBytes + attn_backward_scratch_bytes(s);
+    const size_t a = attn_backward_scratch_bytes(s), r = route_backward_scratch_bytes(s);
+    return kStatusBytes + (a > r ? a : r);
+}
+
+gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r, const float* dlogits, float* dx,
+                              float* dW_r, float* dbias, void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!x || !W_r || !dlogits || !dx || !dW_r) return GQE_ERR_INVALID_ARGUMENT;
+    if ((int64_t)s->B * s->T > (int64_t)65535 * 16) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + route_backward_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    RouteBwdArgs a;
+    a.s = s;
+    a.x = x;
+    a.W_r = W_r;
+    a.dlogits = dlogits;
+    a.dx = dx;
+    a.dW = dW_r;
+    a.dbias = dbias;
+    a.scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_route_backward(a));
 }
 
 gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const void* K, const void* V,

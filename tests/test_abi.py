@@ -161,19 +161,27 @@ def test_attn_backward_validation():
 
     fake = 0x10000
     s = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_BF16)
-    need = g.gqe_attn_backward_workspace_bytes(s)
-    assert need == 256 + 3 * 2 * 64 * 8 * 4
+    need = g.gqe_backward_workspace_bytes(s)
+    # status word + the larger of the attention scratch (gate, D, lse per (b,t,j))
+    # and the router's dW_r partials (64 token ranges here)
+    assert need == 256 + max(3 * 2 * 64 * 8 * 4, 64 * 128 * 8 * 4)
     call = lambda s, dQ, ws_bytes: g._lib.gqe_attn_prefill_backward(
         ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, dQ, fake, fake, fake, fake,
         ws_bytes, None)
     assert call(s, None, need) == 1             # no dQ
     assert call(s, fake + 8, need) == 1         # misaligned dQ
-    assert call(s, fake, need - 1) == 1         # workspace too small
+    assert call(s, fake, 256 + 3 * 2 * 64 * 8 * 4 - 1) == 1  # workspace too small for the attention scratch
     s96 = g.make_shape(2, 64, 128, 8, 2, 96, 2, g.GQE_BF16)
     assert call(s96, fake, 1 << 30) == 2        # d_h 96 not implemented
     bad = g.make_shape(2, 64, 128, 8, 3, 128, 2, g.GQE_BF16)
     assert call(bad, fake, 1 << 30) == 1        # h % g != 0
-    assert g.gqe_attn_backward_workspace_bytes(bad) == 0
+    assert g.gqe_backward_workspace_bytes(bad) == 0
+    rcall = lambda s, dx, ws_bytes: g._lib.gqe_route_backward(ctypes.byref(s), fake, fake, fake, dx, fake, None,
+                                                              fake, ws_bytes, None)
+    assert rcall(s, None, need) == 1            # no dx
+    assert rcall(s, fake, 255) == 1             # workspace too small
+    huge = g.make_shape(1 << 11, 1 << 10, 128, 8, 2, 128, 2, g.GQE_BF16)
+    assert rcall(huge, fake, 1 << 40) == 2      # more tokens than the dx grid covers
 
 
 def test_unsupported_cases_report_unsupported():

@@ -1,5 +1,5 @@
-"""GPU parity of the routed attention backward (gqe_attn_prefill_backward)
-against the oracle's backward on the same seeded inputs.
+"""GPU parity of the backward pass (gqe_attn_prefill_backward, then
+gqe_route_backward) against the oracle's backward on the same seeded inputs.
 
 The small cases feed the oracle's routing (selection, gates and the position
 lists built from it) to the GPU kernels, so both sides differentiate the same
@@ -54,7 +54,7 @@ def gpu_backward_oracle_routing(w, inp, dO, idx_o, gate_o, idx_override=None):
     gate_d = torch.from_numpy(gate_o.astype(np.float32)).cuda()
     shape = g.make_shape(w.B, w.T, w.d_model, w.h, w.g, w.d_h, w.k, w.torch_dtype)
     dQ, dK, dV, dl = _outputs(w)
-    ws = torch.zeros(g.gqe_attn_backward_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(g.gqe_backward_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
     g.gqe_attn_prefill_backward(shape, U.to_dev(inp["Q"]), U.to_dev(inp["K"]), U.to_dev(inp["V"]), idx_d, gate_d,
                                 offs, pos, chunk, U.to_dev(dO), dQ, dK, dV, dl, ws)
     torch.cuda.synchronize()
@@ -71,12 +71,47 @@ def test_backward_small(w):
     assert st == 0, f"device status {st}"
     want_q, want_k, want_v, dgate = oracle.attn_backward(inp["Q"], inp["K"], inp["V"], idx_o, gate_o,
                                                          dO.float().numpy())
-    want_l = oracle.route_backward(inp["x"], inp["W_r"], idx_o, gate_o, dgate)[0]
+    want_l, want_x, want_w, want_b = oracle.route_backward(inp["x"], inp["W_r"], idx_o, gate_o, dgate)
     tol = U.TOL[w.dtype]
     for name, got, want in (("dQ", dQ, want_q), ("dK", dK, want_k), ("dV", dV, want_v), ("dlogits", dl, want_l)):
         assert np.isfinite(got).all(), f"{w.name}: {name} has unwritten or non-finite elements"
         err = float(np.abs(got - want).max())
         assert err <= tol, f"{w.name}: {name} max abs error {err} (scale {np.abs(want).max():.3g})"
+    # on through the router, from the GPU's own logit gradients
+    dx, dW, db = gpu_route_backward(w, inp, torch.from_numpy(dl.astype(np.float32)))
+    for name, got, want in (("dx", dx, want_x), ("dW_r", dW, want_w), ("dbias", db, want_b)):
+        err = float(np.abs(got - want).max())
+        assert err <= tol, f"{w.name}: {name} max abs error {err} (scale {np.abs(want).max():.3g})"
+
+
+def gpu_route_backward(w, inp, dlogits):
+    g = U.gqe()
+    shape = g.make_shape(w.B, w.T, w.d_model, w.h, w.g, w.d_h, w.k, w.torch_dtype)
+    nan = float("nan")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dx = torch.full((w.B, w.T, w.d_model), nan, **f32)
+    dW = torch.full((w.d_model, w.h), nan, **f32)
+    db = torch.full((w.h,), nan, **f32)
+    ws = torch.zeros(g.gqe_backward_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    g.gqe_route_backward(shape, U.to_dev(inp["x"]), U.to_dev(inp["W_r"]), dlogits.cuda(), dx, dW, db, ws)
+    torch.cuda.synchronize()
+    return [t.cpu().numpy().astype(np.float64) for t in (dx, dW, db)]
+
+
+@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill"])
+def test_route_backward_full_size(name):
+    """Router gradients at full size from a seeded gate gradient: the oracle's
+    logit gradients go in, dx, dW_r and dbias are compared in full."""
+    w = W[name]
+    inp = gqe_synth.make_inputs(w)
+    idx_o, gate_o, _, _ = U.oracle_route(w, inp)
+    dgate = np.random.default_rng(w.seed + 7).standard_normal(idx_o.shape)
+    want_l, want_x, want_w, want_b = oracle.route_backward(inp["x"], inp["W_r"], idx_o, gate_o, dgate)
+    dx, dW, db = gpu_route_backward(w, inp, torch.from_numpy(want_l.astype(np.float32)))
+    for nm, got, want in (("dx", dx, want_x), ("dW_r", dW, want_w), ("dbias", db, want_b)):
+        assert np.isfinite(got).all(), f"{nm} has unwritten or non-finite elements"
+        err = float(np.abs(got - want).max())
+        assert err <= U.TOL["bf16"], f"{name}: {nm} max abs error {err} (scale {np.abs(want).max():.3g})"
 
 
 def test_backward_reports_foreign_index():
