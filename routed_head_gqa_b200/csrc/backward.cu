@@ -12,15 +12,15 @@
 //   ds_s   = p_s * (gm * dO . v_s - D)
 //   dQ     = sum_s ds_s k_s / sqrt(d_h)
 //   dK_s  += ds_s q / sqrt(d_h),   dV_s += p_s * gm * dO
-// o is recomputed in fp32 rather than read back from the forward's output, so
-// D carries no rounding of O to the input dtype.
+// D is summed in fp32 from p_s and gm dO . v_s rather than read back from the
+// forward's output, so it carries no rounding of O to the input dtype.
 //
 // Three launches, all on CUDA cores in fp32 (a first, correct path: the
 // contractions are not yet on the tensor cores):
 //  1. bwd_dq_kernel, one block per 32 consecutive entries of a (b, j) list:
-//     a first sweep over the visible keys gives each row's log-sum-exp and o,
-//     hence D; a second accumulates dQ.  The gate, D and the log-sum-exp of
-//     every routed row go to scratch.
+//     a first sweep over the visible keys gives each row's log-sum-exp; a
+//     second accumulates D, sum_s p_s dp_s k_s and sum_s p_s k_s, hence dQ.
+//     The gate, D and the log-sum-exp of every routed row go to scratch.
 //  2. bwd_rows_kernel, one warp per (b, t, group): the group's logit
 //     gradients, and zero dQ rows for the unselected heads.
 //  3. bwd_dkdv_kernel, one block per (b, group, 32-key tile): every routed row
@@ -63,6 +63,19 @@ __device__ __forceinline__ void axpy4(float a, const float4& x, float4& y) {
     y.y = fmaf(a, x.y, y.y);
     y.z = fmaf(a, x.z, y.z);
     y.w = fmaf(a, x.w, y.w);
+}
+
+// Sum of NM independent partial dot products (short dependency chains).
+template <int NM>
+__device__ __forceinline__ float dot_rows(const float4 (&a)[NM], const float4 (&b)[NM]) {
+    float p[NM];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) p[m] = dot4(a[m], b[m], 0.f);
+#pragma unroll
+    for (int w = 1; w < NM; w *= 2)
+#pragma unroll
+        for (int m = 0; m + w < NM; m += 2 * w) p[m] += p[m + w];
+    return p[0];
 }
 
 // Sum over the 8 lanes of a row.
@@ -127,56 +140,40 @@ bwd_dq_kernel(int T_, int h, int g, int k, float scale, float scale_log2, const 
             *reinterpret_cast<float4*>(&dst[key][c]) = v;
         }
     };
-    // sweep 1: the row's log2-sum-exp over keys s <= t_r and its output o (in acc)
+    // sweep 1: the row's log2-sum-exp over keys s <= t_r
     float mx = -INFINITY, l = 0.f;
     for (int kt = 0; kt <= t_max; kt += kRows) {
         __syncthreads();
         load_tile(Ks, K, kt);
-        load_tile(Vs, V, kt);
         __syncthreads();
         float sv[kRows];
         float tmx = -INFINITY;
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
-            float part = 0.f;
+            float4 kk[NM];
 #pragma unroll
-            for (int m = 0; m < NM; ++m)
-                part = dot4(qv[m], *reinterpret_cast<const float4*>(&Ks[i][32 * m + 4 * seg]), part);
-            part = seg_sum(part);
+            for (int m = 0; m < NM; ++m) kk[m] = *reinterpret_cast<const float4*>(&Ks[i][32 * m + 4 * seg]);
+            const float part = seg_sum(dot_rows<NM>(qv, kk));
             sv[i] = (kt + i <= t_r) ? part * scale_log2 : -INFINITY;
             tmx = fmaxf(tmx, sv[i]);
         }
         const float mnew = fmaxf(mx, tmx);
         if (mnew != -INFINITY) {
-            const float corr = exp2f(mx - mnew);
-            l *= corr;
+            float sum = 0.f;
 #pragma unroll
-            for (int m = 0; m < NM; ++m)
-                acc[m] = make_float4(acc[m].x * corr, acc[m].y * corr, acc[m].z * corr, acc[m].w * corr);
-#pragma unroll
-            for (int i = 0; i < kRows; ++i) {
-                const float p = exp2f(sv[i] - mnew);
-                l += p;
-#pragma unroll
-                for (int m = 0; m < NM; ++m)
-                    axpy4(p, *reinterpret_cast<const float4*>(&Vs[i][32 * m + 4 * seg]), acc[m]);
-            }
+            for (int i = 0; i < kRows; ++i) sum += exp2f(sv[i] - mnew);
+            l = l * exp2f(mx - mnew) + sum;
             mx = mnew;
         }
     }
     const float lse2 = l > 0.f ? mx + log2f(l) : 0.f;
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    float Dr = 0.f;
+    // sweep 2: with dp_s = gm dO . v_s, D = sum_s p_s dp_s and
+    // dQ = scale * sum_s p_s (dp_s - D) k_s = scale * (sum_s p_s dp_s k_s - D sum_s p_s k_s),
+    // so D is found in the same sweep and o is never formed.
+    float4 ck[NM];  // sum_s p_s k_s; acc holds sum_s p_s dp_s k_s
 #pragma unroll
-    for (int m = 0; m < NM; ++m) {
-        Dr = fmaf(dov[m].x, acc[m].x * inv_l, Dr);
-        Dr = fmaf(dov[m].y, acc[m].y * inv_l, Dr);
-        Dr = fmaf(dov[m].z, acc[m].z * inv_l, Dr);
-        Dr = fmaf(dov[m].w, acc[m].w * inv_l, Dr);
-        acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);  // from here on: dQ
-    }
-    Dr = seg_sum(Dr);
-    // sweep 2: dQ
+    for (int m = 0; m < NM; ++m) ck[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Dr = 0.f;
     for (int kt = 0; kt <= t_max; kt += kRows) {
         __syncthreads();
         load_tile(Ks, K, kt);
@@ -184,21 +181,30 @@ bwd_dq_kernel(int T_, int h, int g, int k, float scale, float scale_log2, const 
         __syncthreads();
 #pragma unroll 4
         for (int i = 0; i < kRows; ++i) {
-            float4 kk[NM];
-            float pqk = 0.f, pdv = 0.f;
+            float4 kk[NM], vk[NM];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
                 kk[m] = *reinterpret_cast<const float4*>(&Ks[i][32 * m + 4 * seg]);
-                pqk = dot4(qv[m], kk[m], pqk);
-                pdv = dot4(dov[m], *reinterpret_cast<const float4*>(&Vs[i][32 * m + 4 * seg]), pdv);
+                vk[m] = *reinterpret_cast<const float4*>(&Vs[i][32 * m + 4 * seg]);
             }
-            pqk = seg_sum(pqk);
-            pdv = seg_sum(pdv);
+            const float pqk = seg_sum(dot_rows<NM>(qv, kk));
+            const float pdv = seg_sum(dot_rows<NM>(dov, vk));
             const float p = (kt + i <= t_r) ? exp2f(pqk * scale_log2 - lse2) : 0.f;
-            const float ds = p * (pdv - Dr);
+            const float pd = p * pdv;
+            Dr += pd;
 #pragma unroll
-            for (int m = 0; m < NM; ++m) axpy4(ds, kk[m], acc[m]);
+            for (int m = 0; m < NM; ++m) {
+                axpy4(pd, kk[m], acc[m]);
+                axpy4(p, kk[m], ck[m]);
+            }
         }
+    }
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+        acc[m].x = fmaf(-Dr, ck[m].x, acc[m].x);
+        acc[m].y = fmaf(-Dr, ck[m].y, acc[m].y);
+        acc[m].z = fmaf(-Dr, ck[m].z, acc[m].z);
+        acc[m].w = fmaf(-Dr, ck[m].w, acc[m].w);
     }
     if (t_r < 0) return;
 #pragma unroll
@@ -268,7 +274,7 @@ bwd_rows_kernel(int64_t BT, int h, int g, int k, const int32_t* __restrict__ idx
 // 3. dK, dV per (b, group, 32-key tile).
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 bwd_dkdv_kernel(int T_, int h, int g, int nchunk, float scale, float scale_log2, const T* __restrict__ Q,
                 const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ dO,
                 const int32_t* __restrict__ head_offsets, const int32_t* __restrict__ head_pos,
@@ -335,16 +341,13 @@ bwd_dkdv_kernel(int T_, int h, int g, int nchunk, float scale, float scale_log2,
 #pragma unroll 4
             for (int r = 0; r < n; ++r) {
                 float4 qr[NM], dr[NM];
-                float pqk = 0.f, pdv = 0.f;
 #pragma unroll
                 for (int m = 0; m < NM; ++m) {
                     qr[m] = *reinterpret_cast<const float4*>(&Qs[r][32 * m + 4 * seg]);
                     dr[m] = *reinterpret_cast<const float4*>(&dOs[r][32 * m + 4 * seg]);
-                    pqk = dot4(qr[m], kv[m], pqk);
-                    pdv = dot4(dr[m], vv[m], pdv);
                 }
-                pqk = seg_sum(pqk);
-                pdv = seg_sum(pdv);
+                const float pqk = seg_sum(dot_rows<NM>(qr, kv));
+                const float pdv = seg_sum(dot_rows<NM>(dr, vv));
                 const int t = row_t[r];
                 const float p = (key_ok && s <= t) ? exp2f(pqk * scale_log2 - row_lse[r]) : 0.f;
                 const float ds = p * (pdv - row_d[r]);
