@@ -329,12 +329,12 @@ gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const vo
  *
  *   x [B*T, d_model], W_r [d_model, h]   device, dtype (as passed to gqe_route)
  *   dlogits [B*T, h]     device float32 (from gqe_attn_prefill_backward)
- *   dx [B*T, d_model]    device float32 out
+ *   dx [B*T, d_model]    device float32 out, 16-byte aligned
  *   dW_r [d_model, h]    device float32 out (summed over token ranges in a
  *                        fixed order: the result is reproducible)
  *   dbias [h]            device float32 out, or NULL to skip it
  *   workspace            at least gqe_backward_workspace_bytes(s) bytes
- * Implemented cases: bf16 or fp32, B*T <= 1048560; others return
+ * Implemented cases: bf16 or fp32, B*T <= 4194240; others return
  * GQE_ERR_UNSUPPORTED.
  */
 gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r, const float* dlogits, float* dx,

@@ -316,7 +316,8 @@ gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r
     gqe_status st = check_shape(s);
     if (st != GQE_OK) return st;
     if (!x || !W_r || !dlogits || !dx || !dW_r) return GQE_ERR_INVALID_ARGUMENT;
-    if ((int64_t)s->B * s->T > (int64_t)65535 * 16) return GQE_ERR_UNSUPPORTED;
+    if (!aligned16(dx)) return GQE_ERR_INVALID_ARGUMENT;
+    if ((int64_t)s->B * s->T > (int64_t)65535 * 64) return GQE_ERR_UNSUPPORTED;
     st = check_workspace(workspace, workspace_bytes, kStatusBytes + route_backward_scratch_bytes(s));
     if (st != GQE_OK) return st;
     RouteBwdArgs a;

@@ -180,7 +180,8 @@ def test_attn_backward_validation():
                                                               fake, ws_bytes, None)
     assert rcall(s, None, need) == 1            # no dx
     assert rcall(s, fake, 255) == 1             # workspace too small
-    huge = g.make_shape(1 << 11, 1 << 10, 128, 8, 2, 128, 2, g.GQE_BF16)
+    assert rcall(s, fake + 4, need) == 1        # misaligned dx
+    huge = g.make_shape(1 << 13, 1 << 10, 128, 8, 2, 128, 2, g.GQE_BF16)
     assert rcall(huge, fake, 1 << 40) == 2      # more tokens than the dx grid covers
 
 
