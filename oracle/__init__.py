@@ -16,6 +16,9 @@ Sources, per function (the same citations are in ``gqe_oracle.c``):
               kernels consume (bookkeeping of the selection made by ``route``).
   attn_backward, route_backward -- the chain rule through the forward's own
               steps (attention, gating, renormalised gates, linear router).
+  aux_loss -- the same page, "Entrainement et Perte": a load-balancing loss
+              that spreads tokens evenly over each group's experts (read as
+              the fraction-times-probability form; the page gives no formula).
   attn_rows, decode -- IBM "Que es la atencion de consultas agrupadas"
               (scaled dot-product attention, 1/sqrt(d_k)), ml-canon "56 GQA /
               MQA" (KV head expansion), freenetmedia.pl "Grouped-Query
@@ -103,7 +106,8 @@ class Oracle:
         lib.oracle_attn_backward.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P,
                                              i32]
         lib.oracle_route_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, i32]
-        for f in (lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
+        lib.oracle_aux_loss.argtypes = [i64, i32, i32, i32, P, P, P, P]
+        for f in (lib.oracle_aux_loss, lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
                   lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows,
                   lib.oracle_decode_paged, lib.oracle_attn_backward, lib.oracle_route_backward):
             f.restype = ctypes.c_int
@@ -318,6 +322,22 @@ class Oracle:
             raise ValueError(f"oracle_route_backward failed ({rc})")
         return dl.reshape(*lead, h), dx.reshape(*lead, d_model), dW, db
 
+    def aux_loss(self, logits, idx):
+        """Load-balancing auxiliary loss for fp32 router logits [..., h] and the
+        selection idx [..., g, k]: returns (loss, dlogits [..., h] float64)."""
+        la = np.ascontiguousarray(np.asarray(logits, dtype=np.float32))
+        h = la.shape[-1]
+        lead = la.shape[:-1]
+        N = int(np.prod(lead)) if lead else 1
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        g, k = ia.shape[-2], ia.shape[-1]
+        loss = ctypes.c_double()
+        dl = np.empty((N, h), np.float64)
+        rc = self.lib.oracle_aux_loss(N, h, g, k, _ptr(la), _ptr(ia.reshape(N, g, k)), ctypes.byref(loss), _ptr(dl))
+        if rc:
+            raise ValueError(f"oracle_aux_loss failed ({rc})")
+        return loss.value, dl.reshape(*lead, h)
+
     def attn(self, Q, K, V, idx, gate, n_threads=None):
         """Full GQE output O [B, T, h, d_h] (float64)."""
         B, T, h, d_h = tuple(Q.shape)
@@ -397,3 +417,7 @@ def attn_backward(*a, **kw):
 
 def route_backward(*a, **kw):
     return default().route_backward(*a, **kw)
+
+
+def aux_loss(*a, **kw):
+    return default().aux_loss(*a, **kw)

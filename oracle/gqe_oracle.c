@@ -54,6 +54,9 @@
  *  - Backward (training; the pages state no formula for it): the gradients of
  *    the routed attention, of the gates and of the router's logits, x, W_r and
  *    bias, by the chain rule through the steps above in reverse order.
+ *  - Load-balancing auxiliary loss (same page, "Entrainement et Perte": it
+ *    makes the router spread tokens evenly over each group's experts; no
+ *    formula given): the fraction-times-probability form, per group.
  */
 #include <math.h>
 #include <stdint.h>
@@ -678,5 +681,95 @@ int oracle_route_backward(int64_t BT, int d_model, int h, int g, int k, int dtyp
             dbias[j] = acc;
         }
     }
+    return 0;
+}
+
+/*
+ * Load-balancing auxiliary loss.  The GQE page ("Entrainement et Perte") adds
+ * an auxiliary loss that makes the router spread tokens evenly over the experts
+ * of each group, and gives no formula.  Reading: the fraction-times-probability
+ * form of mixture-of-experts routers, taken per group and averaged over groups.
+ * With N tokens, hpg = h/g and p[t,j] the softmax of token t's logits over ALL
+ * heads of j's group (not only the selected ones):
+ *   f_j = #{t : j in S(t)} / (N k)          share of the group's selections
+ *   P_j = sum_t p[t,j] / N                  mean router probability
+ *   L   = (1/g) sum_q hpg sum_{j in q} f_j P_j      (= 1 when both are uniform)
+ * f is a count and passes no gradient, so
+ *   dL/dl[t,j] = hpg/(g N) * p[t,j] * (f_j - sum_{i in q} p[t,i] f_i).
+ *
+ * logits [N, h] float (the router's fp32 logits, bias included); idx [N, g, k].
+ * Out: *loss; dlogits [N, h] (double, may be NULL).
+ */
+int oracle_aux_loss(int64_t N, int h, int g, int k, const float* logits, const int32_t* idx,
+                    double* loss, double* dlogits) {
+    if (N < 1 || h < 1 || g < 1 || h % g != 0) return 1;
+    const int hpg = h / g;
+    if (k < 1 || k > hpg) return 1;
+    double* f = (double*)calloc((size_t)h, sizeof(double));
+    double* P = (double*)calloc((size_t)h, sizeof(double));
+    double* p = (double*)malloc(sizeof(double) * (size_t)hpg);
+    if (!f || !P || !p) {
+        free(f);
+        free(P);
+        free(p);
+        return 2;
+    }
+    for (int64_t t = 0; t < N; ++t)
+        for (int q = 0; q < g; ++q)
+            for (int s = 0; s < k; ++s) {
+                const int j = idx[((size_t)t * g + q) * k + s];
+                if (j < q * hpg || j >= (q + 1) * hpg) {
+                    free(f);
+                    free(P);
+                    free(p);
+                    return 1;
+                }
+                f[j] += 1.0 / ((double)N * k);
+            }
+    /* mean probabilities */
+    for (int64_t t = 0; t < N; ++t)
+        for (int q = 0; q < g; ++q) {
+            double m = -INFINITY, den = 0.0;
+            for (int jj = 0; jj < hpg; ++jj) {
+                const double l = (double)logits[(size_t)t * h + q * hpg + jj];
+                if (l > m) m = l;
+            }
+            for (int jj = 0; jj < hpg; ++jj) {
+                p[jj] = exp((double)logits[(size_t)t * h + q * hpg + jj] - m);
+                den += p[jj];
+            }
+            for (int jj = 0; jj < hpg; ++jj) P[q * hpg + jj] += p[jj] / den / (double)N;
+        }
+    double L = 0.0;
+    for (int q = 0; q < g; ++q) {
+        double s = 0.0;
+        for (int jj = 0; jj < hpg; ++jj) s += f[q * hpg + jj] * P[q * hpg + jj];
+        L += (double)hpg * s / (double)g;
+    }
+    *loss = L;
+    if (dlogits) {
+        const double c = (double)hpg / ((double)g * (double)N);
+        for (int64_t t = 0; t < N; ++t)
+            for (int q = 0; q < g; ++q) {
+                double m = -INFINITY, den = 0.0, pf = 0.0;
+                for (int jj = 0; jj < hpg; ++jj) {
+                    const double l = (double)logits[(size_t)t * h + q * hpg + jj];
+                    if (l > m) m = l;
+                }
+                for (int jj = 0; jj < hpg; ++jj) {
+                    p[jj] = exp((double)logits[(size_t)t * h + q * hpg + jj] - m);
+                    den += p[jj];
+                }
+                for (int jj = 0; jj < hpg; ++jj) {
+                    p[jj] /= den;
+                    pf += p[jj] * f[q * hpg + jj];
+                }
+                for (int jj = 0; jj < hpg; ++jj)
+                    dlogits[(size_t)t * h + q * hpg + jj] = c * p[jj] * (f[q * hpg + jj] - pf);
+            }
+    }
+    free(f);
+    free(P);
+    free(p);
     return 0;
 }

@@ -691,10 +691,51 @@ def check_backward_invariants(o):
     assert np.all(dl1 == 0.0), "one head per group: the logit gradient must be 0"
 
 
+def check_aux_loss(o):
+    """Load-balancing loss: equal logits give exactly 1 whatever the selection;
+    a balanced routing (token t of each group favours head t, k = 1) gives 1
+    and a zero gradient; a collapsed routing (every token on head 0 with
+    probability ~1) gives h/g; the gradient matches central differences of the
+    loss with the selection held fixed, and sums to 0 over each group."""
+    N, h, g, k = 6, 6, 2, 2
+    hpg = h // g
+    idx = np.stack([np.stack([q * hpg + (np.arange(k) + t) % hpg for q in range(g)]) for t in range(N)]).astype(np.int32)
+    L, dl = o.aux_loss(np.zeros((N, h), np.float32), idx)
+    assert abs(L - 1.0) < 1e-15, f"equal logits: {L}"
+    # balanced: N = hpg tokens, token t puts +2 on head t of every group, selects it (k = 1)
+    lb = np.zeros((hpg, h), np.float32)
+    ib = np.zeros((hpg, g, 1), np.int32)
+    for t in range(hpg):
+        for q in range(g):
+            lb[t, q * hpg + t] = 2.0
+            ib[t, q, 0] = q * hpg + t
+    L, dl = o.aux_loss(lb, ib)
+    assert abs(L - 1.0) < 1e-14 and np.abs(dl).max() < 1e-15, f"balanced: {L}, {np.abs(dl).max()}"
+    # collapsed: head 0 of every group at +60, always selected
+    lc = np.zeros((N, h), np.float32)
+    lc[:, ::hpg] = 60.0
+    ic = np.zeros((N, g, 1), np.int32)
+    ic[:, :, 0] = np.arange(g) * hpg
+    L, _ = o.aux_loss(lc, ic)
+    assert abs(L - hpg) < 1e-12, f"collapsed: {L}"
+    # gradient: central differences with the selection fixed, on a skewed
+    # selection (head 0 of each group in every token's pair: f = 1/2, 1/4, 1/4)
+    lr = _f32((N, h), 700)
+    isk = np.stack([np.stack([q * hpg + np.array([0, 1 + t % 2]) for q in range(g)]) for t in range(N)])
+    isk = isk.astype(np.int32)
+    L0, dl = o.aux_loss(lr, isk)
+    assert np.abs(dl).max() > 1e-3, "the skewed selection must give a gradient"
+    assert np.abs(dl.reshape(N, g, hpg).sum(-1)).max() < 1e-15, "group sum of the gradient"
+    for i in range(lr.size):
+        fd = _central(lambda a: o.aux_loss(a, isk)[0], lr, i, 1e-3)
+        assert abs(fd - dl.flat[i]) < 1e-7, f"aux dlogits[{i}]: fd {fd} vs {dl.flat[i]}"
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
     check_shared_head_closed_forms, check_group_slots, check_qproj, check_decode_paged,
     check_backward_sdpa_autograd, check_backward_finite_differences, check_backward_invariants,
+    check_aux_loss,
 ]

@@ -56,6 +56,9 @@ MUTANTS = [
     ("router_bwd_dw_wrong_head", "acc += load_elem(x, (size_t)bt * d_model + i, dtype) * dlogits[bt * h + j];",
      "acc += load_elem(x, (size_t)bt * d_model + i, dtype) * dlogits[bt * h + (j + 1) % h];"),
     ("router_bwd_dbias_halved", "dbias[j] = acc;", "dbias[j] = 0.5 * acc;"),
+    ("aux_fraction_per_token", "f[j] += 1.0 / ((double)N * k);", "f[j] += 1.0 / (double)N;"),
+    ("aux_no_group_size_factor", "L += (double)hpg * s / (double)g;", "L += s / (double)g;"),
+    ("aux_grad_drops_mean", "c * p[jj] * (f[q * hpg + jj] - pf);", "c * p[jj] * f[q * hpg + jj];"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
