@@ -134,10 +134,26 @@ gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const f
  * needs clearing): calls whose kernels may overlap on the GPU (different
  * streams, or concurrent host threads on one device) race on it and must be
  * serialised by the caller.
+ * Device-side failures (a bounded wait in the router that expired, which
+ * leaves idx, gate and the lists incomplete, or counts the compaction found
+ * inconsistent, whose writes it skips) are recorded in a status word at the
+ * head of the same array, not in a caller workspace: read them with
+ * gqe_route_static_status.
  */
 gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
                             int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
                             int32_t* head_chunk_offsets, void* stream);
+
+/*
+ * gqe_route_static_status -- the device status word of gqe_route_static on
+ * the calling thread's current device (no counterpart in the paper; it goes
+ * with gqe_route_static).  Synchronises `stream`, returns the first error that
+ * any gqe_route_static call recorded since the last read (GQE_OK if none:
+ * GQE_ERR_DEVICE_TIMEOUT for an expired wait, GQE_ERR_INVALID_ARGUMENT for
+ * inconsistent counts) and clears it.  Allocates nothing; GQE_ERR_CUDA if the
+ * copy or the synchronisation fails.
+ */
+gqe_status gqe_route_static_status(void* stream);
 
 /*
  * gqe_attn_prefill -- routed causal attention with the gated scatter.

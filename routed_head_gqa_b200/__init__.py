@@ -27,6 +27,7 @@ GQE_F32 = 0
 GQE_BF16 = 1
 
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
+            "gqe_route_static_status",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
             "gqe_group_slots", "gqe_routed_qproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
             "gqe_route_backward",
@@ -66,6 +67,7 @@ def _load():
     lib.gqe_workspace_init.argtypes = [_P, _SZ, _P]
     lib.gqe_route.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_route_static.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+    lib.gqe_route_static_status.argtypes = [_P]
     lib.gqe_attn_prefill.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_shared_head.argtypes = [S, _P, _P, _P, _I, _P, _P, _SZ, _P]
@@ -79,7 +81,8 @@ def _load():
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
-    for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_attn_prefill", "gqe_attn_decode",
+    for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_route_static_status",
+              "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
               "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status"):
         getattr(lib, f).restype = _I
@@ -159,6 +162,12 @@ def gqe_route_static(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, hea
     _check("gqe_route_static", _lib.gqe_route_static(ctypes.byref(shape), _ptr(x), _ptr(W_r), _ptr(bias),
                                                      _ptr(idx), _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
                                                      _ptr(head_chunk_offsets), _stream(stream)))
+
+
+def gqe_route_static_status(stream=None) -> int:
+    """Device status of gqe_route_static on the current device (synchronises
+    the stream; returns the first recorded error code and clears it)."""
+    return _lib.gqe_route_static_status(_stream(stream))
 
 
 def gqe_attn_prefill(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, O, workspace,

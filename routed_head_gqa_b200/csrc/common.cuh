@@ -106,11 +106,12 @@ cudaError_t launch_router_tc(const RouteArgs& a);  // a1+a2 on tensor cores (bf1
 // the 32-token chunk), so the separate count pass is skipped.
 bool router_tc_fuses_counts(const gqe_shape* s);
 
-// Library-held scratch for gqe_route_static: per-(b, head, chunk) counts,
-// at most kRouteStaticScratchBytes.  Resolves the calling thread's current
-// device's copy of the array (once per device) into *out.
-constexpr size_t kRouteStaticScratchBytes = size_t(4) << 20;  // 4 MiB
-cudaError_t route_static_scratch(int32_t** out);
+// Library-held scratch for gqe_route_static: a kStatusBytes status region
+// (the device status word of these calls), then the per-(b, head, chunk)
+// counts, at most kRouteStaticScratchBytes of them.  Resolves the calling
+// thread's current device's copy of the array (once per device) into *out.
+constexpr size_t kRouteStaticScratchBytes = size_t(4) << 20;  // 4 MiB of counts
+cudaError_t route_static_scratch(uint8_t** out);
 
 struct PrefillArgs {
     const gqe_shape* s;

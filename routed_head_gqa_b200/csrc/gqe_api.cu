@@ -102,7 +102,7 @@ gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, 
     if (!aligned16(x) || !aligned16(W_r)) return GQE_ERR_INVALID_ARGUMENT;
     const size_t need = (size_t)s->B * s->h * gqe_chunk_count(s->T) * sizeof(int32_t);
     if (need > kRouteStaticScratchBytes) return GQE_ERR_SCRATCH_LIMIT;
-    int32_t* scratch = nullptr;
+    uint8_t* scratch = nullptr;
     if (route_static_scratch(&scratch) != cudaSuccess) return GQE_ERR_CUDA;
     RouteArgs a;
     a.s = s;
@@ -114,10 +114,20 @@ gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, 
     a.head_offsets = head_offsets;
     a.head_pos = head_pos;
     a.head_chunk_offsets = head_chunk_offsets;
-    a.counts = scratch;  // every count is written before it is read: nothing to clear
-    a.status = nullptr;  // the route kernels report nothing through the status word
+    // Every count is written before it is read: nothing to clear.  A bounded
+    // wait that expires in the router, or counts the compaction cannot trust,
+    // are recorded in the status word at the head of the array (read and
+    // cleared by gqe_route_static_status).
+    a.counts = reinterpret_cast<int32_t*>(scratch + kStatusBytes);
+    a.status = scratch;
     a.stream = (cudaStream_t)stream;
     return from_cuda(launch_route(a));
+}
+
+gqe_status gqe_route_static_status(void* stream) {
+    uint8_t* scratch = nullptr;
+    if (route_static_scratch(&scratch) != cudaSuccess) return GQE_ERR_CUDA;
+    return gqe_get_device_status(scratch, stream);
 }
 
 gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, const void* V,

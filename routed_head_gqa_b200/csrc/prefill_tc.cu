@@ -26,6 +26,7 @@
 // S into P, the tensor core runs the other tile's P.V and next QK^T.
 // TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512); P_t (bf16
 // pairs) overwrites the first 64 columns of S_t once S_t is in registers.
+#include <atomic>
 #include <climits>
 
 #include "sm100.cuh"
@@ -744,15 +745,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     u.nwin = (s.T + kQT * u.W - 1) / (kQT * u.W);
     u.nchunk = gqe_chunk_count(s.T);
 
-    // The setmaxnreg split needs exactly kRegsLaunch registers per thread at launch.
-    static int regs_checked = 0;
-    if (regs_checked == 0) {
+    // The setmaxnreg split needs exactly kRegsLaunch registers per thread at
+    // launch (a property of the compiled kernel: checked once per process).
+    static std::atomic<int> regs_checked{0};
+    if (regs_checked.load(std::memory_order_acquire) == 0) {
         cudaFuncAttributes fa;
         cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel);
         if (e != cudaSuccess) return e;
-        regs_checked = (fa.numRegs == kRegsLaunch) ? 1 : -1;
+        regs_checked.store((fa.numRegs == kRegsLaunch) ? 1 : -1, std::memory_order_release);
     }
-    if (regs_checked != 1) return cudaErrorNotSupported;
+    if (regs_checked.load(std::memory_order_acquire) != 1) return cudaErrorNotSupported;
 
     CUtensorMap mapK, mapV;
     const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)a.kv_g, (uint64_t)s.T, (uint64_t)s.B};

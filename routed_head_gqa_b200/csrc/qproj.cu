@@ -64,11 +64,18 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 __global__ void __launch_bounds__(128)
 qproj_kernel(const __grid_constant__ CUtensorMap mapXT, const __grid_constant__ CUtensorMap mapW,
              const int32_t* __restrict__ head_offsets, const int32_t* __restrict__ head_pos, int T, int h,
-             int d_model, const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Q,
+             int d_model, int32_t total, const __nv_bfloat16* __restrict__ X, __nv_bfloat16* __restrict__ Q,
              uint32_t* __restrict__ status) {
     const int mb = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
-    const int32_t beg = head_offsets[(int64_t)b * h + j];
-    const int n = head_offsets[(int64_t)b * h + j + 1] - beg;
+    // A list that does not lie inside head_pos ([0, B*T*g*k)) is reported and
+    // read as empty; a position outside [0, T) is reported and skipped below.
+    int32_t beg = head_offsets[(int64_t)b * h + j];
+    int32_t end = head_offsets[(int64_t)b * h + j + 1];
+    if (beg < 0 || end < beg || end > total) {
+        if (mb == 0 && threadIdx.x == 0) report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereQproj, 1);
+        beg = end = 0;
+    }
+    const int n = end - beg;
     if (mb * kTiles * kM >= n) return;  // the whole CTA leaves before any barrier or TMEM use
 
     extern __shared__ uint8_t smem_raw[];
@@ -78,7 +85,16 @@ qproj_kernel(const __grid_constant__ CUtensorMap mapXT, const __grid_constant__ 
 
     for (int r = tid; r < kTiles * kM; r += 128) {
         const int e = mb * kTiles * kM + r;
-        sm.rows[r] = (e < n) ? (int32_t)((int64_t)b * T + head_pos[beg + e]) : -1;
+        int32_t row = -1;
+        if (e < n) {
+            const int32_t t = head_pos[beg + e];
+            if (t >= 0 && t < T) {
+                row = (int32_t)((int64_t)b * T + t);
+            } else {
+                report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereQproj, 2);
+            }
+        }
+        sm.rows[r] = row;
     }
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -269,6 +285,7 @@ cudaError_t launch_qproj(const QprojArgs& a) {
     // every (b, j) list holds at most T positions
     const dim3 grid((unsigned)((s.T + kTiles * kM - 1) / (kTiles * kM)), (unsigned)s.h, (unsigned)s.B);
     qproj_kernel<<<grid, 128, smem, a.stream>>>(mapXT, mapW, a.head_offsets, a.head_pos, s.T, s.h, s.d_model,
+                                                (int32_t)((int64_t)s.B * s.T * s.g * s.k),
                                                 (const __nv_bfloat16*)a.x, (__nv_bfloat16*)a.Q,
                                                 (uint32_t*)a.status);
     return cudaGetLastError();

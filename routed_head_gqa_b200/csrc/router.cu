@@ -17,6 +17,7 @@ namespace {
 constexpr int kRouterThreads = 256;
 constexpr int kRouterTokPerThread = 4;
 constexpr int kRouterKC = 32;  // d_model chunk staged in shared memory
+constexpr uint32_t kWhereScan = 7;  // status "where" id of the compaction scan
 
 // One block: kRouterTokPerThread * tokgroups tokens, all h heads.
 // Thread (tg, j): head j, tokens tg*4 .. tg*4+3 of the block.
@@ -144,7 +145,7 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
                                             int nchunk, const int32_t* __restrict__ counts,
                                             int32_t* __restrict__ head_offsets,
                                             int32_t* __restrict__ head_chunk_offsets,
-                                            int32_t* __restrict__ head_pos) {
+                                            int32_t* __restrict__ head_pos, uint32_t* __restrict__ status) {
     extern __shared__ int32_t sh[];  // [h] head totals -> head bases, [h] prefix within head
     int32_t* total = sh;
     int32_t* before = sh + h;
@@ -155,10 +156,15 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
     const int c = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const int32_t* cnt = counts + (int64_t)b * h * nchunk;
+    // Counts that do not match a complete routing (a router that gave up on a
+    // bounded wait leaves idx and counts unwritten) must not steer a write out
+    // of the batch's T*g*k entries: sums are clamped to that range here and
+    // every scatter index is checked below.
+    const long long per_batch = (long long)T * g * k;
     for (int j = warp; j < h; j += nwarps) {
-        int tot = 0, pre = 0;
+        long long tot = 0, pre = 0;
         for (int cc = lane; cc < nchunk; cc += 32) {
-            const int v = cnt[(int64_t)j * nchunk + cc];
+            const long long v = min(max(cnt[(int64_t)j * nchunk + cc], 0), kChunk);
             tot += v;
             if (cc < c) pre += v;
         }
@@ -168,30 +174,30 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
             pre += __shfl_xor_sync(0xffffffffu, pre, d);
         }
         if (lane == 0) {
-            total[j] = tot;
-            before[j] = pre;
+            total[j] = (int32_t)min(tot, (long long)per_batch);
+            before[j] = (int32_t)min(pre, (long long)per_batch);
         }
     }
     __syncthreads();
     if (warp == 0) {
-        int carry = 0;
+        long long carry = 0;
         for (int j0 = 0; j0 < h; j0 += 32) {
             const int j = j0 + lane;
-            const int v = (j < h) ? total[j] : 0;
-            int incl = v;
+            const long long v = (j < h) ? total[j] : 0;
+            long long incl = v;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                const long long y = __shfl_up_sync(0xffffffffu, incl, d);
                 if (lane >= d) incl += y;
             }
-            if (j < h) total[j] = carry + incl - v;  // exclusive: head j's base within the batch
-            carry += __shfl_sync(0xffffffffu, incl, 31);
+            if (j < h) total[j] = (int32_t)min(carry + incl - v, (long long)per_batch);  // head j's base
+            carry = min(carry + __shfl_sync(0xffffffffu, incl, 31), (long long)per_batch);
         }
     }
     __syncthreads();
-    const int64_t base = (int64_t)b * T * g * k;  // every batch holds exactly T*g*k entries
+    const int64_t base = (int64_t)b * per_batch;  // every batch holds exactly T*g*k entries
     for (int j = threadIdx.x; j < h; j += blockDim.x) {
-        const int32_t off = (int32_t)(base + total[j] + before[j]);
+        const int32_t off = (int32_t)(base + min((long long)total[j] + before[j], per_batch));
         head_chunk_offsets[((int64_t)b * h + j) * nchunk + c] = off;
         if (c == 0) head_offsets[(int64_t)b * h + j] = off;
     }
@@ -208,7 +214,14 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
             bool hit = false;
             for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
             const unsigned ball = __ballot_sync(0xffffffffu, hit);
-            if (hit) head_pos[base + total[j] + before[j] + __popc(ball & below)] = t;
+            if (hit) {
+                const long long e = (long long)total[j] + before[j] + __popc(ball & below);
+                if (e < per_batch) {
+                    head_pos[base + e] = t;
+                } else if (status != nullptr) {  // counts and selections disagree: report, skip
+                    report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereScan, (uint32_t)b);
+                }
+            }
         }
     }
 }
@@ -261,7 +274,7 @@ cudaError_t launch_route(const RouteArgs& a) {
     cfg.numAttrs = 1;
     cudaError_t e2 = cudaLaunchKernelEx(&cfg, compact_scan_scatter_kernel, (const int32_t*)a.idx, s.B, s.T, s.h,
                                         s.g, s.k, nchunk, (const int32_t*)a.counts, a.head_offsets,
-                                        a.head_chunk_offsets, a.head_pos);
+                                        a.head_chunk_offsets, a.head_pos, (uint32_t*)a.status);
     if (e2 != cudaSuccess) return e2;
     return cudaGetLastError();
 }
@@ -270,21 +283,23 @@ cudaError_t launch_route(const RouteArgs& a) {
 
 // ---------------------------------------------------------------------------
 // Scratch owned by the library, for callers that cannot allocate device memory
-// (gqe_route_static).  Every device that loads this library holds one copy of
-// the array until the process exits.  In host code the array's name is only a
+// (gqe_route_static): the status word of those calls, then their per-chunk
+// counts.  Every device that loads this library holds one copy of the array
+// until the process exits; the loader zero-fills it, so the status word starts
+// clear.  In host code the array's name is only a
 // host-side stand-in: the device address of this device's copy comes from
 // cudaGetSymbolAddress, looked up once per device with that device current.
 // ---------------------------------------------------------------------------
 #include <mutex>
 
-static __device__ __align__(256) int32_t g_route_static_scratch[gqe::kRouteStaticScratchBytes / sizeof(int32_t)];
+static __device__ __align__(256) uint8_t g_route_static_scratch[gqe::kStatusBytes + gqe::kRouteStaticScratchBytes];
 
 namespace gqe {
 
-cudaError_t route_static_scratch(int32_t** out) {
+cudaError_t route_static_scratch(uint8_t** out) {
     constexpr int kMaxDevices = 64;
     static std::mutex mu;
-    static int32_t* addr[kMaxDevices] = {};
+    static uint8_t* addr[kMaxDevices] = {};
     int dev = -1;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -294,7 +309,7 @@ cudaError_t route_static_scratch(int32_t** out) {
         void* p = nullptr;
         err = cudaGetSymbolAddress(&p, g_route_static_scratch);
         if (err != cudaSuccess) return err;
-        addr[dev] = static_cast<int32_t*>(p);
+        addr[dev] = static_cast<uint8_t*>(p);
     }
     *out = addr[dev];
     return cudaSuccess;

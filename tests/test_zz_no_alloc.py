@@ -56,6 +56,8 @@ def test_route_static_matches_route_twice():
                                      torch.cuda.current_stream().cuda_stream)
         assert rc == g.GQE_OK, g.gqe_status_string(rc)
         torch.cuda.synchronize()
+        st = g.gqe_route_static_status()  # the array's own status word: no expired wait, no bad counts
+        assert st == g.GQE_OK, g.gqe_status_string(st)
         assert torch.equal(out["idx"], ref.idx), w.name
         assert (out["gate"] - ref.gate).abs().max().item() <= 1e-5, w.name
         assert torch.equal(out["head_offsets"], ref.head_offsets), w.name
