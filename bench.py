@@ -8,7 +8,9 @@ input, with inputs resident in HBM:
                      gqe_attn_prefill (routed causal attention + gated scatter)
   decode workload:   gqe_route on the new tokens + gqe_attn_decode
 Metric: active-head TFLOP/s for prefill (4*d_h*(t+1) per routed row), KV-cache
-GB/s for decode (2*g*d_h*L_b bf16 elements per sequence).  The L2 is flushed
+GB/s for decode (2*g*d_h*L_b bf16 elements per sequence).  The headline is the
+largest prefill config (gqe_prefill: B=8 T=4096 h=32 g=8 k=2); every config's
+attention time and roofline fraction go into the line's "configs" map.  The L2 is flushed
 before every timed step, outside the step's CUDA events: a 256 MB buffer is
 written, then read back, so the step starts with clean, unrelated lines in L2.
 
@@ -37,8 +39,9 @@ sys.path.insert(0, ROOT)
 
 import gqe_synth  # noqa: E402
 
-PRIMARY = "dense_gqa"
-SECONDARY = ["gqe_prefill", "gqe_long", "gqe_decode"]
+PRIMARY = "gqe_prefill"
+# Every config, in order, in the line's compact "configs" map (the primary included).
+CONFIG_ORDER = ["tiny_f32", "dense_gqa", "gqe_prefill", "gqe_long", "gqe_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch of the dominant kernels, from `ncu` captures
@@ -298,7 +301,15 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
 
     kern = "decode_partial_kernel" if w.decode else "prefill_tc_kernel"
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
-    if w.decode:
+    if w.dtype == "f32" and not w.decode:
+        achieved = work / (attn_avg_ms * 1e-3) * 1e-12
+        alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 * 1e-12
+        kern = "prefill_simt_kernel"
+        roof = {"bound": "alu", "achieved": round(achieved, 4), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / alu_peak, 6),
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz (derived)",
+                "kernel": "gqe_attn_prefill (prefill_simt_kernel, fp32 CUDA cores)"}
+    elif w.decode:
         achieved = work / (attn_avg_ms * 1e-3) * 1e-9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -313,7 +324,7 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
                 "kernel": "gqe_attn_prefill (prefill_tc_kernel)"}
     tr = NCU_TRAFFIC.get((kern, w.name))
     roof["traffic"] = None
-    if tr and tr["sha"] == kernel_sha(KERNEL_FILES[kern]):
+    if tr and kern in KERNEL_FILES and tr["sha"] == kernel_sha(KERNEL_FILES[kern]):
         roof["traffic"] = tr["bytes_per_launch"]
         roof["traffic_note"] = tr["note"]
     roof["algorithmic_per_launch"] = work
@@ -634,6 +645,17 @@ def run_reference(w, steps, warmup):
     return value, unit, tot_s, desc
 
 
+def compact_entry(r):
+    """One config's figures for the line's "configs" map."""
+    roof = r["roofline"]
+    e = {"value": round(r["value"], 3), "unit": r["unit"], "attn_ms": round(r["attn_ms"], 5),
+         "route_ms": round(r["route_ms"], 5), "bound": roof["bound"], "achieved": roof["achieved"],
+         "frac": roof["frac"]}
+    if roof.get("traffic") is not None:
+        e["traffic"] = roof["traffic"]
+    return e
+
+
 # ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -642,7 +664,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=PRIMARY, choices=sorted(gqe_synth.WORKLOADS))
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
-    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other configs")
+    ap.add_argument("--extras", action="store_true",
+                    help="also time the calls around the hot path (paged decode, Q projection, shared head, "
+                         "group slots, backward); a summary goes into the line")
+    ap.add_argument("--extras-out", default=None, help="write the extras' full figures to this JSON file")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layer-ops-only", action="store_true",
@@ -699,21 +725,23 @@ def main():
         return
     res = time_workload(w, args.steps, args.warmup, ws, rank, peaks, peak_kind, with_clocks=(rank == 0),
                         with_e2e=True)
-    secondary = {}
+    configs = {}
     if not args.no_secondary and args.workload == PRIMARY:
-        for name in SECONDARY:
-            sw = gqe_synth.WORKLOADS[name]
-            r2 = time_workload(sw, max(5, args.steps // 2), 3, ws, rank, peaks, peak_kind, with_clocks=False,
-                               with_e2e=False)
-            secondary[name] = {"value": r2["value"], "unit": r2["unit"], "ms_per_step": r2["ms_per_step"],
-                               "attn_ms": r2["attn_ms"], "route_ms": r2["route_ms"], "roofline": r2["roofline"],
-                               "shape": sw.describe()}
-            if sw.decode:
-                secondary[name]["paged"] = time_paged_decode(sw, max(5, args.steps // 2), 3, peaks, peak_kind)
-    layer_ops = None
-    if not args.no_secondary and args.workload == PRIMARY:
-        layer_ops = time_layer_ops(w, max(5, args.steps // 2), 3, peaks, peak_kind)
-        layer_ops["backward"] = time_backward(w, 3, 3, peaks, peak_kind)
+        for name in CONFIG_ORDER:
+            if name == w.name:
+                r2 = res
+            else:
+                r2 = time_workload(gqe_synth.WORKLOADS[name], max(5, args.steps // 2), 3, ws, rank, peaks,
+                                   peak_kind, with_clocks=False, with_e2e=False)
+            configs[name] = compact_entry(r2)
+    extras = None
+    if args.extras and args.workload == PRIMARY:
+        extras = {}
+        dw = gqe_synth.WORKLOADS["gqe_decode"]
+        extras["paged_decode"] = time_paged_decode(dw, max(5, args.steps // 2), 3, peaks, peak_kind)
+        lw = gqe_synth.WORKLOADS["dense_gqa"]
+        extras["layer_ops"] = time_layer_ops(lw, max(5, args.steps // 2), 3, peaks, peak_kind)
+        extras["backward"] = time_backward(lw, 3, 3, peaks, peak_kind)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)
@@ -725,16 +753,23 @@ def main():
             "data": "synthetic (seeded, gqe_synth recipe)",
             "config": {"workload": w.name, "shape": w.describe(), "per_gpu_batch": w.B,
                        "global_batch": w.B * ws, "parallelism": f"replicas x{ws} (no exchange step)",
-                       "l2": "flushed before every timed step, outside the step events: 256 MB written, "
-                             "then read back (clean lines, no write-back charged to the step)",
-                       "attn_ms": res["attn_ms"], "route_ms": res["route_ms"]},
+                       "l2": "flushed before every timed step, outside the step events (256 MB written, read back)",
+                       "attn_ms": round(res["attn_ms"], 5), "route_ms": round(res["route_ms"], 5)},
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"],
             "gpu_launches": res["gpu_launches"],
         }
-        if secondary:
-            line["workloads"] = secondary
-        if layer_ops:
-            line["gqe_layer_ops"] = layer_ops
+        if configs:
+            line["configs"] = configs
+        if extras:
+            if args.extras_out:
+                with open(args.extras_out, "w") as f:
+                    json.dump(extras, f)
+            line["extras"] = {"paged_decode_frac": extras["paged_decode"]["roofline"]["frac"],
+                              "qproj_frac": extras["layer_ops"]["routed_qproj"]["roofline"]["frac"],
+                              "shared_head_frac": extras["layer_ops"]["shared_head"]["roofline"]["frac"],
+                              "group_slots_frac": extras["layer_ops"]["group_slots"]["roofline"]["frac"],
+                              "backward_ms": round(extras["backward"]["ms"], 3),
+                              "route_backward_ms": round(extras["backward"]["router"]["ms"], 4)}
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist

@@ -3,8 +3,10 @@
 //   mode 0: A [M][K] K-major (smem, TMA, 128B swizzle) x B [N][K] K-major
 //   mode 1: A K-major x B [K][N] MN-major (the P.V operand layout of V tiles)
 //   mode 2: A written into TMEM by tcgen05.st (packed bf16 pairs) x B MN-major
-// C [M][N] fp32 = sum_k A[m,k] * B(k,n).  Test-only; not part of the product API.
+// C [M][N] fp32 = sum_k A[m,k] * B(k,n).  Also the FMA-pipe 2^x of the prefill
+// softmax, element by element.  Test-only; not part of the product API.
 #include "common.cuh"
+#include "exp2_fma.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
 
@@ -122,7 +124,27 @@ __global__ void wait_timeout_kernel(uint32_t* __restrict__ status) {
     if (threadIdx.x == 0) atomicExch(status, ok ? (uint32_t)GQE_OK : (uint32_t)GQE_ERR_DEVICE_TIMEOUT);
 }
 
+// y[i] = the prefill softmax's FMA-pipe 2^x of x[i] (clamped at -126), pairs
+// of consecutive elements per thread as in the kernel.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+    float y0, y1;
+    up2(exp2_poly2_clamped(x0, x1), y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
+
+extern "C" int gqe_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+    if (!x || !y || n < 0) return GQE_ERR_INVALID_ARGUMENT;
+    if (n == 0) return GQE_OK;
+    const int pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? GQE_OK : GQE_ERR_CUDA;
+}
 
 extern "C" int gqe_selftest_wait_timeout(uint32_t* status, void* stream) {
     if (!status) return GQE_ERR_INVALID_ARGUMENT;

@@ -135,11 +135,85 @@ def compare_rows(w, inp, O_gpu, idx_o, gate_o, excl, rows=None):
     return err, len(rows)
 
 
-def prefill_parity(w, rows=None):
+def sm_count(dev=0):
+    return torch.cuda.get_device_properties(dev).multi_processor_count
+
+
+def prefill_windows(w):
+    """(W, number of 2W-position windows) of the tensor-core prefill's work
+    units: a unit is (b, KV group, window of 2W positions), W = 32*floor(4/k)."""
+    W = 32 * (4 // w.k)
+    return W, -(-w.T // (2 * W))
+
+
+def cta_units(w, sms, cta):
+    """The (b, q, window) units that CTA `cta` of the persistent prefill grid
+    runs, in its order: unit j of CTA c is j*grid + (c, or grid-1-c for odd j),
+    units ordered heaviest window first with (b, q) fastest."""
+    _, nwin = prefill_windows(w)
+    n_units = w.B * w.g * nwin
+    grid = min(n_units, sms)
+    out = []
+    j = 0
+    while True:
+        unit = j * grid + ((grid - 1 - cta) if (j & 1) else cta)
+        if unit >= n_units:
+            break
+        wr, rem = divmod(unit, w.B * w.g)
+        out.append((rem // w.g, rem % w.g, nwin - 1 - wr))
+        j += 1
+    return out
+
+
+def cover_rows(w, idx_o, sms, n_min=4096, seed=4321):
+    """Flattened rows (b*T + t) for a full-size parity check that reaches
+    every path of the persistent prefill: every position of the first, a middle
+    and the last unit run by the first, a middle and the last CTA (first units
+    exercise the pipeline fill, later ones the double-buffered row tables,
+    barrier phases and TMEM reuse across units), every sequence's last window,
+    the three windows with the most skewed head loads, then seeded random rows
+    up to n_min.  Whole windows are compared for every head."""
+    W, nwin = prefill_windows(w)
+    span = 2 * W
+    wins = set()
+    grid = min(w.B * w.g * nwin, sms)
+    for c in sorted({0, grid // 2, grid - 1}):
+        units = cta_units(w, sms, c)
+        for j in sorted({0, len(units) // 2, len(units) - 1}):
+            b, _, win = units[j]
+            wins.add((b, win))
+    wins |= {(b, nwin - 1) for b in range(w.B)}
+    # skew: the largest share of one head among a window's routed rows of one group
+    sel = np.zeros((w.B, w.T, w.h), bool)
+    np.put_along_axis(sel, idx_o.reshape(w.B, w.T, -1).astype(np.int64), True, axis=-1)
+    pad = nwin * span - w.T
+    per = np.pad(sel, ((0, 0), (0, pad), (0, 0))).reshape(w.B, nwin, span, w.h).sum(axis=2)
+    skew = per.max(axis=-1)  # [B, nwin]
+    for flat in np.argsort(-skew.reshape(-1), kind="stable")[:3]:
+        wins.add((int(flat // nwin), int(flat % nwin)))
+    rows = set()
+    for b, win in wins:
+        t0 = win * span
+        rows.update(range(b * w.T + t0, b * w.T + min(t0 + span, w.T)))
+    if len(rows) < n_min:
+        gen = np.random.default_rng(seed)
+        extra = gen.permutation(w.B * w.T)
+        for r in extra:
+            if len(rows) >= n_min:
+                break
+            rows.add(int(r))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def prefill_parity(w, rows=None, cover=False):
+    """Route + prefill on the GPU against the oracle.  rows: flattened rows to
+    compare (all when None); cover=True picks them with cover_rows."""
     inp = gqe_synth.make_inputs(w)
     buf = run_prefill(w, inp)
     excl, idx_o, gate_o = check_routing(w, inp, buf.idx, buf.gate)
     check_compaction(w, buf.idx, buf.head_offsets, buf.head_pos, buf.head_chunk_offsets, excl, idx_o)
+    if cover:
+        rows = cover_rows(w, idx_o, sm_count())
     err, n = compare_rows(w, inp, buf.O, idx_o, gate_o, excl, rows)
     return err, n, int(excl.sum())
 

@@ -47,10 +47,11 @@ def test_shared_head_small(w, kv):
 
 
 def test_shared_head_full_size_sampled():
-    """The dense_gqa shapes in the bench's launch configuration (KV group 5)."""
+    """The dense_gqa shapes in the bench's launch configuration (KV group 5),
+    on 4096 sampled rows (each sequence's last position included)."""
     w, kv = W["dense_gqa"], 5
     inp, Qs, Os = run_shared(w, kv)
-    rows = gqe_synth.sample_rows(w, 48).numpy()
+    rows = gqe_synth.sample_rows(w, 4096).numpy()
     want = oracle.shared_rows(Qs, inp["K"], inp["V"], kv, rows=rows)
     got = Os.float().reshape(w.B * w.T, w.d_h)[torch.from_numpy(rows).cuda()].cpu().numpy()
     err = float(np.abs(got.astype(np.float64) - want).max())
@@ -65,7 +66,7 @@ SLOTS = [
 ]
 
 
-def slots_parity(w, rows=None):
+def slots_parity(w, rows=None, cover=False):
     g = U.gqe()
     inp = gqe_synth.make_inputs(w)
     buf = U.run_prefill(w, inp)
@@ -81,6 +82,8 @@ def slots_parity(w, rows=None):
     wsum = torch.empty((w.B, w.T, w.g, w.d_h), dtype=w.torch_dtype, device="cuda")
     g.gqe_group_slots(shape, buf.O, buf.idx, buf.gate, cat, wsum)
     torch.cuda.synchronize()
+    if cover:
+        rows = U.cover_rows(w, idx_o, U.sm_count())
     if rows is None:
         rows = np.arange(w.B * w.T)
     rows = np.asarray(rows, dtype=np.int64)
@@ -100,7 +103,10 @@ def test_group_slots_small(w):
 
 
 @pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill"])
-def test_group_slots_full_size_sampled(name):
+def test_group_slots_full_size_covered(name):
+    """At least 4096 rows: whole prefill work units of a first, a middle and the
+    last CTA, every sequence's last window, the most skewed windows, random rows."""
     w = W[name]
-    ec, ew, n = slots_parity(w, gqe_synth.sample_rows(w, 48).numpy())
+    ec, ew, n = slots_parity(w, cover=True)
+    assert n >= 4096 - 64, f"{name}: only {n} rows compared"
     assert ec <= U.TOL["bf16"] and ew <= U.TOL["bf16"], f"{name}: cat {ec}, wsum {ew} over {n} rows"

@@ -54,14 +54,34 @@ def test_prefill_small(w):
 
 
 @pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill", "gqe_long"])
-def test_prefill_full_size_sampled(name):
-    """Full-size workloads in the benchmark's launch configuration; the oracle
-    computes a seeded sample of rows (always including each sequence's last
-    position)."""
+def test_prefill_full_size_covered(name):
+    """Full-size workloads in the benchmark's launch configuration.  The oracle
+    computes at least 4096 rows, chosen to reach every path of the persistent
+    kernel: whole work units (every position of each, all heads) that a first,
+    a middle and the last CTA run first, midway and last, every sequence's last
+    window, the most skewed windows, and random rows."""
     w = W[name]
-    rows = gqe_synth.sample_rows(w, 48).numpy()
-    err, n, excl = U.prefill_parity(w, rows)
+    err, n, excl = U.prefill_parity(w, cover=True)
+    assert n >= 4096 - 64, f"{name}: only {n} rows compared"
     assert err <= U.TOL[w.dtype], f"{name}: max abs error {err} over {n} rows ({excl} tokens excluded)"
+
+
+def test_full_size_repeatable():
+    """Routing and prefill at the gqe_prefill size (the bench's launch
+    configuration) run twice on the same inputs give bit-identical tables and
+    outputs."""
+    w = W["gqe_prefill"]
+    inp = gqe_synth.make_inputs(w)
+    a = U.run_prefill(w, inp)
+    first = [t.clone() for t in (a.idx, a.gate, a.head_offsets, a.head_pos, a.head_chunk_offsets, a.O)]
+    a.O.fill_(float("nan"))
+    a.route(U.to_dev(inp["x"]), U.to_dev(inp["W_r"]), U.to_dev(inp["bias"]))
+    a.prefill(U.to_dev(inp["Q"]), U.to_dev(inp["K"]), U.to_dev(inp["V"]))
+    torch.cuda.synchronize()
+    assert a.status() == 0
+    second = (a.idx, a.gate, a.head_offsets, a.head_pos, a.head_chunk_offsets, a.O)
+    for name, x, y in zip(("idx", "gate", "head_offsets", "head_pos", "head_chunk_offsets", "O"), first, second):
+        assert torch.equal(x, y), f"{name} differs between two runs"
 
 
 SMALL_DECODE = [

@@ -26,7 +26,7 @@ SMALL = [
 SENTINEL = -12288.0  # -1.5 * 2^13: exactly representable in bf16
 
 
-def qproj_parity(w, rows=None):
+def qproj_parity(w, rows=None, cover=False):
     g = U.gqe()
     inp = gqe_synth.make_inputs(w)
     W_Q = gqe_synth.make_qproj_weight(w)
@@ -38,6 +38,8 @@ def qproj_parity(w, rows=None):
     torch.cuda.synchronize()
     assert buf.status() == 0
     excl, idx_o, _ = U.check_routing(w, inp, buf.idx, buf.gate)
+    if cover:
+        rows = U.cover_rows(w, idx_o, U.sm_count())
     if rows is None:
         rows = np.arange(w.B * w.T)
     rows = np.asarray(rows, dtype=np.int64)
@@ -62,9 +64,13 @@ def test_qproj_small(w):
     assert untouched, "rows of unselected heads were written"
 
 
-@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill"])
-def test_qproj_full_size_sampled(name):
+@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill", "gqe_long"])
+def test_qproj_full_size_covered(name):
+    """At least 4096 token rows (every routed head of each): whole windows of
+    consecutive positions (first, middle and last prefill units of three CTAs,
+    each sequence's last window, the most skewed windows) plus random rows."""
     w = W[name]
-    err, n, untouched = qproj_parity(w, gqe_synth.sample_rows(w, 32).numpy())
+    err, n, untouched = qproj_parity(w, cover=True)
+    assert n >= 4096 - 64, f"{name}: only {n} rows compared"
     assert err <= U.TOL["bf16"], f"{name}: max abs error {err} over {n} rows"
     assert untouched
