@@ -356,6 +356,44 @@ gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const vo
 gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r, const float* dlogits, float* dx,
                               float* dW_r, float* dbias, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gqe_route_train -- gqe_route that also writes the router's fp32 logits, for
+ * training: the load-balancing loss (gqe_aux_loss) and the router's own
+ * gradient path read them.  Arguments and results are those of gqe_route, plus
+ *   logits [B*T, h]      device float32 out: x . W_r + bias, the values the
+ *                        top-k selected on
+ */
+gqe_status gqe_route_train(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                           int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                           int32_t* head_chunk_offsets, float* logits, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * gqe_aux_loss -- the router's load-balancing auxiliary loss and its gradient
+ * with respect to the logits.  The GQE summary (gist.science, "Entrainement et
+ * Perte") adds such a loss so that the router spreads the tokens evenly over
+ * the experts of each group, without a formula; this library's reading is the
+ * fraction-times-probability form of mixture-of-experts routers, per group,
+ * averaged over groups.  With N = B*T tokens and p[t,j] the softmax of token
+ * t's logits over ALL heads of j's group:
+ *   f_j = #{t : j selected for t} / (N k),  P_j = mean_t p[t,j],
+ *   loss = (1/g) sum_q (h/g) sum_{j in q} f_j P_j       (1 when balanced)
+ *   dlogits[t,j] = (h/g)/(g N) * p[t,j] * (f_j - sum_{i in j's group} p[t,i] f_i)
+ * (f is a count: no gradient flows through it).
+ *
+ *   logits [B*T, h]      device float32 (gqe_route_train)
+ *   idx [B*T, g, k]      device int32 (the selection); a head outside its
+ *                        group is reported in the status word and skipped
+ *   loss [1]             device float32 out
+ *   dlogits [B*T, h]     device float32 out, or NULL for the loss only
+ *   workspace            at least gqe_aux_loss_workspace_bytes(s) bytes
+ * The sums run in a fixed order: the result is reproducible.  h/g <= 64;
+ * larger groups return GQE_ERR_UNSUPPORTED.
+ */
+size_t gqe_aux_loss_workspace_bytes(const gqe_shape* s);
+gqe_status gqe_aux_loss(const gqe_shape* s, const float* logits, const int32_t* idx, float* loss, float* dlogits,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, read the workspace status word, reset it to zero and
  * return it (GQE_OK when no kernel reported a failure). */
 gqe_status gqe_get_device_status(void* workspace, void* stream);

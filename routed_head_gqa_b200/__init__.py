@@ -30,7 +30,7 @@ EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe
             "gqe_route_static_status",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
             "gqe_group_slots", "gqe_routed_qproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
-            "gqe_route_backward",
+            "gqe_route_backward", "gqe_route_train", "gqe_aux_loss_workspace_bytes", "gqe_aux_loss",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -78,13 +78,18 @@ def _load():
     lib.gqe_backward_workspace_bytes.restype = _SZ
     lib.gqe_attn_prefill_backward.argtypes = [S] + [_P] * 14 + [_SZ, _P]
     lib.gqe_route_backward.argtypes = [S] + [_P] * 7 + [_SZ, _P]
+    lib.gqe_route_train.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_aux_loss_workspace_bytes.argtypes = [S]
+    lib.gqe_aux_loss_workspace_bytes.restype = _SZ
+    lib.gqe_aux_loss.argtypes = [S, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_route_static_status",
               "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
-              "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status"):
+              "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status", "gqe_route_train",
+              "gqe_aux_loss"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -228,6 +233,23 @@ def gqe_routed_qproj(shape, x, W_Q, head_offsets, head_pos, Q, workspace, stream
 def gqe_group_slots(shape, O, idx, gate, O_cat, O_wsum, stream=None) -> None:
     _check("gqe_group_slots", _lib.gqe_group_slots(ctypes.byref(shape), _ptr(O), _ptr(idx), _ptr(gate),
                                                    _ptr(O_cat), _ptr(O_wsum), _stream(stream)))
+
+
+def gqe_route_train(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, head_chunk_offsets, logits, workspace,
+                    stream=None) -> None:
+    _check("gqe_route_train", _lib.gqe_route_train(ctypes.byref(shape), _ptr(x), _ptr(W_r), _ptr(bias), _ptr(idx),
+                                                   _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
+                                                   _ptr(head_chunk_offsets), _ptr(logits), _ptr(workspace),
+                                                   _nbytes(workspace), _stream(stream)))
+
+
+def gqe_aux_loss_workspace_bytes(shape) -> int:
+    return int(_lib.gqe_aux_loss_workspace_bytes(ctypes.byref(shape)))
+
+
+def gqe_aux_loss(shape, logits, idx, loss, dlogits, workspace, stream=None) -> None:
+    _check("gqe_aux_loss", _lib.gqe_aux_loss(ctypes.byref(shape), _ptr(logits), _ptr(idx), _ptr(loss),
+                                             _ptr(dlogits), _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def gqe_get_device_status(workspace, stream=None) -> int:

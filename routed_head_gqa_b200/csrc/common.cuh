@@ -98,6 +98,7 @@ struct RouteArgs {
     int32_t* counts;  // workspace: [B*h*nchunk]
     void* status;
     cudaStream_t stream;
+    float* logits = nullptr;  // optional out: fp32 router logits (bias included) [B*T, h]
 };
 cudaError_t launch_route(const RouteArgs& a);
 bool router_tc_supported(const gqe_shape* s);
@@ -166,6 +167,20 @@ struct IdentityTables {
 };
 size_t shared_tables_bytes(int B, int T);
 cudaError_t launch_identity_tables(int B, int T, void* tables, IdentityTables* out, cudaStream_t stream);
+
+// Load-balancing auxiliary loss (aux_loss.cu).
+struct AuxLossArgs {
+    const gqe_shape* s;
+    const float* logits;   // [B*T, h]
+    const int32_t* idx;    // [B*T, g, k]
+    float* loss;           // [1]
+    float* dlogits;        // [B*T, h] or null
+    void* scratch;         // aux_loss_scratch_bytes(s)
+    void* status;
+    cudaStream_t stream;
+};
+size_t aux_loss_scratch_bytes(const gqe_shape* s);
+cudaError_t launch_aux_loss(const AuxLossArgs& a);
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a);

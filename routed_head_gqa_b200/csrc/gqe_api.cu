@@ -92,6 +92,59 @@ gqe_status gqe_route(const gqe_shape* s, const void* x, const void* W_r, const f
     return from_cuda(launch_route(a));
 }
 
+gqe_status gqe_route_train(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
+                           int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
+                           int32_t* head_chunk_offsets, float* logits, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!x || !W_r || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets || !logits)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(W_r)) return GQE_ERR_INVALID_ARGUMENT;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + route_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    RouteArgs a;
+    a.s = s;
+    a.x = x;
+    a.W_r = W_r;
+    a.bias = bias;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes);
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    a.logits = logits;
+    return from_cuda(launch_route(a));
+}
+
+size_t gqe_aux_loss_workspace_bytes(const gqe_shape* s) {
+    if (check_shape(s) == GQE_ERR_INVALID_ARGUMENT) return 0;
+    return kStatusBytes + aux_loss_scratch_bytes(s);
+}
+
+gqe_status gqe_aux_loss(const gqe_shape* s, const float* logits, const int32_t* idx, float* loss, float* dlogits,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!logits || !idx || !loss) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->h / s->g > 64) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + aux_loss_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    AuxLossArgs a;
+    a.s = s;
+    a.logits = logits;
+    a.idx = idx;
+    a.loss = loss;
+    a.dlogits = dlogits;
+    a.scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_aux_loss(a));
+}
+
 gqe_status gqe_route_static(const gqe_shape* s, const void* x, const void* W_r, const float* bias,
                             int32_t* idx, float* gate, int32_t* head_offsets, int32_t* head_pos,
                             int32_t* head_chunk_offsets, void* stream) {

@@ -25,7 +25,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRouterThreads)
 router_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ bias,
               int64_t BT, int d_model, int h, int g, int k, int32_t* __restrict__ idx,
-              float* __restrict__ gate) {
+              float* __restrict__ gate, float* __restrict__ logits) {
     extern __shared__ float smem[];
     const int tokgroups = blockDim.x / h;
     const int tok_per_block = tokgroups * kRouterTokPerThread;
@@ -70,8 +70,11 @@ router_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __r
     if (active) {
         const float bj = bias ? bias[j] : 0.f;
 #pragma unroll
-        for (int r = 0; r < kRouterTokPerThread; ++r)
+        for (int r = 0; r < kRouterTokPerThread; ++r) {
+            const int64_t tok = tok0 + tg * kRouterTokPerThread + r;
             lg[(tg * kRouterTokPerThread + r) * h + j] = acc[r] + bj;
+            if (logits != nullptr && tok < BT) logits[tok * h + j] = acc[r] + bj;
+        }
     }
     __syncthreads();
 
@@ -244,12 +247,12 @@ cudaError_t launch_route(const RouteArgs& a) {
         auto kern = router_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<blocks, threads, smem, a.stream>>>((const __nv_bfloat16*)a.x, (const __nv_bfloat16*)a.W_r,
-                                                  a.bias, BT, s.d_model, s.h, s.g, s.k, a.idx, a.gate);
+                                                  a.bias, BT, s.d_model, s.h, s.g, s.k, a.idx, a.gate, a.logits);
     } else {
         auto kern = router_kernel<float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<blocks, threads, smem, a.stream>>>((const float*)a.x, (const float*)a.W_r, a.bias, BT,
-                                                  s.d_model, s.h, s.g, s.k, a.idx, a.gate);
+                                                  s.d_model, s.h, s.g, s.k, a.idx, a.gate, a.logits);
     }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

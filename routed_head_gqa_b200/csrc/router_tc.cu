@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(128)
 router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
                  const float* __restrict__ bias, int64_t BT, int d_model, int h, int g, int k, int T,
                  int nchunk, int32_t* __restrict__ idx, float* __restrict__ gate, int32_t* __restrict__ counts,
-                 uint32_t* __restrict__ status) {
+                 uint32_t* __restrict__ status, float* __restrict__ logits) {
     extern __shared__ uint8_t smem_raw[];
     using Smem = RouterSmem<NB>;
     constexpr int S = Smem::kStages;
@@ -206,6 +206,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         __syncthreads();
     }
     const bool failed = sm.failed != 0;  // final: every writer is before the barrier above
+    if (!failed && logits != nullptr) {
+        // fp32 logits of this CTA's rows (bias included), heads fastest: coalesced
+        for (int e = tid; e < kRows * h; e += 128) {
+            const int rloc = e / h, j = e % h;
+            const int row = (int)rank * kRows + rloc;
+            const int64_t tok = tok0 + row;
+            if (tok < BT) logits[tok * h + j] = lg_base[row * ld + j] + (bias ? bias[j] : 0.f);
+        }
+    }
     if (!failed) {
         // Top-k over (row, group) items, rows fastest: the 32 lanes of a warp
         // take 32 consecutive tokens of one group, which is also one chunk for
@@ -329,7 +338,7 @@ cudaError_t launch_nb(const RouteArgs& a, bool fused_counts) {
     cfg.numAttrs = (KS > 1) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, mapX, mapW, a.bias, BT, s.d_model, s.h, s.g, s.k, s.T,
                               gqe_chunk_count(s.T), a.idx, a.gate, fused_counts ? a.counts : (int32_t*)nullptr,
-                              (uint32_t*)a.status);
+                              (uint32_t*)a.status, a.logits);
 }
 
 template <int NB, int KMAX>
