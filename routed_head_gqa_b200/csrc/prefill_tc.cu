@@ -49,7 +49,7 @@ constexpr uint32_t kTileBytes = 2 * kHalf; // [128][128] bf16, 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * tile
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: p <= 2^8 between rescales
-constexpr int kPolyPairs = 7;               // of every 16 element pairs, exp2 on the FMA pipe
+constexpr int kPolyPairs = 4;               // of every 16 element pairs, exp2 on the FMA pipe
 constexpr uint32_t kWhereTc = 2;            // status "where" id of this kernel
 // Register split (setmaxnreg): 4 control warps at 88, 8 softmax warps at 208.
 // 128*88 + 256*208 = 64512 = 384 * 168, the block's registers at launch.
@@ -225,24 +225,33 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, kD, false, true);
             uint32_t kv_it = 0, u_it = 0, c[kQT] = {0, 0};
             bool ok = true;
+            // Shared-memory descriptors are built once: a K step only moves the
+            // start address (16-byte units in the low word), so each MMA adds a
+            // compile-time offset instead of rebuilding the descriptor (the
+            // single issuing thread's scalar work would otherwise outlast the
+            // MMAs).  The high word (stride offset 1024, 128-byte swizzle) is
+            // shared by every operand here.
+            const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
+            const uint32_t qlo0 = smem_desc_lo(smem_u32(sm.q[0]), 16), qlo1 = smem_desc_lo(smem_u32(sm.q[1]), 16);
+            const uint32_t klo0 = smem_desc_lo(smem_u32(sm.k[0]), 16), klo1 = smem_desc_lo(smem_u32(sm.k[1]), 16);
+            const uint32_t vlo0 = smem_desc_lo(smem_u32(sm.v[0]), kHalf), vlo1 = smem_desc_lo(smem_u32(sm.v[1]), kHalf);
+            auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
             auto issue_s = [&](int t, uint32_t it) {
-                const uint32_t qaddr = smem_u32(sm.q[t]);
-                const uint32_t kaddr = smem_u32(sm.k[it & 1]);
+                const uint32_t a0 = t ? qlo1 : qlo0, b0 = (it & 1) ? klo1 : klo0;
+                const uint32_t d = tmem + kColS + t * 128;
+#pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    const uint64_t adesc = smem_desc(qaddr + off, 16, 1024, kSwizzle128B);
-                    const uint64_t bdesc = smem_desc(kaddr + off, 16, 1024, kSwizzle128B);
-                    umma_ss(tmem + kColS + t * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                    umma_ss(d, desc(a0 + off), desc(b0 + off), idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sm.s_full[t]);
             };
             auto issue_pv = [&](int t, uint32_t it, bool first) {
-                const uint32_t vaddr = smem_u32(sm.v[it & 1]);
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t bdesc = smem_desc(vaddr + kk * 2048, kHalf, 1024, kSwizzle128B);
-                    umma_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + kk * 8, bdesc, idesc_pv,
-                            (first && kk == 0) ? 0u : 1u);
-                }
+                const uint32_t b0 = (it & 1) ? vlo1 : vlo0;
+                const uint32_t d = tmem + kColO + t * 128, a = tmem + kColS + t * 128;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    umma_ts(d, a + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
             };
             auto wait_k = [&](uint32_t it) { return mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1); };
             auto wait_v = [&](uint32_t it) { return mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1); };
@@ -587,7 +596,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     l *= alpha;
                 }
                 // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
-                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
+                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe (4 of 16
+                // measured fastest with both softmax warpgroups active: MUFU is then
+                // about 80 % busy and the FMA and integer pipes take the rest).
                 const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);
                 const uint64_t NM2 = pk2(-m_use, -m_use);
                 uint64_t sum2[4] = {0, 0, 0, 0};

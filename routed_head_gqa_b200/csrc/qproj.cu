@@ -196,18 +196,22 @@ qproj_kernel(const __grid_constant__ CUtensorMap mapXT, const __grid_constant__ 
     if (warp == 1 && lane == 0) {
         // MMA issuer: D[128 tokens][128] += x_rows . W_Q block
         const uint32_t idesc = idesc_bf16_f32(kM, kN, false, true);
+        const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
+        const uint32_t alo0 = smem_desc_lo(smem_u32(sm.a[0][0]), 16);
+        const uint32_t blo0 = smem_desc_lo(smem_u32(sm.b[0][0]), kBBlock);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kStages;
             if (!mbar_wait(&sm.full[s], (kb / kStages) & 1)) { sm.failed = 1; break; }
             tc_fence_after();
-            const uint32_t ba = smem_u32(sm.b[s][0]);
+            // stage s, tile t: constant strides from stage 0 (16-byte units in the low word)
+            const uint32_t blo = blo0 + (uint32_t)s * ((2 * kBBlock) >> 4);
+#pragma unroll
             for (int t = 0; t < kTiles; ++t) {
-                const uint32_t aa = smem_u32(sm.a[s][t]);
-                for (int kk = 0; kk < kTK / 16; ++kk) {
-                    const uint64_t adesc = smem_desc(aa + kk * 32, 16, 1024, kSwizzle128B);
-                    const uint64_t bdesc = smem_desc(ba + kk * 2048, kBBlock, 1024, kSwizzle128B);
-                    umma_ss(tmem + t * kN, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                }
+                const uint32_t alo = alo0 + (uint32_t)(s * kTiles + t) * (kABytes >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kTK / 16; ++kk)
+                    umma_ss(tmem + t * kN, smem_desc_join(alo + kk * 2, dhi), smem_desc_join(blo + kk * 128, dhi),
+                            idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&sm.empty[s]);
         }

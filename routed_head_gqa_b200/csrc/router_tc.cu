@@ -138,17 +138,20 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
     } else if (warp == 1 && lane == 0) {
         // MMA issuer: D[128 tokens][64*NB heads] += x_tile . W_block over the slice
         const uint32_t idesc = idesc_bf16_f32(kTM, 64 * NB, false, true);
+        const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
+        const uint32_t xlo0 = smem_desc_lo(smem_u32(sm.x[0]), 16);
+        const uint32_t wlo0 = smem_desc_lo(smem_u32(sm.w[0][0]), kWBlock);
         for (int i = 0; i < nkl; ++i) {
             const int s = i % S;
             if (!mbar_wait(&sm.full[s], (i / S) & 1)) { sm.failed = 1; break; }
             tc_fence_after();
-            const uint32_t xa = smem_u32(sm.x[s]);
-            const uint32_t wa = smem_u32(sm.w[s][0]);
-            for (int kk = 0; kk < kTK / 16; ++kk) {
-                const uint64_t adesc = smem_desc(xa + kk * 32, 16, 1024, kSwizzle128B);
-                const uint64_t bdesc = smem_desc(wa + kk * 2048, kWBlock, 1024, kSwizzle128B);
-                umma_ss(tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-            }
+            // stage s starts s * sizeof(stage) bytes after stage 0 (16-byte units in the low word)
+            const uint32_t xlo = xlo0 + (uint32_t)s * (kXBytes >> 4);
+            const uint32_t wlo = wlo0 + (uint32_t)s * ((NB * kWBlock) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kTK / 16; ++kk)
+                umma_ss(tmem, smem_desc_join(xlo + kk * 2, dhi), smem_desc_join(wlo + kk * 128, dhi), idesc,
+                        (i > 0 || kk > 0) ? 1u : 0u);
             umma_commit(&sm.empty[s]);
         }
         umma_commit(&sm.acc_full);
