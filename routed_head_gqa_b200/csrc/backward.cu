@@ -403,10 +403,12 @@ cudaError_t launch_typed(const AttnBwdArgs& a) {
 }  // namespace
 
 size_t attn_backward_scratch_bytes(const gqe_shape* s) {
+    if (attn_backward_tc_supported(s)) return attn_backward_tc_scratch_bytes(s);
     return 3 * a256((size_t)s->B * s->T * s->h * sizeof(float));
 }
 
 cudaError_t launch_attn_backward(const AttnBwdArgs& a) {
+    if (attn_backward_tc_supported(a.s)) return launch_attn_backward_tc(a);
     const bool bf16 = a.s->dtype == GQE_BF16;
     switch (a.s->d_h) {
         case 32: return bf16 ? launch_typed<__nv_bfloat16, 32>(a) : launch_typed<float, 32>(a);

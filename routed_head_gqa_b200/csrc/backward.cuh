@@ -25,9 +25,15 @@ struct AttnBwdArgs {
     cudaStream_t stream;
 };
 
-// Per-(b,t,j) scratch of the backward: gate, D = dO.O and the row's log2-sum-exp.
+// Per-(b,t,j) scratch of the backward: gate, D = dO.O and the row's log2-sum-exp
+// (plus, on the tensor-core path, each routed row's ungated fp32 output).
 size_t attn_backward_scratch_bytes(const gqe_shape* s);
 cudaError_t launch_attn_backward(const AttnBwdArgs& a);
+
+// Tensor-core backward (backward_tc.cu): bf16, d_h = 128, k <= 4, h/g <= 32.
+bool attn_backward_tc_supported(const gqe_shape* s);
+size_t attn_backward_tc_scratch_bytes(const gqe_shape* s);
+cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a);
 
 struct RouteBwdArgs {
     const gqe_shape* s;

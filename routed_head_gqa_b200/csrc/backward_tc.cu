@@ -1,0 +1,924 @@
+// backward_tc.cu -- backward of the routed attention on the sm_100a tensor
+// cores (bf16 inputs, d_h = 128, fp32 gradients).
+//
+// The pages give no backward for GQE; this is the chain rule through the
+// forward ("Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention",
+// gist.science summary, "Architecture et Routage" and "Somme Ponderee
+// Renormalisee"; IBM GQA page for the scaled dot-product attention).  For a
+// routed row r = (b, t, j) of group q with gate g_r, weights p_rs over the keys
+// s <= t, ungated output o_r and incoming gradient dO_r:
+//   D_r   = g_r dO_r . o_r
+//   dS_rs = p_rs (g_r dO_r . v_s - D_r)
+//   dQ_r  = sum_s dS_rs k_s / sqrt(d),   dK_s = sum_r dS_rs q_r / sqrt(d),
+//   dV_s  = sum_r p_rs g_r dO_r,         dlogit_j = D_j - g_j sum_{i in S} D_i.
+//
+// Launches (after the tensor-core prefill has written o_r in fp32 and the
+// row's log2-sum-exp lse_r into the workspace, so p_rs = 2^(s_rs c - lse_r)):
+//  1. bwd_prep_kernel: one warp per (b, t, group): D_r, the gates, the logit
+//     gradients, and zero dQ rows for the unselected heads.
+//  2. dq_tc_kernel: per 128-row tile of routed rows (the prefill's half-window
+//     tiles): S = Q K^T and dP = dO V^T on the tensor cores, dS in registers,
+//     dQ += dS K accumulated in TMEM.
+//  3. dkdv_tc_kernel: per (b, group, 128-key tile): S^T = K Q^T and
+//     dP^T = V dO^T over the group's routed row tiles at or after the keys,
+//     then dV += (g p)^T dO and dK += dS^T Q accumulated in TMEM.
+// Every sum runs in a fixed order: the gradients are reproducible.
+#include <climits>
+
+#include "backward.cuh"
+#include "sm100.cuh"
+#include "tma_host.cuh"
+#include "units.cuh"
+
+namespace gqe {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kBM = 128;                   // rows (or keys) per tile
+constexpr int kThreads = 256;              // 8 warps
+constexpr uint32_t kHalf = 128 * 64 * 2;   // [128][64] bf16 box, 16 KB
+constexpr uint32_t kTile = 2 * kHalf;      // [128][128] bf16, 32 KB
+constexpr uint32_t kWhereBwdTc = 9;
+constexpr int kQT = 2;                     // half-window tiles per window
+
+__device__ __forceinline__ bool aborted(const int32_t* flag) { return *((volatile const int32_t*)flag) != 0; }
+
+// ------------------------------------------------------------------ row tables
+// The routed rows of one half-window tile (b, group q, first position w0, W
+// positions): the concatenation over the group's heads of each head's slice of
+// its packed position list.  Built by one warp; rows past the tile's count
+// (and rows whose position falls outside the tile) are padding (t = -1).
+struct RowTable {
+    int32_t t[kBM];
+    int32_t j[kBM];
+    float gate[kBM];
+    float lse[kBM];
+    float dlt[kBM];
+    int32_t qrow[kBM];  // row of Q / dO viewed as [B*T*h, 128]; padding rows name q_rows (zero fill)
+};
+
+__device__ void build_rows(const UnitGeom& u, int b, int q, int w0, const int32_t* head_offsets,
+                           const int32_t* head_chunk_offsets, const int32_t* head_pos, const int32_t* idx,
+                           const float* gate_in, const float* lse, const float* dlt, int q_rows, RowTable& rt,
+                           int32_t* cut_start, int32_t* cut_prefix, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int32_t total = (int32_t)((int64_t)u.B * u.T * u.g * u.k);
+    if (lane < u.hpg) {
+        const int jh = q * u.hpg + lane;
+        int32_t a0 = list_cut(u, head_offsets, head_chunk_offsets, b, jh, w0);
+        int32_t a1 = list_cut(u, head_offsets, head_chunk_offsets, b, jh, w0 + u.W);
+        if (a0 < 0 || a1 < a0 || a1 > total) {
+            report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 1);
+            a0 = a1 = 0;
+        }
+        cut_start[lane] = a0;
+        cut_prefix[lane + 1] = a1 - a0;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        int acc = 0;
+        cut_prefix[0] = 0;
+        for (int jj = 0; jj < u.hpg; ++jj) {
+            acc = min(acc + cut_prefix[jj + 1], kBM);
+            cut_prefix[jj + 1] = acc;
+        }
+    }
+    __syncwarp();
+    const int nrows = cut_prefix[u.hpg];
+    for (int r = lane; r < kBM; r += 32) {
+        int tt = -1, jh = 0;
+        float gv = 0.f, lv = 0.f, dv = 0.f;
+        if (r < nrows) {
+            int jj = 0;
+            while (cut_prefix[jj + 1] <= r) ++jj;
+            jh = q * u.hpg + jj;
+            tt = head_pos[cut_start[jj] + (r - cut_prefix[jj])];
+            if (tt < w0 || tt >= min(w0 + u.W, u.T)) {
+                report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 2);
+                tt = -1;
+            }
+        }
+        if (tt >= 0) {
+            const int64_t sel = (((int64_t)b * u.T + tt) * u.g + q) * u.k;
+            for (int s2 = 0; s2 < u.k; ++s2)
+                if (idx[sel + s2] == jh) gv = gate_in[sel + s2];
+            const int64_t row = ((int64_t)b * u.T + tt) * u.h + jh;
+            lv = lse[row];
+            dv = dlt[row];
+        }
+        rt.t[r] = tt;
+        rt.j[r] = jh;
+        rt.gate[r] = gv;
+        rt.lse[r] = lv;
+        rt.dlt[r] = dv;
+        rt.qrow[r] = (tt >= 0) ? (int32_t)(((int64_t)b * u.T + tt) * u.h + jh) : q_rows;
+    }
+    __syncwarp();
+}
+
+// Q and dO rows of a table by TMA gather (four rows per copy, two 64-column
+// halves), 128B-swizzled [128][64] boxes; padding rows are zero-filled.
+__device__ __forceinline__ void gather_rows(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, const RowTable& rt) {
+    const int lane = threadIdx.x & 31;
+    const int r0 = lane * 4;
+    tma_gather4_2d(map, bar, dst + r0 * 128, 0, rt.qrow[r0], rt.qrow[r0 + 1], rt.qrow[r0 + 2], rt.qrow[r0 + 3]);
+    tma_gather4_2d(map, bar, dst + kHalf + r0 * 128, 64, rt.qrow[r0], rt.qrow[r0 + 1], rt.qrow[r0 + 2],
+                   rt.qrow[r0 + 3]);
+}
+
+// p = 2^(s c - lse) (0 where masked), pg = gate p, ds = p (gate dp - D), as
+// bf16 pairs; 32 values of s and dp, one pair of table entries per step.
+struct Elem2 {
+    uint32_t pg, ds;
+};
+
+// ------------------------------------------------------------------ 1. prep
+__global__ void __launch_bounds__(256)
+bwd_prep_kernel(int64_t BT, int h, int g, int k, const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                const __nv_bfloat16* __restrict__ dO, const float* __restrict__ o32, float* __restrict__ gamma,
+                float* __restrict__ delta, float* __restrict__ dlogits, float* __restrict__ dQ, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t item = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // bt * g + q
+    if (item >= BT * g) return;
+    const int64_t bt = item / g;
+    const int q = (int)(item % g), hpg = h / g;
+    float dsel[16], gsel[16];
+    int jsel[16];
+    float dsum = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        dsel[s] = 0.f;
+        gsel[s] = 0.f;
+        jsel[s] = -1;
+        if (s < k) {
+            const int j = idx[item * k + s];
+            if (j < q * hpg || j >= (q + 1) * hpg) {
+                if (lane == 0) report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 3);
+                continue;
+            }
+            const float gm = gate[item * k + s];
+            const int64_t row = bt * h + j;
+            // D = g dO . o over the row's 128 elements, 4 per lane, then a butterfly
+            const uint2 dv = *reinterpret_cast<const uint2*>(dO + row * kD + lane * 4);
+            const float4 ov = *reinterpret_cast<const float4*>(o32 + row * kD + lane * 4);
+            float acc = __uint_as_float(dv.x << 16) * ov.x + __uint_as_float(dv.x & 0xffff0000u) * ov.y +
+                        __uint_as_float(dv.y << 16) * ov.z + __uint_as_float(dv.y & 0xffff0000u) * ov.w;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+            jsel[s] = j;
+            gsel[s] = gm;
+            dsel[s] = gm * acc;
+            dsum += dsel[s];
+            if (lane == 0) {
+                gamma[row] = gm;
+                delta[row] = dsel[s];
+            }
+        }
+    }
+    for (int jj = lane; jj < hpg; jj += 32) {
+        const int j = q * hpg + jj;
+        float dl = 0.f;
+#pragma unroll
+        for (int s = 0; s < 16; ++s)
+            if (s < k && jsel[s] == j) dl = dsel[s] - gsel[s] * dsum;
+        dlogits[bt * h + j] = dl;
+    }
+    for (int jj = 0; jj < hpg; ++jj) {  // dQ of an unselected head is 0
+        const int j = q * hpg + jj;
+        bool sel = false;
+#pragma unroll
+        for (int s = 0; s < 16; ++s) sel |= (s < k && jsel[s] == j);
+        if (sel) continue;
+        *reinterpret_cast<float4*>(dQ + (bt * h + j) * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// ------------------------------------------------------------------ shared pieces
+struct Params {
+    UnitGeom u;
+    const int32_t* idx;
+    const float* gate;
+    const int32_t* head_offsets;
+    const int32_t* head_pos;
+    const int32_t* head_chunk_offsets;
+    const float* lse;
+    const float* dlt;
+    float* dQ;
+    float* dK;
+    float* dV;
+    uint32_t* status;
+    float scale_log2;  // log2(e) / sqrt(128)
+    float scale;       // 1 / sqrt(128)
+    int q_rows;        // B*T*h
+};
+
+__device__ __forceinline__ void fail(int32_t* abort_flag, uint32_t* status, uint32_t detail) {
+    atomicExch(abort_flag, 1);
+    report_error(status, GQE_ERR_DEVICE_TIMEOUT, kWhereBwdTc, detail);
+}
+
+// One 32-column chunk of the elementwise step: s (scores) and d (dP) for 32
+// columns c0..c0+31 of this thread's TMEM lane; per column the table entry gives
+// lse, gate, D and visibility.  Returns 16 packed pairs of pg and ds.
+template <bool KEY_ROWS>
+__device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float c, float lse_or_row,
+                                         float gate_row, float dlt_row, int key_or_t, const RowTable& rt, int col0,
+                                         int kv0, uint32_t (&pg)[16], uint32_t (&ds)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float p2[2], q2[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int cc = col0 + 2 * e + h2;
+            float lse, gm, dl;
+            bool vis;
+            if (KEY_ROWS) {  // thread = key (global index key_or_t), column = row cc of the table
+                lse = rt.lse[cc];
+                gm = rt.gate[cc];
+                dl = rt.dlt[cc];
+                const int tr = rt.t[cc];
+                vis = tr >= 0 && key_or_t <= tr;
+            } else {         // thread = row (position key_or_t), column = key kv0 + cc
+                lse = lse_or_row;
+                gm = gate_row;
+                dl = dlt_row;
+                vis = key_or_t >= 0 && kv0 + cc <= key_or_t;
+            }
+            const float x = __uint_as_float(s[2 * e + h2]) * c - lse;
+            const float p = vis ? fast_exp2(x) : 0.f;
+            p2[h2] = p * gm;
+            q2[h2] = p * (gm * __uint_as_float(dp[2 * e + h2]) - dl);
+        }
+        pg[e] = pack_bf16x2(p2[0], p2[1]);
+        ds[e] = pack_bf16x2(q2[0], q2[1]);
+    }
+}
+
+// ------------------------------------------------------------------ 2. dQ
+// One CTA per SM; work item = one half-window tile of 128 routed rows.
+// Roles: warp 0 K/V producer (2-stage ring), warp 1 MMA issuer, warp 2 row
+// table + Q/dO gather, warps 4-7 elementwise + epilogue (thread = row).
+// TMEM: S buffers [0,128) and [128,256), dP [256,384), dQ [384,512); dS
+// (bf16 pairs) overwrites the first 64 columns of dP once dP is in registers.
+struct DqSmem {
+    uint8_t q[kTile];
+    uint8_t dO[kTile];
+    uint8_t k[2][kTile];
+    uint8_t v[2][kTile];
+    RowTable rt;
+    int32_t cut_start[32];
+    int32_t cut_prefix[33];
+    uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
+    uint64_t rows_full, rows_empty, s_full[2], dp_full, ew_done, dq_full, dq_empty, drain;
+    uint32_t tmem_base;
+    int32_t abort_flag;
+};
+
+__device__ __forceinline__ int dq_items(const UnitGeom& u) { return (int)(u.count() * kQT); }
+// Item i: heaviest windows first (unit order of the prefill), two halves per unit.
+__device__ __forceinline__ void dq_item(const UnitGeom& u, int64_t i, int& b, int& q, int& w0, int& nkv) {
+    int w;
+    unit_coords(u, i / kQT, b, q, w);
+    const int half = (int)(i % kQT);
+    w0 = (w * kQT + half) * u.W;
+    const int end = min(w0 + u.W, u.T);
+    nkv = (end + kBM - 1) / kBM;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+             const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    DqSmem& sm = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const UnitGeom& u = p.u;
+    const int64_t n_items = dq_items(u);
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.kv_full_k[i], 1);
+            mbar_init(&sm.kv_full_v[i], 1);
+            mbar_init(&sm.kv_empty_k[i], 1);
+            mbar_init(&sm.kv_empty_v[i], 1);
+            mbar_init(&sm.s_full[i], 1);
+        }
+        mbar_init(&sm.rows_full, 1);
+        mbar_init(&sm.rows_empty, 2);  // the MMA issuer (operands read) and the elementwise warps (table read)
+        mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.ew_done, 128);
+        mbar_init(&sm.dq_full, 1);
+        mbar_init(&sm.dq_empty, 128);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ K/V producer
+        if (lane == 0) {
+            uint32_t kv = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+                int b, q, w0, nkv;
+                dq_item(u, it, b, q, w0, nkv);
+                for (int i = 0; i < nkv; ++i, ++kv) {
+                    const int st = kv & 1;
+                    const uint32_t par = ((kv >> 1) & 1) ^ 1;
+                    if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(&sm.abort_flag, p.status, 1); ok = false; break; }
+                    mbar_arrive_expect_tx(&sm.kv_full_k[st], kTile);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, q, i * kBM, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, q, i * kBM, b);
+                    if (!mbar_wait(&sm.kv_empty_v[st], par)) { fail(&sm.abort_flag, p.status, 2); ok = false; break; }
+                    mbar_arrive_expect_tx(&sm.kv_full_v[st], kTile);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, q, i * kBM, b);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, q, i * kBM, b);
+                }
+            }
+            // every issued load lands before the CTA may exit
+            for (uint32_t back = 1; back <= 2 && back <= kv; ++back) {
+                const uint32_t it = kv - back;
+                mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1);
+                mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
+            const uint32_t idesc_dq = idesc_bf16_f32(kBM, kD, false, true);
+            const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
+            const uint32_t qlo = smem_desc_lo(smem_u32(sm.q), 16), dolo = smem_desc_lo(smem_u32(sm.dO), 16);
+            const uint32_t klo0 = smem_desc_lo(smem_u32(sm.k[0]), 16), klo1 = smem_desc_lo(smem_u32(sm.k[1]), 16);
+            const uint32_t kmlo0 = smem_desc_lo(smem_u32(sm.k[0]), kHalf), kmlo1 = smem_desc_lo(smem_u32(sm.k[1]), kHalf);
+            const uint32_t vlo0 = smem_desc_lo(smem_u32(sm.v[0]), 16), vlo1 = smem_desc_lo(smem_u32(sm.v[1]), 16);
+            const uint32_t c_s = tmem, c_dp = tmem + 256, c_dq = tmem + 384;
+            auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
+            // S(kv tile) into S buffer sb: Q . K^T (both K-major).
+            auto issue_s = [&](uint32_t kvi, uint32_t sb) {
+                const uint32_t kb = (kvi & 1) ? klo1 : klo0;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                    umma_ss(c_s + sb * 128, desc(qlo + off), desc(kb + off), idesc_ss, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.s_full[sb]);
+            };
+            // dP = dO . V^T (V rows as a K-major operand).
+            auto issue_dp = [&](uint32_t kvi) {
+                const uint32_t vb = (kvi & 1) ? vlo1 : vlo0;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                    umma_ss(c_dp, desc(dolo + off), desc(vb + off), idesc_ss, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.dp_full);
+            };
+            // dQ (+)= dS . K (dS bf16 pairs in dP's first 64 columns; K MN-major).
+            auto issue_dq = [&](uint32_t kvi, bool first) {
+                const uint32_t kb = (kvi & 1) ? kmlo1 : kmlo0;
+#pragma unroll
+                for (int kk = 0; kk < kBM / 16; ++kk)
+                    umma_ts(c_dq, c_dp + kk * 8, desc(kb + (uint32_t)((kk * 2048) >> 4)), idesc_dq,
+                            (first && kk == 0) ? 0u : 1u);
+            };
+            auto wait_k = [&](uint32_t x) { return mbar_wait(&sm.kv_full_k[x & 1], (x >> 1) & 1); };
+            auto wait_v = [&](uint32_t x) { return mbar_wait(&sm.kv_full_v[x & 1], (x >> 1) & 1); };
+            uint32_t kv = 0, sc = 0, ec = 0, item_no = 0;  // kv tiles, S issued, elementwise steps, items
+            bool ok = true;
+            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+                int b, q, w0, nkv;
+                dq_item(u, it, b, q, w0, nkv);
+                if (!mbar_wait(&sm.rows_full, item_no & 1)) { fail(&sm.abort_flag, p.status, 10); break; }
+                tc_fence_after();
+                // prologue: S(0), dP(0), S(1)
+                if (!(ok = wait_k(kv))) { fail(&sm.abort_flag, p.status, 11); break; }
+                tc_fence_after();
+                issue_s(kv, sc & 1);
+                ++sc;
+                if (!(ok = wait_v(kv))) { fail(&sm.abort_flag, p.status, 12); break; }
+                tc_fence_after();
+                issue_dp(kv);
+                umma_commit(&sm.kv_empty_v[kv & 1]);  // V(0) is only read by dP(0)
+                if (nkv > 1) {
+                    if (!(ok = wait_k(kv + 1))) { fail(&sm.abort_flag, p.status, 13); break; }
+                    tc_fence_after();
+                    issue_s(kv + 1, sc & 1);
+                    ++sc;
+                }
+                for (int i = 0; i < nkv; ++i) {
+                    const uint32_t x = kv + i;
+                    // dS(i) is in dP's columns once the elementwise step i is done
+                    if (!(ok = mbar_wait(&sm.ew_done, ec & 1))) { fail(&sm.abort_flag, p.status, 14); break; }
+                    ++ec;
+                    if (i == 0 && !(ok = mbar_wait(&sm.dq_empty, (item_no & 1) ^ 1))) {
+                        fail(&sm.abort_flag, p.status, 15);
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_dq(x, i == 0);
+                    umma_commit(&sm.kv_empty_k[x & 1]);  // K(i): read by S(i) and dQ(i)
+                    if (i == nkv - 1) {
+                        umma_commit(&sm.dq_full);
+                        umma_commit(&sm.rows_empty);  // Q and dO of the item are no longer read
+                    }
+                    if (i + 1 < nkv) {
+                        if (!(ok = wait_v(x + 1))) { fail(&sm.abort_flag, p.status, 16); break; }
+                        tc_fence_after();
+                        issue_dp(x + 1);
+                        umma_commit(&sm.kv_empty_v[(x + 1) & 1]);
+                    }
+                    if (i + 2 < nkv) {
+                        if (!(ok = wait_k(x + 2))) { fail(&sm.abort_flag, p.status, 17); break; }
+                        tc_fence_after();
+                        issue_s(x + 2, sc & 1);
+                        ++sc;
+                    }
+                }
+                kv += nkv;
+            }
+            umma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ row table + Q / dO gather
+        uint32_t item_no = 0;
+        bool armed = false;
+        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+            int b, q, w0, nkv;
+            dq_item(u, it, b, q, w0, nkv);
+            // the previous item's operands and table are free
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_empty, (item_no & 1) ^ 1))) {
+                if (lane == 0) fail(&sm.abort_flag, p.status, 20);
+                break;
+            }
+            build_rows(u, b, q, w0, p.head_offsets, p.head_chunk_offsets, p.head_pos, p.idx, p.gate, p.lse, p.dlt,
+                       p.q_rows, sm.rt, sm.cut_start, sm.cut_prefix, p.status);
+            if (lane == 0) mbar_arrive_expect_tx(&sm.rows_full, 2 * kTile);
+            __syncwarp();
+            gather_rows(&mapQ, &sm.rows_full, sm.q, sm.rt);
+            gather_rows(&mapdO, &sm.rows_full, sm.dO, sm.rt);
+            armed = true;
+        }
+        if (armed) mbar_wait(&sm.rows_full, (item_no - 1) & 1);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ elementwise + epilogue (thread = row)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        uint32_t sc = 0, item_no = 0;
+        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+            int b, q, w0, nkv;
+            dq_item(u, it, b, q, w0, nkv);
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_full, item_no & 1))) {
+                if (lane == 0) fail(&sm.abort_flag, p.status, 30);
+                break;
+            }
+            const int t_row = sm.rt.t[r];
+            const float lse = sm.rt.lse[r], gm = sm.rt.gate[r], dl = sm.rt.dlt[r];
+            const int j_row = sm.rt.j[r];
+            bool ok = true;
+            for (int i = 0; i < nkv; ++i, ++sc) {
+                const uint32_t sb = sc & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (sc >> 1) & 1) &&
+                                                 mbar_wait(&sm.dp_full, sc & 1))) {
+                    if (lane == 0) fail(&sm.abort_flag, p.status, 31);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t s_addr = tmem + lane_off + sb * 128, d_addr = tmem + lane_off + 256;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {  // two 64-column halves; dS of half hh goes to columns 32hh..
+                    uint32_t pg[2][16], ds[2][16];
+#pragma unroll
+                    for (int cb = 0; cb < 2; ++cb) {
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(s_addr + hh * 64 + cb * 32, sv);
+                        tmem_ld32(d_addr + hh * 64 + cb * 32, dv);
+                        tmem_ld_wait();
+                        ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.rt, hh * 64 + cb * 32, i * kBM,
+                                        pg[cb], ds[cb]);
+                    }
+                    tmem_st16(d_addr + hh * 32, ds[0]);
+                    tmem_st16(d_addr + hh * 32 + 16, ds[1]);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.ew_done);
+            }
+            if (!ok) break;
+            // epilogue: dQ = (sum_s dS k_s) / sqrt(d), fp32 rows of the routed heads
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.dq_full, item_no & 1))) {
+                if (lane == 0) fail(&sm.abort_flag, p.status, 34);
+                break;
+            }
+            tc_fence_after();
+            float* drow = p.dQ + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD;
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + 384 + cb * 32, o);
+                tmem_ld_wait();
+                if (t_row >= 0) {
+                    float4* dst = reinterpret_cast<float4*>(drow + cb * 32);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        dst[v] = make_float4(__uint_as_float(o[4 * v]) * p.scale, __uint_as_float(o[4 * v + 1]) * p.scale,
+                                             __uint_as_float(o[4 * v + 2]) * p.scale,
+                                             __uint_as_float(o[4 * v + 3]) * p.scale);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.dq_empty);
+            if (wq == 0 && lane == 0) mbar_arrive(&sm.rows_empty);  // this item's table is no longer read
+            // (the table is read until here; the MMA issuer's rows_empty commit covers the operands)
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ 3. dK, dV
+// Work item = (b, group q, 128-key tile kt), heaviest (earliest keys) first.
+// Its rows are the group's half-window tiles from the one holding key 128*kt
+// on.  Roles: warp 0 K/V of the item, warp 1 MMA issuer, warp 2 row tables +
+// Q/dO gather (double buffered), warps 4-7 elementwise + epilogue (thread =
+// key).  TMEM: dK [0,128), dV [128,256), S^T [256,384), dP^T [384,512); g p
+// and dS (bf16 pairs) overwrite the first 64 columns of S^T and dP^T.
+struct KvSmem {
+    uint8_t k[kTile];
+    uint8_t v[kTile];
+    uint8_t q[2][kTile];
+    uint8_t dO[2][kTile];
+    RowTable rt[2];
+    int32_t cut_start[32];
+    int32_t cut_prefix[33];
+    uint64_t kv_full, kv_empty, rows_full[2], rows_empty[2], st_full, ew_done, acc_full, acc_empty, drain;
+    uint32_t tmem_base;
+    int32_t abort_flag;
+};
+
+__device__ __forceinline__ int64_t kv_items(const UnitGeom& u) {
+    return (int64_t)u.B * u.g * ((u.T + kBM - 1) / kBM);
+}
+__device__ __forceinline__ void kv_item(const UnitGeom& u, int64_t i, int& b, int& q, int& kt, int& tile0,
+                                        int& ntiles) {
+    const int64_t per = (int64_t)u.B * u.g;
+    kt = (int)(i / per);
+    const int rem = (int)(i % per);
+    b = rem / u.g;
+    q = rem % u.g;
+    tile0 = (kt * kBM) / u.W;           // first half-window tile holding a position >= 128 kt
+    ntiles = (u.T + u.W - 1) / u.W - tile0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+               const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    KvSmem& sm = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const UnitGeom& u = p.u;
+    const int64_t n_items = kv_items(u);
+    if (tid == 0) {
+        mbar_init(&sm.kv_full, 1);
+        mbar_init(&sm.kv_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.rows_full[i], 1);
+            mbar_init(&sm.rows_empty[i], 2);  // MMA issuer (operands) and elementwise warps (table)
+        }
+        mbar_init(&sm.st_full, 1);
+        mbar_init(&sm.ew_done, 128);
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, 128);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ K/V of each item
+        if (lane == 0) {
+            uint32_t n = 0;
+            for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+                int b, q, kt, tile0, ntiles;
+                kv_item(u, it, b, q, kt, tile0, ntiles);
+                if (!mbar_wait(&sm.kv_empty, (n & 1) ^ 1)) { fail(&sm.abort_flag, p.status, 101); break; }
+                mbar_arrive_expect_tx(&sm.kv_full, 2 * kTile);
+                tma_load_4d(&mapK, &sm.kv_full, sm.k, 0, q, kt * kBM, b);
+                tma_load_4d(&mapK, &sm.kv_full, sm.k + kHalf, 64, q, kt * kBM, b);
+                tma_load_4d(&mapV, &sm.kv_full, sm.v, 0, q, kt * kBM, b);
+                tma_load_4d(&mapV, &sm.kv_full, sm.v + kHalf, 64, q, kt * kBM, b);
+            }
+            if (n > 0) mbar_wait(&sm.kv_full, (n - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
+            const uint32_t idesc_acc = idesc_bf16_f32(kBM, kD, false, true);
+            const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
+            const uint32_t klo = smem_desc_lo(smem_u32(sm.k), 16), vlo = smem_desc_lo(smem_u32(sm.v), 16);
+            const uint32_t qlo0 = smem_desc_lo(smem_u32(sm.q[0]), 16), dolo0 = smem_desc_lo(smem_u32(sm.dO[0]), 16);
+            const uint32_t qmlo0 = smem_desc_lo(smem_u32(sm.q[0]), kHalf), domlo0 = smem_desc_lo(smem_u32(sm.dO[0]), kHalf);
+            const uint32_t buf_step = kTile >> 4;  // the second Q / dO buffer, in 16-byte units
+            const uint32_t c_dk = tmem, c_dv = tmem + 128, c_st = tmem + 256, c_dpt = tmem + 384;
+            auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
+            uint32_t n = 0, rc = 0;  // items, row tiles
+            bool ok = true;
+            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+                int b, q, kt, tile0, ntiles;
+                kv_item(u, it, b, q, kt, tile0, ntiles);
+                if (!mbar_wait(&sm.kv_full, n & 1)) { fail(&sm.abort_flag, p.status, 110); break; }
+                if (!mbar_wait(&sm.acc_empty, (n & 1) ^ 1)) { fail(&sm.abort_flag, p.status, 111); break; }
+                tc_fence_after();
+                for (int i = 0; i < ntiles; ++i, ++rc) {
+                    const uint32_t rb = rc & 1;
+                    if (!(ok = mbar_wait(&sm.rows_full[rb], (rc >> 1) & 1))) { fail(&sm.abort_flag, p.status, 112); break; }
+                    tc_fence_after();
+                    const uint32_t qb = qlo0 + rb * buf_step, dob = dolo0 + rb * buf_step;
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {  // S^T = K . Q^T
+                        const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                        umma_ss(c_st, desc(klo + off), desc(qb + off), idesc_ss, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {  // dP^T = V . dO^T
+                        const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                        umma_ss(c_dpt, desc(vlo + off), desc(dob + off), idesc_ss, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&sm.st_full);
+                    if (!(ok = mbar_wait(&sm.ew_done, rc & 1))) { fail(&sm.abort_flag, p.status, 113); break; }
+                    tc_fence_after();
+                    const uint32_t qmb = qmlo0 + rb * buf_step, domb = domlo0 + rb * buf_step;
+#pragma unroll
+                    for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += (g p)^T . dO ; dK += dS^T . Q
+                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                        umma_ts(c_dv, c_st + kk * 8, desc(domb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
+                        umma_ts(c_dk, c_dpt + kk * 8, desc(qmb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
+                    }
+                    umma_commit(&sm.rows_empty[rb]);
+                }
+                if (!ok) break;
+                umma_commit(&sm.kv_empty);
+                umma_commit(&sm.acc_full);
+            }
+            umma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ row tables + Q / dO gather
+        uint32_t rc = 0;
+        int64_t armed = -1;
+        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x) {
+            int b, q, kt, tile0, ntiles;
+            kv_item(u, it, b, q, kt, tile0, ntiles);
+            bool ok = true;
+            for (int i = 0; i < ntiles; ++i, ++rc) {
+                const uint32_t rb = rc & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_empty[rb], ((rc >> 1) & 1) ^ 1))) {
+                    if (lane == 0) fail(&sm.abort_flag, p.status, 120);
+                    ok = false;
+                    break;
+                }
+                const int w0 = (tile0 + i) * u.W;
+                build_rows(u, b, q, w0, p.head_offsets, p.head_chunk_offsets, p.head_pos, p.idx, p.gate, p.lse,
+                           p.dlt, p.q_rows, sm.rt[rb], sm.cut_start, sm.cut_prefix, p.status);
+                if (lane == 0) mbar_arrive_expect_tx(&sm.rows_full[rb], 2 * kTile);
+                __syncwarp();
+                gather_rows(&mapQ, &sm.rows_full[rb], sm.q[rb], sm.rt[rb]);
+                gather_rows(&mapdO, &sm.rows_full[rb], sm.dO[rb], sm.rt[rb]);
+                armed = rc;
+            }
+            if (!ok) break;
+        }
+        if (armed >= 0) mbar_wait(&sm.rows_full[armed & 1], (armed >> 1) & 1);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ elementwise + epilogue (thread = key)
+        const int wq = warp & 3;
+        const int kr = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t st_addr = tmem + lane_off + 256, dpt_addr = tmem + lane_off + 384;
+        uint32_t n = 0, rc = 0;
+        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+            int b, q, kt, tile0, ntiles;
+            kv_item(u, it, b, q, kt, tile0, ntiles);
+            const int key = kt * kBM + kr;
+            bool ok = true;
+            for (int i = 0; i < ntiles; ++i, ++rc) {
+                const uint32_t rb = rc & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full, rc & 1))) {
+                    if (lane == 0) fail(&sm.abort_flag, p.status, 130);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const RowTable& rt = sm.rt[rb];
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t pg[2][16], ds[2][16];
+#pragma unroll
+                    for (int cb = 0; cb < 2; ++cb) {
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(st_addr + hh * 64 + cb * 32, sv);
+                        tmem_ld32(dpt_addr + hh * 64 + cb * 32, dv);
+                        tmem_ld_wait();
+                        ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, rt, hh * 64 + cb * 32, 0, pg[cb],
+                                       ds[cb]);
+                    }
+                    tmem_st16(st_addr + hh * 32, pg[0]);
+                    tmem_st16(st_addr + hh * 32 + 16, pg[1]);
+                    tmem_st16(dpt_addr + hh * 32, ds[0]);
+                    tmem_st16(dpt_addr + hh * 32 + 16, ds[1]);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.ew_done);
+                if (wq == 0 && lane == 0) mbar_arrive(&sm.rows_empty[rb]);  // the table is no longer read
+            }
+            if (!ok) break;
+            // epilogue: dK (scaled by 1/sqrt(d)) and dV rows of the item's keys
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full, n & 1))) {
+                if (lane == 0) fail(&sm.abort_flag, p.status, 134);
+                break;
+            }
+            tc_fence_after();
+            const bool key_ok = key < u.T;
+            const int64_t kv_row = ((int64_t)b * u.T + (key_ok ? key : 0)) * u.g + q;
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
+                float* dst_row = (part == 0 ? p.dK : p.dV) + kv_row * kD;
+                const float f = (part == 0) ? p.scale : 1.0f;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + part * 128 + cb * 32, o);
+                    tmem_ld_wait();
+                    if (key_ok) {
+                        float4* dst = reinterpret_cast<float4*>(dst_row + cb * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * f, __uint_as_float(o[4 * v + 1]) * f,
+                                                 __uint_as_float(o[4 * v + 2]) * f, __uint_as_float(o[4 * v + 3]) * f);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+size_t a256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool attn_backward_tc_supported(const gqe_shape* s) {
+    return s->dtype == GQE_BF16 && s->d_h == kD && s->k <= 4 && s->h / s->g <= 32;
+}
+
+size_t attn_backward_tc_scratch_bytes(const gqe_shape* s) {
+    const size_t bth = (size_t)s->B * s->T * s->h;
+    return 3 * a256(bth * sizeof(float)) + a256(bth * kD * sizeof(float));
+}
+
+cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
+    const gqe_shape& s = *a.s;
+    const int64_t BT = (int64_t)s.B * s.T;
+    const size_t plane = a256((size_t)BT * s.h * sizeof(float));
+    float* gamma = static_cast<float*>(a.scratch);
+    float* delta = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + plane);
+    float* lse = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + 2 * plane);
+    float* o32 = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + 3 * plane);
+
+    // 0. the forward again, writing o and the log2-sum-exp of every routed row
+    PrefillArgs f;
+    f.s = a.s;
+    f.Q = a.Q;
+    f.K = a.K;
+    f.V = a.V;
+    f.idx = a.idx;
+    f.gate = a.gate;
+    f.head_offsets = a.head_offsets;
+    f.head_pos = a.head_pos;
+    f.head_chunk_offsets = a.head_chunk_offsets;
+    f.O = nullptr;
+    f.status = a.status;
+    f.stream = a.stream;
+    f.kv_g = s.g;
+    f.kv_q0 = 0;
+    f.o32 = o32;
+    f.lse = lse;
+    cudaError_t e = launch_prefill_tc(f);
+    if (e != cudaSuccess) return e;
+
+    // 1. D, gates, logit gradients, zero dQ of unselected heads
+    const int64_t warps = BT * s.g;
+    bwd_prep_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, a.stream>>>(
+        BT, s.h, s.g, s.k, a.idx, a.gate, (const __nv_bfloat16*)a.dO, o32, gamma, delta, a.dlogits, a.dQ,
+        (uint32_t*)a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // tensor maps: K, V as [B, T, g, 128] (128-key boxes of 64 columns); Q, dO as
+    // [B*T*h, 128] rows (one-row boxes for the gathers)
+    CUtensorMap mapK, mapV, mapQ, mapdO;
+    {
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
+        const uint32_t box[4] = {64, 1, (uint32_t)kBM, 1};
+        if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    const int64_t q_rows = BT * s.h;
+    if (q_rows >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
+    {
+        const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)q_rows};
+        const uint64_t strides[1] = {(uint64_t)kD * 2};
+        const uint32_t box[2] = {64, 1};
+        if (!make_bf16_map(&mapQ, a.Q, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_bf16_map(&mapdO, a.dO, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    Params p;
+    p.u.B = s.B;
+    p.u.T = s.T;
+    p.u.h = s.h;
+    p.u.g = s.g;
+    p.u.k = s.k;
+    p.u.hpg = s.h / s.g;
+    p.u.W = 32 * (4 / s.k);
+    p.u.nwin = (s.T + kQT * p.u.W - 1) / (kQT * p.u.W);
+    p.u.nchunk = gqe_chunk_count(s.T);
+    p.idx = a.idx;
+    p.gate = a.gate;
+    p.head_offsets = a.head_offsets;
+    p.head_pos = a.head_pos;
+    p.head_chunk_offsets = a.head_chunk_offsets;
+    p.lse = lse;
+    p.dlt = delta;
+    p.dQ = a.dQ;
+    p.dK = a.dK;
+    p.dV = a.dV;
+    p.status = (uint32_t*)a.status;
+    p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    p.scale = 1.0f / sqrtf((float)kD);
+    p.q_rows = (int)q_rows;
+
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+    // 2. dQ
+    {
+        const size_t smem = sizeof(DqSmem) + 1024;
+        e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t items = p.u.count() * kQT;
+        const int grid = (int)(items < sms ? items : sms);
+        dq_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, mapdO, p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // 3. dK, dV
+    {
+        const size_t smem = sizeof(KvSmem) + 1024;
+        e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t items = (int64_t)s.B * s.g * ((s.T + kBM - 1) / kBM);
+        const int grid = (int)(items < sms ? items : sms);
+        dkdv_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, mapdO, p);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace gqe

@@ -80,7 +80,9 @@ struct Params {
     const int32_t* head_offsets;
     const int32_t* head_pos;
     const int32_t* head_chunk_offsets;
-    __nv_bfloat16* O;
+    __nv_bfloat16* O;   // gated bf16 output; null when the training outputs are asked for instead
+    float* o32;         // training: ungated fp32 output of every routed row, [B, T, h, 128]
+    float* lse;         // training: log2-sum-exp of every routed row's scaled scores, [B, T, h]
     uint32_t* status;
     float scale_log2;
     int q_rows;  // B*T*h: rows of Q viewed as [B*T*h, 128]
@@ -134,6 +136,7 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
 
 
 // ---------------------------------------------------------------------------
+template <bool kTrain>  // kTrain: write the training outputs (o32, lse) instead of O
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQB,
@@ -246,12 +249,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 }
                 umma_commit(&sm.s_full[t]);
             };
+            // For the training outputs P.V runs over [P | R] against V twice: R (in
+            // S's columns 64-127) holds p - bf16(p), so o is accurate far beyond
+            // bf16 P (the backward's D = g dO . o needs it).
+            constexpr bool train = kTrain;
             auto issue_pv = [&](int t, uint32_t it, bool first) {
                 const uint32_t b0 = (it & 1) ? vlo1 : vlo0;
                 const uint32_t d = tmem + kColO + t * 128, a = tmem + kColS + t * 128;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
                     umma_ts(d, a + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
+                if (train) {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        umma_ts(d, a + 64 + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, 1u);
+                }
             };
             auto wait_k = [&](uint32_t it) { return mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1); };
             auto wait_v = [&](uint32_t it) { return mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1); };
@@ -461,7 +473,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         // selections at once; the warp then zeroes the unselected 256-byte
         // slots, 16 lanes per slot.
         const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
-        for (int64_t j = 0;; ++j) {
+        for (int64_t j = 0; !kTrain; ++j) {  // the training outputs leave O alone
             const int64_t unit = cta_unit(j, n_units);
             if (unit < 0 || aborted(sm)) break;
             int b, q, w;
@@ -521,6 +533,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + kColS + t * 128;
         const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
+        constexpr bool train = kTrain;  // also write R = p - bf16(p) for the exact P.V
         uint32_t ctile = 0, u_it = 0;
         for (int64_t j = 0;; ++j, ++u_it) {
             const int64_t unit = cta_unit(j, n_units);
@@ -605,7 +618,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 if (need_mask) {
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t pk[16];
+                        uint32_t pk[16], rk[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             float x0, x1;
@@ -614,13 +627,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                             const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                             sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
                             pk[e] = pack_bf16x2(p0, p1);
+                            if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
+                                                           p1 - __uint_as_float(pk[e] & 0xffff0000u));
                         }
                         tmem_st16(s_addr + cb * 16, pk);
+                        if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
                     }
                 } else {
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t pk[16];
+                        uint32_t pk[16], rk[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const uint64_t x2 =
@@ -638,8 +654,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                             }
                             sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
                             pk[e] = pack_bf16x2(p0, p1);
+                            if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
+                                                           p1 - __uint_as_float(pk[e] & 0xffff0000u));
                         }
                         tmem_st16(s_addr + cb * 16, pk);
+                        if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
                     }
                 }
                 float sa, sb;
@@ -659,8 +678,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             }
             tc_fence_after();
             const int j_row = sm.row_j[rs][t][r];
+            const int64_t orow_idx = ((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row;
+            if (kTrain) {
+                // Training: the ungated output o = O_t / l in fp32 and the row's
+                // log2-sum-exp m + log2(l) (so that p_s = 2^(s_s * c - lse)).
+                const float inv = 1.0f / l;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cb * 32, o);
+                    ld_wait_bind(o);
+                    if (t_row >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(p.o32 + orow_idx * kD + cb * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                 __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                    }
+                }
+                if (t_row >= 0) p.lse[orow_idx] = m + log2f(l);
+                tc_fence_before();
+                mbar_arrive(&sm.o_empty[t]);
+                mbar_arrive(&sm.rows_free[rs]);
+                continue;
+            }
             const float f = (t_row >= 0) ? sm.row_gate[rs][t][r] / l : 0.f;
-            __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD;
+            __nv_bfloat16* orow = p.O + orow_idx * kD;
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t o[32];
@@ -709,10 +752,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     // launch (a property of the compiled kernel: checked once per process).
     static std::atomic<int> regs_checked{0};
     if (regs_checked.load(std::memory_order_acquire) == 0) {
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel);
+        cudaFuncAttributes fa, fb;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel<false>);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fb, prefill_tc_kernel<true>);
         if (e != cudaSuccess) return e;
-        regs_checked.store((fa.numRegs == kRegsLaunch) ? 1 : -1, std::memory_order_release);
+        regs_checked.store((fa.numRegs == kRegsLaunch && fb.numRegs == kRegsLaunch) ? 1 : -1,
+                           std::memory_order_release);
     }
     if (regs_checked.load(std::memory_order_acquire) != 1) return cudaErrorNotSupported;
 
@@ -748,6 +793,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     p.head_pos = a.head_pos;
     p.head_chunk_offsets = a.head_chunk_offsets;
     p.O = (__nv_bfloat16*)a.O;
+    p.o32 = a.o32;
+    p.lse = a.lse;
     p.status = (uint32_t*)a.status;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     p.q_rows = (int)q_rows;
@@ -759,7 +806,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     const int64_t units = u.count();
     const int grid = (int)(units < sms ? units : sms);
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool train = a.o32 != nullptr;
+    auto kern = train ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -771,7 +820,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_tc_kernel, mapK, mapV, mapQ, mapQB, p);
+    return cudaLaunchKernelEx(&cfg, kern, mapK, mapV, mapQ, mapQB, p);
 }
 
 }  // namespace gqe

@@ -163,7 +163,10 @@ def test_backward_dense_gqa_full_size():
                             ("dV suffix", dV[:, t0:], sv[:, t0:])):
         err = float(np.abs(got - want).max())
         assert err <= tol, f"{name}: max abs error {err}"
-    # softmax shift invariance: the score gradients of every row sum to zero
-    assert np.abs(dK.sum(axis=1)).max() <= 1e-2, "sum_s dK != 0"
+    # softmax shift invariance: the score gradients of every row sum to zero.  dK
+    # accumulates dS rounded to bf16 on the tensor cores, so each row's sum over
+    # its keys carries about 2^-9 |dS| sqrt(n) of rounding, and the invariant
+    # holds to the element tolerance, not tighter.
+    assert np.abs(dK.sum(axis=1)).max() <= tol, "sum_s dK != 0"
     # and every group's logit gradients sum to zero
     assert np.abs(dl.reshape(w.B, w.T, w.g, -1).sum(-1)).max() <= 1e-4
