@@ -430,10 +430,10 @@ def time_backward(w, steps, warmup, peaks, peak_kind):
     workload's shapes, after one forward step, timed alone with CUDA events (L2
     flushed before each call, outside the events).  Algorithmic FLOPs: the
     five contractions of an attention backward over the visible (row, key)
-    pairs of the routed rows, 2.5x the forward's 4*d_h per pair.  The kernels
-    run on the fp32 CUDA cores, so the roofline is the fp32 FMA peak (148 SMs x
-    128 lanes x 2 FLOP x the 1965 MHz SM clock), with the fraction of the bf16
-    tensor peak given beside it."""
+    pairs of the routed rows, 2.5x the forward's 4*d_h per pair.  bf16 inputs
+    with d_h = 128 run on the tensor cores (the roofline is the bf16 tensor
+    peak); other inputs run on the fp32 CUDA cores (the roofline is the fp32
+    FMA peak: 148 SMs x 128 lanes x 2 FLOP x the 1965 MHz SM clock)."""
     from routed_head_gqa_b200 import metrics
 
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -470,6 +470,7 @@ def time_backward(w, steps, warmup, peaks, peak_kind):
     flops = 2.5 * metrics.prefill_active_flops(w.B, w.T, w.g, w.k, w.d_h)
     tf = flops / (ms * 1e-3) * 1e-12
     alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 * 1e-12
+    tensor = w.dtype == "bf16" and w.d_h == 128 and w.k <= 4 and w.h // w.g <= 32
     el = 2 if w.dtype == "bf16" else 4
     BT = w.B * w.T
     # x read once per 32 heads and dx written (fp32); dlogits read twice; W_r, dW_r, dbias are small
@@ -477,12 +478,19 @@ def time_backward(w, steps, warmup, peaks, peak_kind):
     r_gbs = r_bytes / (rms * 1e-3) * 1e-9
     del r, flush
     torch.cuda.empty_cache()
-    return {"ms": ms, "value": tf, "unit": "TFLOP/s", "flops": flops, "launches": 3,
-            "roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(tf / alu_peak, 4),
-                         "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz (derived)",
-                         "frac_of_bf16_tensor": round(tf / peaks["bf16_tflops"], 4),
-                         "kernel": "gqe_attn_prefill_backward (bwd_dq_kernel + bwd_rows_kernel + bwd_dkdv_kernel)"},
+    if tensor:
+        roof = {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tf / peaks["bf16_tflops"], 4), "peak_source": f"bf16_tflops burst ({peak_kind})",
+                "kernel": "gqe_attn_prefill_backward (prefill_tc_kernel<train> + bwd_prep_kernel + "
+                          "bwd_tiles_kernel + dq_tc_kernel + dkdv_tc_kernel)"}
+    else:
+        roof = {"bound": "alu", "achieved": round(tf, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                "frac": round(tf / alu_peak, 4),
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x 1965 MHz (derived)",
+                "frac_of_bf16_tensor": round(tf / peaks["bf16_tflops"], 4),
+                "kernel": "gqe_attn_prefill_backward (bwd_dq_kernel + bwd_rows_kernel + bwd_dkdv_kernel)"}
+    return {"ms": ms, "value": tf, "unit": "TFLOP/s", "flops": flops, "launches": 5 if tensor else 3,
+            "roofline": roof,
             "router": {"ms": rms, "value": r_gbs, "unit": "GB/s", "bytes": r_bytes, "launches": 4,
                        "roofline": {"bound": "hbm", "achieved": round(r_gbs, 1), "peak": peaks["hbm_gbs"],
                                     "unit": "GB/s", "frac": round(r_gbs / peaks["hbm_gbs"], 4),

@@ -16,6 +16,10 @@
 // row's log2-sum-exp lse_r into the workspace, so p_rs = 2^(s_rs c - lse_r)):
 //  1. bwd_prep_kernel: one warp per (b, t, group): D_r, the gates, the logit
 //     gradients, and zero dQ rows for the unselected heads.
+//  1b. bwd_tiles_kernel: one warp per half-window tile of a group (the
+//     prefill's row tiles): the tile's row table (position, head, and per row
+//     lse, gate, D) and its Q and dO rows, packed contiguously in the workspace,
+//     so that the two tensor-core kernels load each tile with plain TMA boxes.
 //  2. dq_tc_kernel: per 128-row tile of routed rows (the prefill's half-window
 //     tiles): S = Q K^T and dP = dO V^T on the tensor cores, dS in registers,
 //     dQ += dS K accumulated in TMEM.
@@ -118,14 +122,26 @@ __device__ void build_rows(const UnitGeom& u, int b, int q, int w0, const int32_
     __syncwarp();
 }
 
-// Q and dO rows of a table by TMA gather (four rows per copy, two 64-column
-// halves), 128B-swizzled [128][64] boxes; padding rows are zero-filled.
-__device__ __forceinline__ void gather_rows(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, const RowTable& rt) {
+// A packed tile: per row (lse, gate, D, position t) in one 16-byte record
+// (t = -1 for padding) and the row's head, as the tensor-core kernels read them.
+struct RowRec {
+    float lse, gate, dlt;
+    int32_t t;
+};
+struct TileTab {
+    RowRec rec[kBM];
+    int32_t j[kBM];
+};
+
+// One warp copies a packed tile's table from the workspace into shared memory.
+__device__ __forceinline__ void load_tab(const RowRec* rec_g, const int32_t* j_g, TileTab& tt) {
     const int lane = threadIdx.x & 31;
-    const int r0 = lane * 4;
-    tma_gather4_2d(map, bar, dst + r0 * 128, 0, rt.qrow[r0], rt.qrow[r0 + 1], rt.qrow[r0 + 2], rt.qrow[r0 + 3]);
-    tma_gather4_2d(map, bar, dst + kHalf + r0 * 128, 64, rt.qrow[r0], rt.qrow[r0 + 1], rt.qrow[r0 + 2],
-                   rt.qrow[r0 + 3]);
+    const int4* src = reinterpret_cast<const int4*>(rec_g);
+    int4* dst = reinterpret_cast<int4*>(tt.rec);
+#pragma unroll
+    for (int i = 0; i < kBM / 32; ++i) dst[lane + 32 * i] = src[lane + 32 * i];
+#pragma unroll
+    for (int i = 0; i < kBM / 32; ++i) tt.j[lane + 32 * i] = j_g[lane + 32 * i];
 }
 
 // p = 2^(s c - lse) (0 where masked), pg = gate p, ds = p (gate dp - D), as
@@ -195,6 +211,52 @@ bwd_prep_kernel(int64_t BT, int h, int g, int k, const int32_t* __restrict__ idx
     }
 }
 
+// ------------------------------------------------------------------ 1b. packed tiles
+// Tile id (b*g + q) * ntiles + ti covers positions [ti*W, (ti+1)*W) of group q of
+// sequence b; one warp per tile (four per block).
+__global__ void __launch_bounds__(128)
+bwd_tiles_kernel(UnitGeom u, int ntiles, const int32_t* __restrict__ head_offsets,
+                 const int32_t* __restrict__ head_chunk_offsets, const int32_t* __restrict__ head_pos,
+                 const int32_t* __restrict__ idx, const float* __restrict__ gate, const float* __restrict__ lse,
+                 const float* __restrict__ dlt, const __nv_bfloat16* __restrict__ Q,
+                 const __nv_bfloat16* __restrict__ dO, RowRec* __restrict__ rec, int32_t* __restrict__ jtab,
+                 __nv_bfloat16* __restrict__ Qc, __nv_bfloat16* __restrict__ dOc, uint32_t* status) {
+    __shared__ RowTable rt[4];
+    __shared__ int32_t cut_start[4][32], cut_prefix[4][33];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tile = (int64_t)blockIdx.x * 4 + warp;
+    const int64_t n = (int64_t)u.B * u.g * ntiles;
+    if (tile >= n) return;
+    const int ti = (int)(tile % ntiles);
+    const int bq = (int)(tile / ntiles);
+    const int b = bq / u.g, q = bq % u.g;
+    RowTable& t = rt[warp];
+    build_rows(u, b, q, ti * u.W, head_offsets, head_chunk_offsets, head_pos, idx, gate, lse, dlt, -1, t,
+               cut_start[warp], cut_prefix[warp], status);
+    for (int r = lane; r < kBM; r += 32) {
+        RowRec x;
+        x.lse = t.lse[r];
+        x.gate = t.gate[r];
+        x.dlt = t.dlt[r];
+        x.t = t.t[r];
+        rec[tile * kBM + r] = x;
+        jtab[tile * kBM + r] = t.j[r];
+    }
+    // Q and dO rows: 16 lanes per 256-byte row, two rows per pass
+    const int half = lane >> 4, c = lane & 15;
+    for (int r0 = 0; r0 < kBM; r0 += 2) {
+        const int r = r0 + half;
+        const int32_t src = t.qrow[r];
+        uint4 qv = make_uint4(0, 0, 0, 0), dv = qv;
+        if (t.t[r] >= 0) {
+            qv = reinterpret_cast<const uint4*>(Q + (int64_t)src * kD)[c];
+            dv = reinterpret_cast<const uint4*>(dO + (int64_t)src * kD)[c];
+        }
+        reinterpret_cast<uint4*>(Qc + (tile * kBM + r) * kD)[c] = qv;
+        reinterpret_cast<uint4*>(dOc + (tile * kBM + r) * kD)[c] = dv;
+    }
+}
+
 // ------------------------------------------------------------------ shared pieces
 struct Params {
     UnitGeom u;
@@ -205,6 +267,9 @@ struct Params {
     const int32_t* head_chunk_offsets;
     const float* lse;
     const float* dlt;
+    const RowRec* rec;     // packed tile tables
+    const int32_t* jtab;
+    int ntiles;            // half-window tiles per (b, group): 2 * ceil(T / 2W)
     float* dQ;
     float* dK;
     float* dV;
@@ -224,7 +289,7 @@ __device__ __forceinline__ void fail(int32_t* abort_flag, uint32_t* status, uint
 // lse, gate, D and visibility.  Returns 16 packed pairs of pg and ds.
 template <bool KEY_ROWS>
 __device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float c, float lse_or_row,
-                                         float gate_row, float dlt_row, int key_or_t, const RowTable& rt, int col0,
+                                         float gate_row, float dlt_row, int key_or_t, const RowRec* recs, int col0,
                                          int kv0, uint32_t (&pg)[16], uint32_t (&ds)[16]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -235,11 +300,11 @@ __device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t
             float lse, gm, dl;
             bool vis;
             if (KEY_ROWS) {  // thread = key (global index key_or_t), column = row cc of the table
-                lse = rt.lse[cc];
-                gm = rt.gate[cc];
-                dl = rt.dlt[cc];
-                const int tr = rt.t[cc];
-                vis = tr >= 0 && key_or_t <= tr;
+                const RowRec x = recs[cc];  // one 16-byte shared-memory broadcast
+                lse = x.lse;
+                gm = x.gate;
+                dl = x.dlt;
+                vis = x.t >= 0 && key_or_t <= x.t;
             } else {         // thread = row (position key_or_t), column = key kv0 + cc
                 lse = lse_or_row;
                 gm = gate_row;
@@ -267,9 +332,7 @@ struct DqSmem {
     uint8_t dO[kTile];
     uint8_t k[2][kTile];
     uint8_t v[2][kTile];
-    RowTable rt;
-    int32_t cut_start[32];
-    int32_t cut_prefix[33];
+    TileTab tab;
     uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
     uint64_t rows_full, rows_empty, s_full[2], dp_full, ew_done, dq_full, dq_empty, drain;
     uint32_t tmem_base;
@@ -278,18 +341,20 @@ struct DqSmem {
 
 __device__ __forceinline__ int dq_items(const UnitGeom& u) { return (int)(u.count() * kQT); }
 // Item i: heaviest windows first (unit order of the prefill), two halves per unit.
-__device__ __forceinline__ void dq_item(const UnitGeom& u, int64_t i, int& b, int& q, int& w0, int& nkv) {
+__device__ __forceinline__ void dq_item(const UnitGeom& u, int ntiles, int64_t i, int& b, int& q, int& w0, int& nkv,
+                                        int64_t& tile) {
     int w;
     unit_coords(u, i / kQT, b, q, w);
     const int half = (int)(i % kQT);
     w0 = (w * kQT + half) * u.W;
     const int end = min(w0 + u.W, u.T);
     nkv = (end + kBM - 1) / kBM;
+    tile = ((int64_t)b * u.g + q) * ntiles + (w * kQT + half);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-             const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO, const Params p) {
+             const __grid_constant__ CUtensorMap mapQc, const __grid_constant__ CUtensorMap mapdOc, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     DqSmem& sm = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -329,7 +394,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             bool ok = true;
             for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
                 int b, q, w0, nkv;
-                dq_item(u, it, b, q, w0, nkv);
+                int64_t tile;
+                dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
                 for (int i = 0; i < nkv; ++i, ++kv) {
                     const int st = kv & 1;
                     const uint32_t par = ((kv >> 1) & 1) ^ 1;
@@ -396,7 +462,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             bool ok = true;
             for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
                 int b, q, w0, nkv;
-                dq_item(u, it, b, q, w0, nkv);
+                int64_t tile;
+                dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
                 if (!mbar_wait(&sm.rows_full, item_no & 1)) { fail(&sm.abort_flag, p.status, 10); break; }
                 tc_fence_after();
                 // prologue: S(0), dP(0), S(1)
@@ -454,18 +521,23 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         bool armed = false;
         for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
             int b, q, w0, nkv;
-            dq_item(u, it, b, q, w0, nkv);
+            int64_t tile;
+            dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
             // the previous item's operands and table are free
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_empty, (item_no & 1) ^ 1))) {
                 if (lane == 0) fail(&sm.abort_flag, p.status, 20);
                 break;
             }
-            build_rows(u, b, q, w0, p.head_offsets, p.head_chunk_offsets, p.head_pos, p.idx, p.gate, p.lse, p.dlt,
-                       p.q_rows, sm.rt, sm.cut_start, sm.cut_prefix, p.status);
-            if (lane == 0) mbar_arrive_expect_tx(&sm.rows_full, 2 * kTile);
+            load_tab(p.rec + tile * kBM, p.jtab + tile * kBM, sm.tab);
             __syncwarp();
-            gather_rows(&mapQ, &sm.rows_full, sm.q, sm.rt);
-            gather_rows(&mapdO, &sm.rows_full, sm.dO, sm.rt);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.rows_full, 2 * kTile);
+                const int row0 = (int)(tile * kBM);
+                tma_load_2d(&mapQc, &sm.rows_full, sm.q, 0, row0);
+                tma_load_2d(&mapQc, &sm.rows_full, sm.q + kHalf, 64, row0);
+                tma_load_2d(&mapdOc, &sm.rows_full, sm.dO, 0, row0);
+                tma_load_2d(&mapdOc, &sm.rows_full, sm.dO + kHalf, 64, row0);
+            }
             armed = true;
         }
         if (armed) mbar_wait(&sm.rows_full, (item_no - 1) & 1);
@@ -477,14 +549,16 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         uint32_t sc = 0, item_no = 0;
         for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
             int b, q, w0, nkv;
-            dq_item(u, it, b, q, w0, nkv);
+            int64_t tile;
+            dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_full, item_no & 1))) {
                 if (lane == 0) fail(&sm.abort_flag, p.status, 30);
                 break;
             }
-            const int t_row = sm.rt.t[r];
-            const float lse = sm.rt.lse[r], gm = sm.rt.gate[r], dl = sm.rt.dlt[r];
-            const int j_row = sm.rt.j[r];
+            const RowRec rr = sm.tab.rec[r];
+            const int t_row = rr.t;
+            const float lse = rr.lse, gm = rr.gate, dl = rr.dlt;
+            const int j_row = sm.tab.j[r];
             bool ok = true;
             for (int i = 0; i < nkv; ++i, ++sc) {
                 const uint32_t sb = sc & 1;
@@ -505,8 +579,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                         tmem_ld32(s_addr + hh * 64 + cb * 32, sv);
                         tmem_ld32(d_addr + hh * 64 + cb * 32, dv);
                         tmem_ld_wait();
-                        ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.rt, hh * 64 + cb * 32, i * kBM,
-                                        pg[cb], ds[cb]);
+                        ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.tab.rec, hh * 64 + cb * 32,
+                                        i * kBM, pg[cb], ds[cb]);
                     }
                     tmem_st16(d_addr + hh * 32, ds[0]);
                     tmem_st16(d_addr + hh * 32 + 16, ds[1]);
@@ -522,13 +596,16 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
-            float* drow = p.dQ + (((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row) * kD;
+            // a table entry outside [0, T) x group q's heads is reported, not written
+            const bool row_ok = t_row >= 0 && t_row < u.T && j_row >= q * u.hpg && j_row < (q + 1) * u.hpg;
+            if (t_row >= 0 && !row_ok) report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 4);
+            float* drow = p.dQ + (((int64_t)b * u.T + (row_ok ? t_row : 0)) * u.h + (row_ok ? j_row : 0)) * kD;
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_off + 384 + cb * 32, o);
                 tmem_ld_wait();
-                if (t_row >= 0) {
+                if (row_ok) {
                     float4* dst = reinterpret_cast<float4*>(drow + cb * 32);
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
@@ -564,9 +641,7 @@ struct KvSmem {
     uint8_t v[kTile];
     uint8_t q[2][kTile];
     uint8_t dO[2][kTile];
-    RowTable rt[2];
-    int32_t cut_start[32];
-    int32_t cut_prefix[33];
+    TileTab tab[2];
     uint64_t kv_full, kv_empty, rows_full[2], rows_empty[2], st_full, ew_done, acc_full, acc_empty, drain;
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -588,7 +663,7 @@ __device__ __forceinline__ void kv_item(const UnitGeom& u, int64_t i, int& b, in
 
 __global__ void __launch_bounds__(kThreads, 1)
 dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-               const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO, const Params p) {
+               const __grid_constant__ CUtensorMap mapQc, const __grid_constant__ CUtensorMap mapdOc, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     KvSmem& sm = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -703,13 +778,17 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     ok = false;
                     break;
                 }
-                const int w0 = (tile0 + i) * u.W;
-                build_rows(u, b, q, w0, p.head_offsets, p.head_chunk_offsets, p.head_pos, p.idx, p.gate, p.lse,
-                           p.dlt, p.q_rows, sm.rt[rb], sm.cut_start, sm.cut_prefix, p.status);
-                if (lane == 0) mbar_arrive_expect_tx(&sm.rows_full[rb], 2 * kTile);
+                const int64_t tile = ((int64_t)b * u.g + q) * p.ntiles + (tile0 + i);
+                load_tab(p.rec + tile * kBM, p.jtab + tile * kBM, sm.tab[rb]);
                 __syncwarp();
-                gather_rows(&mapQ, &sm.rows_full[rb], sm.q[rb], sm.rt[rb]);
-                gather_rows(&mapdO, &sm.rows_full[rb], sm.dO[rb], sm.rt[rb]);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.rows_full[rb], 2 * kTile);
+                    const int row0 = (int)(tile * kBM);
+                    tma_load_2d(&mapQc, &sm.rows_full[rb], sm.q[rb], 0, row0);
+                    tma_load_2d(&mapQc, &sm.rows_full[rb], sm.q[rb] + kHalf, 64, row0);
+                    tma_load_2d(&mapdOc, &sm.rows_full[rb], sm.dO[rb], 0, row0);
+                    tma_load_2d(&mapdOc, &sm.rows_full[rb], sm.dO[rb] + kHalf, 64, row0);
+                }
                 armed = rc;
             }
             if (!ok) break;
@@ -735,7 +814,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     break;
                 }
                 tc_fence_after();
-                const RowTable& rt = sm.rt[rb];
+                const RowRec* recs = sm.tab[rb].rec;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t pg[2][16], ds[2][16];
@@ -745,7 +824,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                         tmem_ld32(st_addr + hh * 64 + cb * 32, sv);
                         tmem_ld32(dpt_addr + hh * 64 + cb * 32, dv);
                         tmem_ld_wait();
-                        ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, rt, hh * 64 + cb * 32, 0, pg[cb],
+                        ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, recs, hh * 64 + cb * 32, 0, pg[cb],
                                        ds[cb]);
                     }
                     tmem_st16(st_addr + hh * 32, pg[0]);
@@ -806,19 +885,49 @@ bool attn_backward_tc_supported(const gqe_shape* s) {
     return s->dtype == GQE_BF16 && s->d_h == kD && s->k <= 4 && s->h / s->g <= 32;
 }
 
-size_t attn_backward_tc_scratch_bytes(const gqe_shape* s) {
+namespace {
+// Workspace of the tensor-core backward: gate, D and lse planes [B*T*h] (fp32),
+// o [B*T*h, 128] (fp32), then the packed tiles: records and heads
+// [tiles * 128] and the rows of Q and dO [tiles * 128, 128] (bf16).
+struct BwdLayout {
+    size_t plane, o32, rec, jtab, rows, total;
+    int64_t ntiles, tiles;
+};
+BwdLayout bwd_layout(const gqe_shape* s) {
+    BwdLayout L;
     const size_t bth = (size_t)s->B * s->T * s->h;
-    return 3 * a256(bth * sizeof(float)) + a256(bth * kD * sizeof(float));
+    const int W = 32 * (4 / s->k);
+    // every half of every 2W-position window, as the prefill's units and the dQ
+    // items name them (the last window's second half may lie past T: empty)
+    L.ntiles = 2 * (int64_t)((s->T + 2 * W - 1) / (2 * W));
+    L.tiles = (int64_t)s->B * s->g * L.ntiles;
+    L.plane = a256(bth * sizeof(float));
+    L.o32 = a256(bth * kD * sizeof(float));
+    L.rec = a256((size_t)L.tiles * kBM * sizeof(RowRec));
+    L.jtab = a256((size_t)L.tiles * kBM * sizeof(int32_t));
+    L.rows = a256((size_t)L.tiles * kBM * kD * 2);
+    L.total = 3 * L.plane + L.o32 + L.rec + L.jtab + 2 * L.rows;
+    return L;
 }
+}  // namespace
+
+size_t attn_backward_tc_scratch_bytes(const gqe_shape* s) { return bwd_layout(s).total; }
 
 cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     const gqe_shape& s = *a.s;
     const int64_t BT = (int64_t)s.B * s.T;
-    const size_t plane = a256((size_t)BT * s.h * sizeof(float));
-    float* gamma = static_cast<float*>(a.scratch);
-    float* delta = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + plane);
-    float* lse = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + 2 * plane);
-    float* o32 = reinterpret_cast<float*>(static_cast<char*>(a.scratch) + 3 * plane);
+    const BwdLayout L = bwd_layout(a.s);
+    char* base = static_cast<char*>(a.scratch);
+    float* gamma = reinterpret_cast<float*>(base);
+    float* delta = reinterpret_cast<float*>(base + L.plane);
+    float* lse = reinterpret_cast<float*>(base + 2 * L.plane);
+    float* o32 = reinterpret_cast<float*>(base + 3 * L.plane);
+    RowRec* rec = reinterpret_cast<RowRec*>(base + 3 * L.plane + L.o32);
+    int32_t* jtab = reinterpret_cast<int32_t*>(base + 3 * L.plane + L.o32 + L.rec);
+    __nv_bfloat16* Qc = reinterpret_cast<__nv_bfloat16*>(base + 3 * L.plane + L.o32 + L.rec + L.jtab);
+    __nv_bfloat16* dOc = reinterpret_cast<__nv_bfloat16*>(base + 3 * L.plane + L.o32 + L.rec + L.jtab + L.rows);
+    const int64_t rows_total = L.tiles * kBM;
+    if (rows_total >= ((int64_t)1 << 31) - 1 || BT * s.h >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
 
     // 0. the forward again, writing o and the log2-sum-exp of every routed row
     PrefillArgs f;
@@ -849,25 +958,6 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    // tensor maps: K, V as [B, T, g, 128] (128-key boxes of 64 columns); Q, dO as
-    // [B*T*h, 128] rows (one-row boxes for the gathers)
-    CUtensorMap mapK, mapV, mapQ, mapdO;
-    {
-        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
-        const uint32_t box[4] = {64, 1, (uint32_t)kBM, 1};
-        if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
-        if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
-    }
-    const int64_t q_rows = BT * s.h;
-    if (q_rows >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
-    {
-        const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)q_rows};
-        const uint64_t strides[1] = {(uint64_t)kD * 2};
-        const uint32_t box[2] = {64, 1};
-        if (!make_bf16_map(&mapQ, a.Q, 2, dims, strides, box)) return cudaErrorInvalidValue;
-        if (!make_bf16_map(&mapdO, a.dO, 2, dims, strides, box)) return cudaErrorInvalidValue;
-    }
     Params p;
     p.u.B = s.B;
     p.u.T = s.T;
@@ -885,13 +975,41 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     p.head_chunk_offsets = a.head_chunk_offsets;
     p.lse = lse;
     p.dlt = delta;
+    p.rec = rec;
+    p.jtab = jtab;
+    p.ntiles = (int)L.ntiles;
     p.dQ = a.dQ;
     p.dK = a.dK;
     p.dV = a.dV;
     p.status = (uint32_t*)a.status;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     p.scale = 1.0f / sqrtf((float)kD);
-    p.q_rows = (int)q_rows;
+    p.q_rows = (int)(BT * s.h);
+
+    // 1b. packed tiles (tables, Q and dO rows)
+    bwd_tiles_kernel<<<(unsigned)((L.tiles + 3) / 4), 128, 0, a.stream>>>(
+        p.u, p.ntiles, a.head_offsets, a.head_chunk_offsets, a.head_pos, a.idx, a.gate, lse, delta,
+        (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.dO, rec, jtab, Qc, dOc, (uint32_t*)a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // tensor maps: K, V as [B, T, g, 128] (128-key boxes of 64 columns); the
+    // packed rows of Q and dO as [tiles * 128, 128] (128-row boxes)
+    CUtensorMap mapK, mapV, mapQc, mapdOc;
+    {
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.g, (uint64_t)s.T, (uint64_t)s.B};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.g * kD * 2, (uint64_t)s.T * s.g * kD * 2};
+        const uint32_t box[4] = {64, 1, (uint32_t)kBM, 1};
+        if (!make_bf16_map(&mapK, a.K, 4, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_bf16_map(&mapV, a.V, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kD, (uint64_t)rows_total};
+        const uint64_t strides[1] = {(uint64_t)kD * 2};
+        const uint32_t box[2] = {64, (uint32_t)kBM};
+        if (!make_bf16_map(&mapQc, Qc, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_bf16_map(&mapdOc, dOc, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -904,7 +1022,7 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
         if (e != cudaSuccess) return e;
         const int64_t items = p.u.count() * kQT;
         const int grid = (int)(items < sms ? items : sms);
-        dq_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, mapdO, p);
+        dq_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQc, mapdOc, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -915,7 +1033,7 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
         if (e != cudaSuccess) return e;
         const int64_t items = (int64_t)s.B * s.g * ((s.T + kBM - 1) / kBM);
         const int grid = (int)(items < sms ? items : sms);
-        dkdv_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQ, mapdO, p);
+        dkdv_tc_kernel<<<grid, kThreads, smem, a.stream>>>(mapK, mapV, mapQc, mapdOc, p);
         e = cudaGetLastError();
     }
     return e;
