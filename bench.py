@@ -41,7 +41,7 @@ import gqe_synth  # noqa: E402
 
 PRIMARY = "gqe_prefill"
 # Every config, in order, in the line's compact "configs" map (the primary included).
-CONFIG_ORDER = ["tiny_f32", "dense_gqa", "gqe_prefill", "gqe_long", "gqe_decode"]
+CONFIG_ORDER = ["tiny_f32", "dense_gqa", "gqe_prefill", "gqe_long", "gqe_decode", "gqe_32k"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch of the dominant kernels, from `ncu` captures

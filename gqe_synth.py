@@ -18,6 +18,8 @@ Workloads (sizes, distributions and skews of the GQE prefill/decode cases):
   gqe_decode    B=64 one query token, cache lengths uniform in [1024, 16384],
                 Lmax=16384, h=32 g=8 d_h=128 d_model=4096 k=2 bf16,
                 W_r std 1/64, caches [B, Lmax, g, d_h]
+  gqe_32k       B=1  T=32768 d_model=2048 h=16 g=8 d_h=128 k=1 bf16,
+                W_r std 1/sqrt(2048) (a long-context case beyond the five)
 
 Recipe: one CPU ``torch.Generator`` seeded with the workload's seed draws, in
 this order, lengths (decode only), x, W_r, Q, K, V as fp32 standard normals
@@ -76,6 +78,9 @@ WORKLOADS = {
                          head0_bias=1.0, seed=3),
     "gqe_decode": Workload("gqe_decode", 64, 1, 4096, 32, 8, 128, 2, "bf16", 1.0 / 64, decode=True,
                            Lmin=1024, Lmax=16384, seed=4),
+    # Beyond the five configs: a 32k-token prefill with the GQE summary's main head
+    # layout (16 query heads, 8 KV groups, k = 1), near-uniform router.
+    "gqe_32k": Workload("gqe_32k", 1, 32768, 2048, 16, 8, 128, 1, "bf16", 1.0 / math.sqrt(2048), seed=5),
 }
 
 

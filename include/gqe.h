@@ -357,6 +357,42 @@ gqe_status gqe_route_backward(const gqe_shape* s, const void* x, const void* W_r
                               float* dW_r, float* dbias, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gqe_attn_prefill_train -- gqe_attn_prefill for training: besides the gated
+ * output O it saves, for every routed row (b, t, j), what the backward needs
+ * (the chain rule through the forward; the pages give no backward):
+ *   O32 [B, T, h, 128]   device fp32 out: the ungated attention output o of the
+ *                        row (O = gate * o), computed so that the rounding of
+ *                        the bf16 softmax weights does not reach it (P.V also
+ *                        runs over p - bf16(p)); unselected slots untouched
+ *   lse [B, T, h]        device fp32 out: log2 of the row's softmax
+ *                        denominator in units of the scaled scores, so that the
+ *                        weight of key s is 2^(q.k_s log2(e)/sqrt(128) - lse);
+ *                        unselected slots untouched
+ *   O                    as for gqe_attn_prefill, or NULL to skip it
+ * Other arguments as gqe_attn_prefill.  Implemented for bf16 with d_h = 128,
+ * k <= 4 and h/g <= 32 (the tensor-core path); other shapes return
+ * GQE_ERR_UNSUPPORTED.
+ */
+gqe_status gqe_attn_prefill_train(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                  const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                  const int32_t* head_pos, const int32_t* head_chunk_offsets, void* O, float* O32,
+                                  float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_attn_prefill_backward_saved -- gqe_attn_prefill_backward from the
+ * statistics gqe_attn_prefill_train saved (O32, lse, as written there) instead
+ * of running the forward again.  Same results, arguments, workspace and
+ * errors as gqe_attn_prefill_backward, plus O32 and lse (device, read only);
+ * the same shape limits as gqe_attn_prefill_train.
+ */
+gqe_status gqe_attn_prefill_backward_saved(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                           const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                           const int32_t* head_pos, const int32_t* head_chunk_offsets,
+                                           const void* dO, const float* O32, const float* lse, float* dQ, float* dK,
+                                           float* dV, float* dlogits, void* workspace, size_t workspace_bytes,
+                                           void* stream);
+
+/*
  * gqe_route_train -- gqe_route that also writes the router's fp32 logits, for
  * training: the load-balancing loss (gqe_aux_loss) and the router's own
  * gradient path read them.  Arguments and results are those of gqe_route, plus

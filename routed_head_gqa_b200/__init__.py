@@ -31,6 +31,7 @@ EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
             "gqe_group_slots", "gqe_routed_qproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
             "gqe_route_backward", "gqe_route_train", "gqe_aux_loss_workspace_bytes", "gqe_aux_loss",
+            "gqe_attn_prefill_train", "gqe_attn_prefill_backward_saved",
             "gqe_get_device_status", "gqe_status_string"]
 
 
@@ -82,6 +83,8 @@ def _load():
     lib.gqe_aux_loss_workspace_bytes.argtypes = [S]
     lib.gqe_aux_loss_workspace_bytes.restype = _SZ
     lib.gqe_aux_loss.argtypes = [S, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_attn_prefill_train.argtypes = [S] + [_P] * 12 + [_SZ, _P]
+    lib.gqe_attn_prefill_backward_saved.argtypes = [S] + [_P] * 16 + [_SZ, _P]
     lib.gqe_get_device_status.argtypes = [_P, _P]
     lib.gqe_status_string.argtypes = [_I]
     lib.gqe_status_string.restype = ctypes.c_char_p
@@ -89,7 +92,7 @@ def _load():
               "gqe_attn_prefill", "gqe_attn_decode",
               "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
               "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status", "gqe_route_train",
-              "gqe_aux_loss"):
+              "gqe_aux_loss", "gqe_attn_prefill_train", "gqe_attn_prefill_backward_saved"):
         getattr(lib, f).restype = _I
     _lib_handle = lib
     return lib
@@ -241,6 +244,23 @@ def gqe_route_train(shape, x, W_r, bias, idx, gate, head_offsets, head_pos, head
                                                    _ptr(gate), _ptr(head_offsets), _ptr(head_pos),
                                                    _ptr(head_chunk_offsets), _ptr(logits), _ptr(workspace),
                                                    _nbytes(workspace), _stream(stream)))
+
+
+def gqe_attn_prefill_train(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, O, O32, lse,
+                           workspace, stream=None) -> None:
+    _check("gqe_attn_prefill_train",
+           _lib.gqe_attn_prefill_train(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(gate),
+                                       _ptr(head_offsets), _ptr(head_pos), _ptr(head_chunk_offsets), _ptr(O),
+                                       _ptr(O32), _ptr(lse), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def gqe_attn_prefill_backward_saved(shape, Q, K, V, idx, gate, head_offsets, head_pos, head_chunk_offsets, dO, O32,
+                                    lse, dQ, dK, dV, dlogits, workspace, stream=None) -> None:
+    _check("gqe_attn_prefill_backward_saved",
+           _lib.gqe_attn_prefill_backward_saved(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(gate),
+                                                _ptr(head_offsets), _ptr(head_pos), _ptr(head_chunk_offsets), _ptr(dO),
+                                                _ptr(O32), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dlogits),
+                                                _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def gqe_aux_loss_workspace_bytes(shape) -> int:

@@ -23,6 +23,10 @@ struct AttnBwdArgs {
     void* scratch;   // attn_backward_scratch_bytes(s) bytes, 256-byte aligned
     void* status;
     cudaStream_t stream;
+    // Saved by the training forward (tensor-core path): each routed row's
+    // ungated fp32 output and log2-sum-exp.  Null: the backward recomputes them.
+    const float* o32 = nullptr;
+    const float* lse = nullptr;
 };
 
 // Per-(b,t,j) scratch of the backward: gate, D = dO.O and the row's log2-sum-exp

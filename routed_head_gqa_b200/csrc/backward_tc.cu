@@ -41,13 +41,20 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kBM = 128;                   // rows (or keys) per tile
-constexpr int kThreads = 256;              // 8 warps
+constexpr int kThreads = 384;              // 4 control warps + 8 elementwise warps
 constexpr uint32_t kHalf = 128 * 64 * 2;   // [128][64] bf16 box, 16 KB
 constexpr uint32_t kTile = 2 * kHalf;      // [128][128] bf16, 32 KB
 constexpr uint32_t kWhereBwdTc = 9;
 constexpr int kQT = 2;                     // half-window tiles per window
 
 __device__ __forceinline__ bool aborted(const int32_t* flag) { return *((volatile const int32_t*)flag) != 0; }
+
+// Two elementwise warps share each TMEM lane quarter, one per 64-column half
+// [64hh, 64hh + 64) of a 128-column tile.  Each writes its bf16 pairs over the
+// first 32 columns of its own half, so the MMA's TMEM operand for K step kk
+// (16 elements = 8 columns) sits at column a_col(kk), and neither warp writes
+// a column the other reads.
+__device__ __forceinline__ uint32_t a_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 
 // ------------------------------------------------------------------ row tables
 // The routed rows of one half-window tile (b, group q, first position w0, W
@@ -324,9 +331,10 @@ __device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t
 // ------------------------------------------------------------------ 2. dQ
 // One CTA per SM; work item = one half-window tile of 128 routed rows.
 // Roles: warp 0 K/V producer (2-stage ring), warp 1 MMA issuer, warp 2 row
-// table + Q/dO gather, warps 4-7 elementwise + epilogue (thread = row).
-// TMEM: S buffers [0,128) and [128,256), dP [256,384), dQ [384,512); dS
-// (bf16 pairs) overwrites the first 64 columns of dP once dP is in registers.
+// table + Q/dO gather, warps 4-11 elementwise + epilogue (thread = row, two
+// warps per row, one per 64-column half).  TMEM: S buffers [0,128) and
+// [128,256), dP [256,384), dQ [384,512); dS (bf16 pairs) overwrites dP's
+// columns a_col(0..7) once dP is in registers.
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dO[kTile];
@@ -371,9 +379,9 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         mbar_init(&sm.rows_full, 1);
         mbar_init(&sm.rows_empty, 2);  // the MMA issuer (operands read) and the elementwise warps (table read)
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.ew_done, 128);
+        mbar_init(&sm.ew_done, 256);
         mbar_init(&sm.dq_full, 1);
-        mbar_init(&sm.dq_empty, 128);
+        mbar_init(&sm.dq_empty, 256);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -448,12 +456,12 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 }
                 umma_commit(&sm.dp_full);
             };
-            // dQ (+)= dS . K (dS bf16 pairs in dP's first 64 columns; K MN-major).
+            // dQ (+)= dS . K (dS bf16 pairs in dP's columns a_col(kk); K MN-major).
             auto issue_dq = [&](uint32_t kvi, bool first) {
                 const uint32_t kb = (kvi & 1) ? kmlo1 : kmlo0;
 #pragma unroll
                 for (int kk = 0; kk < kBM / 16; ++kk)
-                    umma_ts(c_dq, c_dp + kk * 8, desc(kb + (uint32_t)((kk * 2048) >> 4)), idesc_dq,
+                    umma_ts(c_dq, c_dp + a_col(kk), desc(kb + (uint32_t)((kk * 2048) >> 4)), idesc_dq,
                             (first && kk == 0) ? 0u : 1u);
             };
             auto wait_k = [&](uint32_t x) { return mbar_wait(&sm.kv_full_k[x & 1], (x >> 1) & 1); };
@@ -543,7 +551,9 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         if (armed) mbar_wait(&sm.rows_full, (item_no - 1) & 1);
     } else if (warp >= 4) {
         // ------------------------------------------------------------ elementwise + epilogue (thread = row)
+        // Warps 4-7 take columns 0-63 of their rows, warps 8-11 columns 64-127.
         const int wq = warp & 3;
+        const int hh = (warp - 4) >> 2;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         uint32_t sc = 0, item_no = 0;
@@ -570,20 +580,16 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 }
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_off + sb * 128, d_addr = tmem + lane_off + 256;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {  // two 64-column halves; dS of half hh goes to columns 32hh..
-                    uint32_t pg[2][16], ds[2][16];
 #pragma unroll
-                    for (int cb = 0; cb < 2; ++cb) {
-                        uint32_t sv[32], dv[32];
-                        tmem_ld32(s_addr + hh * 64 + cb * 32, sv);
-                        tmem_ld32(d_addr + hh * 64 + cb * 32, dv);
-                        tmem_ld_wait();
-                        ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.tab.rec, hh * 64 + cb * 32,
-                                        i * kBM, pg[cb], ds[cb]);
-                    }
-                    tmem_st16(d_addr + hh * 32, ds[0]);
-                    tmem_st16(d_addr + hh * 32 + 16, ds[1]);
+                for (int cb = 0; cb < 2; ++cb) {
+                    // chunk cb's bf16 pairs land on columns this warp has already read
+                    uint32_t sv[32], dv[32], pg[16], ds[16];
+                    tmem_ld32(s_addr + hh * 64 + cb * 32, sv);
+                    tmem_ld32(d_addr + hh * 64 + cb * 32, dv);
+                    tmem_ld_wait();
+                    ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.tab.rec, hh * 64 + cb * 32, i * kBM,
+                                    pg, ds);
+                    tmem_st16(d_addr + hh * 64 + cb * 16, ds);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -601,7 +607,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             if (t_row >= 0 && !row_ok) report_error(p.status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 4);
             float* drow = p.dQ + (((int64_t)b * u.T + (row_ok ? t_row : 0)) * u.h + (row_ok ? j_row : 0)) * kD;
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 2 * hh; cb < 2 * hh + 2; ++cb) {  // this warp's 64 columns
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_off + 384 + cb * 32, o);
                 tmem_ld_wait();
@@ -616,8 +622,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             }
             tc_fence_before();
             mbar_arrive(&sm.dq_empty);
-            if (wq == 0 && lane == 0) mbar_arrive(&sm.rows_empty);  // this item's table is no longer read
-            // (the table is read until here; the MMA issuer's rows_empty commit covers the operands)
+            if (warp == 4 && lane == 0) mbar_arrive(&sm.rows_empty);  // this item's table is no longer read
+            // (the MMA issuer's rows_empty commit follows every elementwise step of the item)
         }
     }
     __syncwarp();
@@ -633,9 +639,10 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
 // Work item = (b, group q, 128-key tile kt), heaviest (earliest keys) first.
 // Its rows are the group's half-window tiles from the one holding key 128*kt
 // on.  Roles: warp 0 K/V of the item, warp 1 MMA issuer, warp 2 row tables +
-// Q/dO gather (double buffered), warps 4-7 elementwise + epilogue (thread =
-// key).  TMEM: dK [0,128), dV [128,256), S^T [256,384), dP^T [384,512); g p
-// and dS (bf16 pairs) overwrite the first 64 columns of S^T and dP^T.
+// Q/dO gather (double buffered), warps 4-11 elementwise + epilogue (thread =
+// key, two warps per key, one per 64-column half).  TMEM: dK [0,128), dV
+// [128,256), S^T [256,384), dP^T [384,512); g p and dS (bf16 pairs) overwrite
+// the columns a_col(0..7) of S^T and dP^T.
 struct KvSmem {
     uint8_t k[kTile];
     uint8_t v[kTile];
@@ -677,9 +684,9 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             mbar_init(&sm.rows_empty[i], 2);  // MMA issuer (operands) and elementwise warps (table)
         }
         mbar_init(&sm.st_full, 1);
-        mbar_init(&sm.ew_done, 128);
+        mbar_init(&sm.ew_done, 256);
         mbar_init(&sm.acc_full, 1);
-        mbar_init(&sm.acc_empty, 128);
+        mbar_init(&sm.acc_empty, 256);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -751,8 +758,8 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
 #pragma unroll
                     for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += (g p)^T . dO ; dK += dS^T . Q
                         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                        umma_ts(c_dv, c_st + kk * 8, desc(domb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
-                        umma_ts(c_dk, c_dpt + kk * 8, desc(qmb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
+                        umma_ts(c_dv, c_st + a_col(kk), desc(domb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
+                        umma_ts(c_dk, c_dpt + a_col(kk), desc(qmb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
                     }
                     umma_commit(&sm.rows_empty[rb]);
                 }
@@ -796,7 +803,9 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         if (armed >= 0) mbar_wait(&sm.rows_full[armed & 1], (armed >> 1) & 1);
     } else if (warp >= 4) {
         // ------------------------------------------------------------ elementwise + epilogue (thread = key)
+        // Warps 4-7 take columns (rows of the tile) 0-63, warps 8-11 columns 64-127.
         const int wq = warp & 3;
+        const int hh = (warp - 4) >> 2;
         const int kr = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t st_addr = tmem + lane_off + 256, dpt_addr = tmem + lane_off + 384;
@@ -815,27 +824,21 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 }
                 tc_fence_after();
                 const RowRec* recs = sm.tab[rb].rec;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t pg[2][16], ds[2][16];
 #pragma unroll
-                    for (int cb = 0; cb < 2; ++cb) {
-                        uint32_t sv[32], dv[32];
-                        tmem_ld32(st_addr + hh * 64 + cb * 32, sv);
-                        tmem_ld32(dpt_addr + hh * 64 + cb * 32, dv);
-                        tmem_ld_wait();
-                        ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, recs, hh * 64 + cb * 32, 0, pg[cb],
-                                       ds[cb]);
-                    }
-                    tmem_st16(st_addr + hh * 32, pg[0]);
-                    tmem_st16(st_addr + hh * 32 + 16, pg[1]);
-                    tmem_st16(dpt_addr + hh * 32, ds[0]);
-                    tmem_st16(dpt_addr + hh * 32 + 16, ds[1]);
+                for (int cb = 0; cb < 2; ++cb) {
+                    // chunk cb's bf16 pairs land on columns this warp has already read
+                    uint32_t sv[32], dv[32], pg[16], ds[16];
+                    tmem_ld32(st_addr + hh * 64 + cb * 32, sv);
+                    tmem_ld32(dpt_addr + hh * 64 + cb * 32, dv);
+                    tmem_ld_wait();
+                    ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, recs, hh * 64 + cb * 32, 0, pg, ds);
+                    tmem_st16(st_addr + hh * 64 + cb * 16, pg);
+                    tmem_st16(dpt_addr + hh * 64 + cb * 16, ds);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.ew_done);
-                if (wq == 0 && lane == 0) mbar_arrive(&sm.rows_empty[rb]);  // the table is no longer read
+                if (warp == 4 && lane == 0) mbar_arrive(&sm.rows_empty[rb]);  // the table is no longer read
             }
             if (!ok) break;
             // epilogue: dK (scaled by 1/sqrt(d)) and dV rows of the item's keys
@@ -851,7 +854,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 float* dst_row = (part == 0 ? p.dK : p.dV) + kv_row * kD;
                 const float f = (part == 0) ? p.scale : 1.0f;
 #pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
+                for (int cb = 2 * hh; cb < 2 * hh + 2; ++cb) {  // this warp's 64 columns
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_off + part * 128 + cb * 32, o);
                     tmem_ld_wait();
@@ -920,8 +923,11 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     char* base = static_cast<char*>(a.scratch);
     float* gamma = reinterpret_cast<float*>(base);
     float* delta = reinterpret_cast<float*>(base + L.plane);
-    float* lse = reinterpret_cast<float*>(base + 2 * L.plane);
-    float* o32 = reinterpret_cast<float*>(base + 3 * L.plane);
+    float* lse_ws = reinterpret_cast<float*>(base + 2 * L.plane);
+    float* o32_ws = reinterpret_cast<float*>(base + 3 * L.plane);
+    const bool saved = a.o32 != nullptr && a.lse != nullptr;
+    const float* lse = saved ? a.lse : lse_ws;
+    const float* o32 = saved ? a.o32 : o32_ws;
     RowRec* rec = reinterpret_cast<RowRec*>(base + 3 * L.plane + L.o32);
     int32_t* jtab = reinterpret_cast<int32_t*>(base + 3 * L.plane + L.o32 + L.rec);
     __nv_bfloat16* Qc = reinterpret_cast<__nv_bfloat16*>(base + 3 * L.plane + L.o32 + L.rec + L.jtab);
@@ -929,26 +935,30 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     const int64_t rows_total = L.tiles * kBM;
     if (rows_total >= ((int64_t)1 << 31) - 1 || BT * s.h >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
 
-    // 0. the forward again, writing o and the log2-sum-exp of every routed row
-    PrefillArgs f;
-    f.s = a.s;
-    f.Q = a.Q;
-    f.K = a.K;
-    f.V = a.V;
-    f.idx = a.idx;
-    f.gate = a.gate;
-    f.head_offsets = a.head_offsets;
-    f.head_pos = a.head_pos;
-    f.head_chunk_offsets = a.head_chunk_offsets;
-    f.O = nullptr;
-    f.status = a.status;
-    f.stream = a.stream;
-    f.kv_g = s.g;
-    f.kv_q0 = 0;
-    f.o32 = o32;
-    f.lse = lse;
-    cudaError_t e = launch_prefill_tc(f);
-    if (e != cudaSuccess) return e;
+    // 0. unless the training forward saved them: the forward again, writing o
+    // and the log2-sum-exp of every routed row
+    cudaError_t e = cudaSuccess;
+    if (!saved) {
+        PrefillArgs f;
+        f.s = a.s;
+        f.Q = a.Q;
+        f.K = a.K;
+        f.V = a.V;
+        f.idx = a.idx;
+        f.gate = a.gate;
+        f.head_offsets = a.head_offsets;
+        f.head_pos = a.head_pos;
+        f.head_chunk_offsets = a.head_chunk_offsets;
+        f.O = nullptr;
+        f.status = a.status;
+        f.stream = a.stream;
+        f.kv_g = s.g;
+        f.kv_q0 = 0;
+        f.o32 = o32_ws;
+        f.lse = lse_ws;
+        e = launch_prefill_tc(f);
+        if (e != cudaSuccess) return e;
+    }
 
     // 1. D, gates, logit gradients, zero dQ of unselected heads
     const int64_t warps = BT * s.g;

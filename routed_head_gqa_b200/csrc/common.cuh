@@ -132,9 +132,10 @@ struct PrefillArgs {
     // group of one head over a chosen KV group of the caller's K/V.
     int kv_g;
     int kv_q0;
-    // Training recompute (tensor-core prefill only): when o32 is set, the kernel
-    // writes each routed row's ungated fp32 output o32[b,t,j,:] and its
-    // log2-sum-exp lse[b,t,j] instead of O (O and its zero fill are skipped).
+    // Training outputs (tensor-core prefill only): when o32 is set, the kernel
+    // also writes each routed row's ungated fp32 output o32[b,t,j,:] and its
+    // log2-sum-exp lse[b,t,j]; O may then be null (a recompute for the
+    // backward: O and its zero fill are skipped).
     float* o32 = nullptr;
     float* lse = nullptr;
 };

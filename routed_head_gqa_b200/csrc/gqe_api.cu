@@ -434,6 +434,79 @@ gqe_status gqe_attn_prefill_backward(const gqe_shape* s, const void* Q, const vo
     return from_cuda(launch_attn_backward(a));
 }
 
+gqe_status gqe_attn_prefill_train(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                  const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                  const int32_t* head_pos, const int32_t* head_chunk_offsets, void* O, float* O32,
+                                  float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!Q || !K || !V || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets || !O32 || !lse)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || (O && !aligned16(O)) || !aligned16(O32))
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!attn_backward_tc_supported(s)) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != GQE_OK) return st;
+    PrefillArgs a;
+    a.s = s;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.O = O;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    a.kv_g = s->g;
+    a.kv_q0 = 0;
+    a.o32 = O32;
+    a.lse = lse;
+    return from_cuda(launch_prefill_tc(a));
+}
+
+gqe_status gqe_attn_prefill_backward_saved(const gqe_shape* s, const void* Q, const void* K, const void* V,
+                                           const int32_t* idx, const float* gate, const int32_t* head_offsets,
+                                           const int32_t* head_pos, const int32_t* head_chunk_offsets,
+                                           const void* dO, const float* O32, const float* lse, float* dQ, float* dK,
+                                           float* dV, float* dlogits, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!Q || !K || !V || !idx || !gate || !head_offsets || !head_pos || !head_chunk_offsets || !dO || !O32 || !lse ||
+        !dQ || !dK || !dV || !dlogits)
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(O32) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV))
+        return GQE_ERR_INVALID_ARGUMENT;
+    if (!attn_backward_tc_supported(s)) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + attn_backward_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    AttnBwdArgs a;
+    a.s = s;
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
+    a.dO = dO;
+    a.idx = idx;
+    a.gate = gate;
+    a.head_offsets = head_offsets;
+    a.head_pos = head_pos;
+    a.head_chunk_offsets = head_chunk_offsets;
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dlogits = dlogits;
+    a.scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.status = workspace;
+    a.stream = (cudaStream_t)stream;
+    a.o32 = O32;
+    a.lse = lse;
+    return from_cuda(launch_attn_backward(a));
+}
+
 gqe_status gqe_get_device_status(void* workspace, void* stream) {
     if (!workspace) return GQE_ERR_INVALID_ARGUMENT;
     DeviceStatus host{};

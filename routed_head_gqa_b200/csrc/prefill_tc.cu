@@ -80,7 +80,7 @@ struct Params {
     const int32_t* head_offsets;
     const int32_t* head_pos;
     const int32_t* head_chunk_offsets;
-    __nv_bfloat16* O;   // gated bf16 output; null when the training outputs are asked for instead
+    __nv_bfloat16* O;   // gated bf16 output (null: a recompute for the backward, training outputs only)
     float* o32;         // training: ungated fp32 output of every routed row, [B, T, h, 128]
     float* lse;         // training: log2-sum-exp of every routed row's scaled scores, [B, T, h]
     uint32_t* status;
@@ -136,7 +136,7 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
 
 
 // ---------------------------------------------------------------------------
-template <bool kTrain>  // kTrain: write the training outputs (o32, lse) instead of O
+template <bool kTrain>  // kTrain: also write the training outputs (o32, lse); O only when asked
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQB,
@@ -473,7 +473,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         // selections at once; the warp then zeroes the unselected 256-byte
         // slots, 16 lanes per slot.
         const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
-        for (int64_t j = 0; !kTrain; ++j) {  // the training outputs leave O alone
+        for (int64_t j = 0; p.O != nullptr; ++j) {  // a recompute for the backward leaves O alone
             const int64_t unit = cta_unit(j, n_units);
             if (unit < 0 || aborted(sm)) break;
             int b, q, w;
@@ -697,10 +697,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     }
                 }
                 if (t_row >= 0) p.lse[orow_idx] = m + log2f(l);
-                tc_fence_before();
-                mbar_arrive(&sm.o_empty[t]);
-                mbar_arrive(&sm.rows_free[rs]);
-                continue;
+                if (p.O == nullptr) {  // a recompute for the backward: O is not wanted
+                    tc_fence_before();
+                    mbar_arrive(&sm.o_empty[t]);
+                    mbar_arrive(&sm.rows_free[rs]);
+                    continue;
+                }
             }
             const float f = (t_row >= 0) ? sm.row_gate[rs][t][r] / l : 0.f;
             __nv_bfloat16* orow = p.O + orow_idx * kD;

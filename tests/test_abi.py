@@ -160,17 +160,37 @@ def test_attn_backward_validation():
     import routed_head_gqa_b200 as g
 
     fake = 0x10000
+    a256 = lambda n: (n + 255) // 256 * 256
+    # fp32 inputs (CUDA-core backward): status word + the larger of the attention
+    # scratch (gate, D, lse per (b,t,j)) and the router's dW_r partials
+    s32 = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_F32)
+    assert g.gqe_backward_workspace_bytes(s32) == 256 + max(3 * 2 * 64 * 8 * 4, 64 * 128 * 8 * 4)
+    # bf16 with d_h = 128 (tensor-core backward): the gate, D and lse planes, the
+    # rows' fp32 outputs, then the packed half-window tiles (2*ceil(T/2W) per
+    # (b, group), W = 64 for k = 2): 16-byte row records, heads, Q and dO rows
     s = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_BF16)
     need = g.gqe_backward_workspace_bytes(s)
-    # status word + the larger of the attention scratch (gate, D, lse per (b,t,j))
-    # and the router's dW_r partials (64 token ranges here)
-    assert need == 256 + max(3 * 2 * 64 * 8 * 4, 64 * 128 * 8 * 4)
+    bth, tiles = 2 * 64 * 8, 2 * 2 * 2
+    attn = 3 * a256(bth * 4) + a256(bth * 128 * 4) + a256(tiles * 128 * 16) + a256(tiles * 128 * 4) \
+        + 2 * a256(tiles * 128 * 128 * 2)
+    assert need == 256 + max(attn, 64 * 128 * 8 * 4)
     call = lambda s, dQ, ws_bytes: g._lib.gqe_attn_prefill_backward(
         ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, dQ, fake, fake, fake, fake,
         ws_bytes, None)
     assert call(s, None, need) == 1             # no dQ
     assert call(s, fake + 8, need) == 1         # misaligned dQ
-    assert call(s, fake, 256 + 3 * 2 * 64 * 8 * 4 - 1) == 1  # workspace too small for the attention scratch
+    assert call(s, fake, 256 + attn - 1) == 1   # workspace too small for the attention scratch
+    train = lambda s, o32, lse: g._lib.gqe_attn_prefill_train(
+        ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, None, o32, lse, fake, 1 << 20, None)
+    assert train(s, None, fake) == 1            # no O32
+    assert train(s, fake, None) == 1            # no lse
+    assert train(s32, fake, fake) == 2          # the training forward is the tensor-core path only
+    saved = lambda s, lse, ws_bytes: g._lib.gqe_attn_prefill_backward_saved(
+        ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, lse, fake, fake, fake, fake,
+        fake, ws_bytes, None)
+    assert saved(s, None, need) == 1            # no lse
+    assert saved(s, fake, 256 + attn - 1) == 1  # workspace too small
+    assert saved(s32, fake, 1 << 30) == 2       # fp32: no saved-statistics path
     s96 = g.make_shape(2, 64, 128, 8, 2, 96, 2, g.GQE_BF16)
     assert call(s96, fake, 1 << 30) == 2        # d_h 96 not implemented
     bad = g.make_shape(2, 64, 128, 8, 3, 128, 2, g.GQE_BF16)

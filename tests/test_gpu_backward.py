@@ -170,3 +170,52 @@ def test_backward_dense_gqa_full_size():
     assert np.abs(dK.sum(axis=1)).max() <= tol, "sum_s dK != 0"
     # and every group's logit gradients sum to zero
     assert np.abs(dl.reshape(w.B, w.T, w.g, -1).sum(-1)).max() <= 1e-4
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[3], W["dense_gqa"]], ids=lambda w: w.name)
+def test_train_forward_and_saved_backward(w):
+    """gqe_attn_prefill_train: O within the forward tolerance of the oracle and
+    O32 * gate equal to it within the same bound (the ungated rows it saves);
+    gqe_attn_prefill_backward_saved on those statistics gives gradients
+    bit-identical to gqe_attn_prefill_backward, which recomputes them."""
+    g = U.gqe()
+    inp = gqe_synth.make_inputs(w)
+    dO = gqe_synth.make_output_grad(w).cuda()
+    shape = g.make_shape(w.B, w.T, w.d_model, w.h, w.g, w.d_h, w.k, w.torch_dtype)
+    buf = g.Buffers(shape, "cuda")
+    buf.route(U.to_dev(inp["x"]), U.to_dev(inp["W_r"]), U.to_dev(inp["bias"]))
+    Q, K, V = (U.to_dev(inp[n]) for n in ("Q", "K", "V"))
+    O32 = torch.full((w.B, w.T, w.h, w.d_h), float("nan"), device="cuda")
+    lse = torch.full((w.B, w.T, w.h), float("nan"), device="cuda")
+    g.gqe_attn_prefill_train(shape, Q, K, V, buf.idx, buf.gate, buf.head_offsets, buf.head_pos,
+                             buf.head_chunk_offsets, buf.O, O32, lse, buf.workspace)
+    torch.cuda.synchronize()
+    assert buf.status() == 0
+    excl, idx_o, gate_o = U.check_routing(w, inp, buf.idx, buf.gate)
+    rows = U.cover_rows(w, idx_o, U.sm_count(), n_min=512) if w.T > 512 else None
+    err, n = U.compare_rows(w, inp, buf.O, idx_o, gate_o, excl, rows)
+    assert err <= U.TOL["bf16"], f"{w.name}: training forward O error {err}"
+    sel = torch.zeros((w.B, w.T, w.h), dtype=torch.bool, device="cuda")
+    sel.scatter_(2, buf.idx.reshape(w.B, w.T, -1).long(), True)
+    gates = torch.zeros((w.B, w.T, w.h), device="cuda").scatter_(2, buf.idx.reshape(w.B, w.T, -1).long(),
+                                                                  buf.gate.reshape(w.B, w.T, -1))
+    gated = (O32 * gates[..., None])[sel]
+    assert torch.isfinite(O32[sel]).all() and torch.isfinite(lse[sel]).all()
+    assert (gated - buf.O.float()[sel]).abs().max().item() <= U.TOL["bf16"]
+    outs = []
+    for saved in (False, True):
+        f32 = dict(dtype=torch.float32, device="cuda")
+        dQ, dK, dV = (torch.full(sh, float("nan"), **f32) for sh in
+                      ((w.B, w.T, w.h, w.d_h), (w.B, w.T, w.g, w.d_h), (w.B, w.T, w.g, w.d_h)))
+        dl = torch.full((w.B, w.T, w.h), float("nan"), **f32)
+        ws = torch.zeros(g.gqe_backward_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+        args = (shape, Q, K, V, buf.idx, buf.gate, buf.head_offsets, buf.head_pos, buf.head_chunk_offsets, dO)
+        if saved:
+            g.gqe_attn_prefill_backward_saved(*args, O32, lse, dQ, dK, dV, dl, ws)
+        else:
+            g.gqe_attn_prefill_backward(*args, dQ, dK, dV, dl, ws)
+        torch.cuda.synchronize()
+        assert g.gqe_get_device_status(ws) == 0
+        outs.append((dQ, dK, dV, dl))
+    for name, a, b in zip(("dQ", "dK", "dV", "dlogits"), outs[0], outs[1]):
+        assert torch.equal(a, b), f"{w.name}: {name} differs between the saved and the recomputing backward"

@@ -66,6 +66,26 @@ def test_prefill_full_size_covered(name):
     assert err <= U.TOL[w.dtype], f"{name}: max abs error {err} over {n} rows ({excl} tokens excluded)"
 
 
+def test_prefill_32k_sampled():
+    """A 32768-token sequence (B=1, h=16, g=8, k=1): every position of the last
+    window and of the windows that the first and the last CTA run first, and
+    random rows, 1024 rows in all (the oracle's cost grows with the context)."""
+    w = W["gqe_32k"]
+    inp = gqe_synth.make_inputs(w)
+    buf = U.run_prefill(w, inp)
+    excl, idx_o, gate_o = U.check_routing(w, inp, buf.idx, buf.gate)
+    _, nwin = U.prefill_windows(w)
+    span = 2 * 32 * (4 // w.k)
+    rows = set(range(w.T - span, w.T))
+    for c in (0, min(w.B * w.g * nwin, U.sm_count()) - 1):
+        b, _, win = U.cta_units(w, U.sm_count(), c)[0]
+        rows.update(range(b * w.T + win * span, b * w.T + min((win + 1) * span, w.T)))
+    rng = np.random.default_rng(32768)
+    rows.update(int(r) for r in rng.choice(w.B * w.T, 1024 - len(rows), replace=False))
+    err, n = U.compare_rows(w, inp, buf.O, idx_o, gate_o, excl, np.array(sorted(rows)))
+    assert n >= 900 and err <= U.TOL["bf16"], f"gqe_32k: max abs error {err} over {n} rows"
+
+
 def test_full_size_repeatable():
     """Routing and prefill at the gqe_prefill size (the bench's launch
     configuration) run twice on the same inputs give bit-identical tables and
