@@ -310,10 +310,23 @@ class Buffers:
         gqe_attn_decode(self.shape, q, K_cache, V_cache, K_cache.shape[1], lengths, self.idx, self.gate, self.O,
                         self.workspace, stream)
 
-    def backward(self, Q, K, V, dO, stream=None):
+    def prefill_train(self, Q, K, V, stream=None):
+        """The training forward: O as `prefill`, plus each routed row's fp32
+        output and log2-sum-exp, kept here for `backward(..., saved=True)`."""
+        sh = self.shape
+        if getattr(self, "_saved", None) is None:
+            f32 = dict(dtype=torch.float32, device=self.idx.device)
+            self._saved = (torch.empty((sh.B, sh.T, sh.h, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.h), **f32))
+        O32, lse = self._saved
+        gqe_attn_prefill_train(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
+                               self.head_chunk_offsets, self.O, O32, lse, self.workspace, stream)
+
+    def backward(self, Q, K, V, dO, stream=None, saved=False):
         """Gradients of the routed attention for output gradient dO (the routing
         of the last `route`): returns (dQ, dK, dV, dlogits), float32 tensors
-        owned by this object and overwritten by the next call."""
+        owned by this object and overwritten by the next call.  saved=True
+        reads the statistics of the last `prefill_train` instead of
+        recomputing the forward."""
         sh = self.shape
         if getattr(self, "_bwd", None) is None:
             dev = self.idx.device
@@ -323,8 +336,15 @@ class Buffers:
                          torch.empty((sh.B, sh.T, sh.g, sh.d_h), **f32), torch.empty((sh.B, sh.T, sh.h), **f32),
                          torch.zeros(nbytes, dtype=torch.uint8, device=dev))
         dQ, dK, dV, dl, ws = self._bwd
-        gqe_attn_prefill_backward(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
-                                  self.head_chunk_offsets, dO, dQ, dK, dV, dl, ws, stream)
+        if saved:
+            if getattr(self, "_saved", None) is None:
+                raise RuntimeError("backward(saved=True) follows prefill_train")
+            gqe_attn_prefill_backward_saved(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
+                                            self.head_chunk_offsets, dO, self._saved[0], self._saved[1], dQ, dK, dV,
+                                            dl, ws, stream)
+        else:
+            gqe_attn_prefill_backward(sh, Q, K, V, self.idx, self.gate, self.head_offsets, self.head_pos,
+                                      self.head_chunk_offsets, dO, dQ, dK, dV, dl, ws, stream)
         return dQ, dK, dV, dl
 
     def route_backward(self, x, W_r, dlogits, stream=None):

@@ -13,23 +13,30 @@
 //   dV_s  = sum_r p_rs g_r dO_r,         dlogit_j = D_j - g_j sum_{i in S} D_i.
 //
 // Launches (after the tensor-core prefill has written o_r in fp32 and the
-// row's log2-sum-exp lse_r into the workspace, so p_rs = 2^(s_rs c - lse_r)):
-//  1. bwd_prep_kernel: one warp per (b, t, group): D_r, the gates, the logit
-//     gradients, and zero dQ rows for the unselected heads.
-//  1b. bwd_tiles_kernel: one warp per half-window tile of a group (the
-//     prefill's row tiles): the tile's row table (position, head, and per row
-//     lse, gate, D) and its Q and dO rows, packed contiguously in the workspace,
-//     so that the two tensor-core kernels load each tile with plain TMA boxes.
-//  2. dq_tc_kernel: per 128-row tile of routed rows (the prefill's half-window
-//     tiles): S = Q K^T and dP = dO V^T on the tensor cores, dS in registers,
-//     dQ += dS K accumulated in TMEM.
+// row's log2-sum-exp lse_r, so p_rs = 2^(s_rs c - lse_r)):
+//  1. bwd_pack_kernel: one block per half-window tile of a group (the
+//     prefill's row tiles): the tile's row table, its Q and dO rows packed
+//     contiguously (so the tensor-core kernels load a tile with plain TMA
+//     boxes), dO_r . o_r, the logit gradients of the tile's positions, and
+//     zero dQ rows for the unselected heads.  The table folds the gate into
+//     the row's statistics: lse2_r = lse_r - log2 g_r and dl2_r = dO_r . o_r,
+//     so that g_r p_rs = 2^(s_rs c - lse2_r) and dS_rs = g_r p_rs (dP_rs - dl2_r)
+//     with dP_rs = dO_r . v_s.
+//  2. dq_tc_kernel: per 128-row tile of routed rows: S = Q K^T and
+//     dP = dO V^T on the tensor cores, dS in registers, dQ += dS K
+//     accumulated in TMEM.
 //  3. dkdv_tc_kernel: per (b, group, 128-key tile): S^T = K Q^T and
 //     dP^T = V dO^T over the group's routed row tiles at or after the keys,
 //     then dV += (g p)^T dO and dK += dS^T Q accumulated in TMEM.
+// In both tensor-core kernels the elementwise step runs in two phases, the
+// exponentials (from S) and dS (from dP), each overlapping an MMA of the
+// neighbouring phase, and only tiles that straddle the causal diagonal are
+// masked.
 // Every sum runs in a fixed order: the gradients are reproducible.
 #include <climits>
 
 #include "backward.cuh"
+#include "exp2_fma.cuh"
 #include "sm100.cuh"
 #include "tma_host.cuh"
 #include "units.cuh"
@@ -66,13 +73,12 @@ struct RowTable {
     int32_t j[kBM];
     float gate[kBM];
     float lse[kBM];
-    float dlt[kBM];
     int32_t qrow[kBM];  // row of Q / dO viewed as [B*T*h, 128]; padding rows name q_rows (zero fill)
 };
 
 __device__ void build_rows(const UnitGeom& u, int b, int q, int w0, const int32_t* head_offsets,
                            const int32_t* head_chunk_offsets, const int32_t* head_pos, const int32_t* idx,
-                           const float* gate_in, const float* lse, const float* dlt, int q_rows, RowTable& rt,
+                           const float* gate_in, const float* lse, int q_rows, RowTable& rt,
                            int32_t* cut_start, int32_t* cut_prefix, uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const int32_t total = (int32_t)((int64_t)u.B * u.T * u.g * u.k);
@@ -100,7 +106,7 @@ __device__ void build_rows(const UnitGeom& u, int b, int q, int w0, const int32_
     const int nrows = cut_prefix[u.hpg];
     for (int r = lane; r < kBM; r += 32) {
         int tt = -1, jh = 0;
-        float gv = 0.f, lv = 0.f, dv = 0.f;
+        float gv = 0.f, lv = 0.f;
         if (r < nrows) {
             int jj = 0;
             while (cut_prefix[jj + 1] <= r) ++jj;
@@ -117,150 +123,135 @@ __device__ void build_rows(const UnitGeom& u, int b, int q, int w0, const int32_
                 if (idx[sel + s2] == jh) gv = gate_in[sel + s2];
             const int64_t row = ((int64_t)b * u.T + tt) * u.h + jh;
             lv = lse[row];
-            dv = dlt[row];
         }
         rt.t[r] = tt;
         rt.j[r] = jh;
         rt.gate[r] = gv;
         rt.lse[r] = lv;
-        rt.dlt[r] = dv;
         rt.qrow[r] = (tt >= 0) ? (int32_t)(((int64_t)b * u.T + tt) * u.h + jh) : q_rows;
     }
     __syncwarp();
 }
 
-// A packed tile: per row (lse, gate, D, position t) in one 16-byte record
-// (t = -1 for padding) and the row's head, as the tensor-core kernels read them.
-struct RowRec {
-    float lse, gate, dlt;
-    int32_t t;
-};
+// A packed tile's table, in the workspace and in shared memory: per row
+// lse2 = lse - log2(gate) (+inf for padding and zero gates), dl2 = dO . o,
+// the position t (-1: padding) and the head j.
 struct TileTab {
-    RowRec rec[kBM];
+    float lse2[kBM];
+    float dl2[kBM];
+    int32_t t[kBM];
     int32_t j[kBM];
 };
+static_assert(sizeof(TileTab) == 2048, "a tile table is 2 KB");
 
 // One warp copies a packed tile's table from the workspace into shared memory.
-__device__ __forceinline__ void load_tab(const RowRec* rec_g, const int32_t* j_g, TileTab& tt) {
+__device__ __forceinline__ void load_tab(const TileTab* src_tab, TileTab& dst_tab) {
     const int lane = threadIdx.x & 31;
-    const int4* src = reinterpret_cast<const int4*>(rec_g);
-    int4* dst = reinterpret_cast<int4*>(tt.rec);
+    const int4* src = reinterpret_cast<const int4*>(src_tab);
+    int4* dst = reinterpret_cast<int4*>(&dst_tab);
 #pragma unroll
-    for (int i = 0; i < kBM / 32; ++i) dst[lane + 32 * i] = src[lane + 32 * i];
-#pragma unroll
-    for (int i = 0; i < kBM / 32; ++i) tt.j[lane + 32 * i] = j_g[lane + 32 * i];
+    for (int i = 0; i < 4; ++i) dst[lane + 32 * i] = src[lane + 32 * i];
 }
 
-// p = 2^(s c - lse) (0 where masked), pg = gate p, ds = p (gate dp - D), as
-// bf16 pairs; 32 values of s and dp, one pair of table entries per step.
-struct Elem2 {
-    uint32_t pg, ds;
-};
-
-// ------------------------------------------------------------------ 1. prep
-__global__ void __launch_bounds__(256)
-bwd_prep_kernel(int64_t BT, int h, int g, int k, const int32_t* __restrict__ idx, const float* __restrict__ gate,
-                const __nv_bfloat16* __restrict__ dO, const float* __restrict__ o32, float* __restrict__ gamma,
-                float* __restrict__ delta, float* __restrict__ dlogits, float* __restrict__ dQ, uint32_t* status) {
-    const int lane = threadIdx.x & 31;
-    const int64_t item = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // bt * g + q
-    if (item >= BT * g) return;
-    const int64_t bt = item / g;
-    const int q = (int)(item % g), hpg = h / g;
-    float dsel[16], gsel[16];
-    int jsel[16];
-    float dsum = 0.f;
-#pragma unroll
-    for (int s = 0; s < 16; ++s) {
-        dsel[s] = 0.f;
-        gsel[s] = 0.f;
-        jsel[s] = -1;
-        if (s < k) {
-            const int j = idx[item * k + s];
-            if (j < q * hpg || j >= (q + 1) * hpg) {
-                if (lane == 0) report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 3);
-                continue;
-            }
-            const float gm = gate[item * k + s];
-            const int64_t row = bt * h + j;
-            // D = g dO . o over the row's 128 elements, 4 per lane, then a butterfly
-            const uint2 dv = *reinterpret_cast<const uint2*>(dO + row * kD + lane * 4);
-            const float4 ov = *reinterpret_cast<const float4*>(o32 + row * kD + lane * 4);
-            float acc = __uint_as_float(dv.x << 16) * ov.x + __uint_as_float(dv.x & 0xffff0000u) * ov.y +
-                        __uint_as_float(dv.y << 16) * ov.z + __uint_as_float(dv.y & 0xffff0000u) * ov.w;
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
-            jsel[s] = j;
-            gsel[s] = gm;
-            dsel[s] = gm * acc;
-            dsum += dsel[s];
-            if (lane == 0) {
-                gamma[row] = gm;
-                delta[row] = dsel[s];
-            }
-        }
-    }
-    for (int jj = lane; jj < hpg; jj += 32) {
-        const int j = q * hpg + jj;
-        float dl = 0.f;
-#pragma unroll
-        for (int s = 0; s < 16; ++s)
-            if (s < k && jsel[s] == j) dl = dsel[s] - gsel[s] * dsum;
-        dlogits[bt * h + j] = dl;
-    }
-    for (int jj = 0; jj < hpg; ++jj) {  // dQ of an unselected head is 0
-        const int j = q * hpg + jj;
-        bool sel = false;
-#pragma unroll
-        for (int s = 0; s < 16; ++s) sel |= (s < k && jsel[s] == j);
-        if (sel) continue;
-        *reinterpret_cast<float4*>(dQ + (bt * h + j) * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-}
-
-// ------------------------------------------------------------------ 1b. packed tiles
-// Tile id (b*g + q) * ntiles + ti covers positions [ti*W, (ti+1)*W) of group q of
-// sequence b; one warp per tile (four per block).
-__global__ void __launch_bounds__(128)
-bwd_tiles_kernel(UnitGeom u, int ntiles, const int32_t* __restrict__ head_offsets,
-                 const int32_t* __restrict__ head_chunk_offsets, const int32_t* __restrict__ head_pos,
-                 const int32_t* __restrict__ idx, const float* __restrict__ gate, const float* __restrict__ lse,
-                 const float* __restrict__ dlt, const __nv_bfloat16* __restrict__ Q,
-                 const __nv_bfloat16* __restrict__ dO, RowRec* __restrict__ rec, int32_t* __restrict__ jtab,
-                 __nv_bfloat16* __restrict__ Qc, __nv_bfloat16* __restrict__ dOc, uint32_t* status) {
-    __shared__ RowTable rt[4];
-    __shared__ int32_t cut_start[4][32], cut_prefix[4][33];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t tile = (int64_t)blockIdx.x * 4 + warp;
-    const int64_t n = (int64_t)u.B * u.g * ntiles;
-    if (tile >= n) return;
+// ------------------------------------------------------------------ 1. packed tiles
+// Block = tile id (b*g + q) * ntiles + ti: positions [ti*W, (ti+1)*W) of group
+// q of sequence b.  Every head of the group selected at one of these positions
+// has its row in this tile, so the logit gradients of the tile's positions
+// (dlogit_j = D_j - g_j sum_i D_i over the selected heads i, 0 for the others)
+// are complete here; the sum runs in head order.
+constexpr int kPackThreads = 256;
+__global__ void __launch_bounds__(kPackThreads)
+bwd_pack_kernel(UnitGeom u, int ntiles, const int32_t* __restrict__ head_offsets,
+                const int32_t* __restrict__ head_chunk_offsets, const int32_t* __restrict__ head_pos,
+                const int32_t* __restrict__ idx, const float* __restrict__ gate, const float* __restrict__ lse,
+                const float* __restrict__ o32, const __nv_bfloat16* __restrict__ Q,
+                const __nv_bfloat16* __restrict__ dO, TileTab* __restrict__ tabs, __nv_bfloat16* __restrict__ Qc,
+                __nv_bfloat16* __restrict__ dOc, float* __restrict__ dlogits, float* __restrict__ dQ,
+                uint32_t* status) {
+    __shared__ RowTable rt;
+    __shared__ int32_t cut_start[32], cut_prefix[33];
+    __shared__ float dot_s[kBM];
+    __shared__ float dsum[kBM];
+    __shared__ int16_t row_of[kBM * 32];  // (position - w0) * hpg + head in group -> row, -1: unselected
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t tile = blockIdx.x;
     const int ti = (int)(tile % ntiles);
     const int bq = (int)(tile / ntiles);
-    const int b = bq / u.g, q = bq % u.g;
-    RowTable& t = rt[warp];
-    build_rows(u, b, q, ti * u.W, head_offsets, head_chunk_offsets, head_pos, idx, gate, lse, dlt, -1, t,
-               cut_start[warp], cut_prefix[warp], status);
-    for (int r = lane; r < kBM; r += 32) {
-        RowRec x;
-        x.lse = t.lse[r];
-        x.gate = t.gate[r];
-        x.dlt = t.dlt[r];
-        x.t = t.t[r];
-        rec[tile * kBM + r] = x;
-        jtab[tile * kBM + r] = t.j[r];
+    const int b = bq / u.g, q = bq % u.g, hpg = u.hpg;
+    const int w0 = ti * u.W;
+    const int npos = max(0, min(u.W, u.T - w0));
+    for (int i = tid; i < u.W * hpg; i += kPackThreads) row_of[i] = -1;
+    for (int i = tid; i < npos * u.k; i += kPackThreads) {  // every selected head belongs to group q
+        const int j = idx[(((int64_t)b * u.T + w0 + i / u.k) * u.g + q) * u.k + i % u.k];
+        if (j < q * hpg || j >= (q + 1) * hpg) report_error(status, GQE_ERR_INVALID_ARGUMENT, kWhereBwdTc, 3);
     }
-    // Q and dO rows: 16 lanes per 256-byte row, two rows per pass
+    if (warp == 0)
+        build_rows(u, b, q, w0, head_offsets, head_chunk_offsets, head_pos, idx, gate, lse, -1, rt, cut_start,
+                   cut_prefix, status);
+    __syncthreads();
+    // Q and dO rows, and dO . o: 16 lanes per 256-byte row, 16 rows per pass
     const int half = lane >> 4, c = lane & 15;
-    for (int r0 = 0; r0 < kBM; r0 += 2) {
-        const int r = r0 + half;
-        const int32_t src = t.qrow[r];
+    for (int r = warp * 2 + half; r < kBM; r += 2 * (kPackThreads / 32)) {
+        const int tt = rt.t[r];
         uint4 qv = make_uint4(0, 0, 0, 0), dv = qv;
-        if (t.t[r] >= 0) {
-            qv = reinterpret_cast<const uint4*>(Q + (int64_t)src * kD)[c];
-            dv = reinterpret_cast<const uint4*>(dO + (int64_t)src * kD)[c];
+        float acc = 0.f;
+        if (tt >= 0) {
+            const int64_t src = rt.qrow[r];
+            qv = reinterpret_cast<const uint4*>(Q + src * kD)[c];
+            dv = reinterpret_cast<const uint4*>(dO + src * kD)[c];
+            const float4 o0 = reinterpret_cast<const float4*>(o32 + src * kD)[2 * c];
+            const float4 o1 = reinterpret_cast<const float4*>(o32 + src * kD)[2 * c + 1];
+            acc = __uint_as_float(dv.x << 16) * o0.x + __uint_as_float(dv.x & 0xffff0000u) * o0.y +
+                  __uint_as_float(dv.y << 16) * o0.z + __uint_as_float(dv.y & 0xffff0000u) * o0.w +
+                  __uint_as_float(dv.z << 16) * o1.x + __uint_as_float(dv.z & 0xffff0000u) * o1.y +
+                  __uint_as_float(dv.w << 16) * o1.z + __uint_as_float(dv.w & 0xffff0000u) * o1.w;
         }
+#pragma unroll
+        for (int d = 8; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);  // within the half-warp
         reinterpret_cast<uint4*>(Qc + (tile * kBM + r) * kD)[c] = qv;
         reinterpret_cast<uint4*>(dOc + (tile * kBM + r) * kD)[c] = dv;
+        if (c == 0) {
+            dot_s[r] = acc;
+            if (tt >= 0) row_of[(tt - w0) * hpg + (rt.j[r] - q * hpg)] = (int16_t)r;
+        }
+    }
+    __syncthreads();
+    // per position: sum of D = g (dO . o) over its selected heads, in head order
+    if (tid < npos) {
+        float sum = 0.f;
+        for (int jj = 0; jj < hpg; ++jj) {
+            const int r = row_of[tid * hpg + jj];
+            if (r >= 0) sum += rt.gate[r] * dot_s[r];
+        }
+        dsum[tid] = sum;
+    }
+    // the table
+    if (tid < kBM) {
+        const int tt = rt.t[tid];
+        const float gm = rt.gate[tid];
+        TileTab& tab = tabs[tile];
+        tab.lse2[tid] = (tt >= 0 && gm > 0.f) ? rt.lse[tid] - log2f(gm) : __int_as_float(0x7f800000);
+        tab.dl2[tid] = (tt >= 0) ? dot_s[tid] : 0.f;
+        tab.t[tid] = tt;
+        tab.j[tid] = rt.j[tid];
+    }
+    __syncthreads();
+    for (int i = tid; i < npos * hpg; i += kPackThreads) {
+        const int pp = i / hpg, jj = i - pp * hpg;
+        const int r = row_of[i];
+        float dl = 0.f;
+        if (r >= 0) {
+            const float gm = rt.gate[r];
+            dl = gm * dot_s[r] - gm * dsum[pp];
+        }
+        dlogits[((int64_t)b * u.T + w0 + pp) * u.h + q * hpg + jj] = dl;
+    }
+    // dQ of an unselected head is 0: one warp per (position, head)
+    for (int i = warp; i < npos * hpg; i += kPackThreads / 32) {
+        if (row_of[i] >= 0) continue;
+        const int pp = i / hpg, jj = i - pp * hpg;
+        float4* dst = reinterpret_cast<float4*>(dQ + (((int64_t)b * u.T + w0 + pp) * u.h + q * hpg + jj) * kD);
+        dst[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -272,10 +263,7 @@ struct Params {
     const int32_t* head_offsets;
     const int32_t* head_pos;
     const int32_t* head_chunk_offsets;
-    const float* lse;
-    const float* dlt;
-    const RowRec* rec;     // packed tile tables
-    const int32_t* jtab;
+    const TileTab* tabs;   // packed tile tables
     int ntiles;            // half-window tiles per (b, group): 2 * ceil(T / 2W)
     float* dQ;
     float* dK;
@@ -291,40 +279,90 @@ __device__ __forceinline__ void fail(int32_t* abort_flag, uint32_t* status, uint
     report_error(status, GQE_ERR_DEVICE_TIMEOUT, kWhereBwdTc, detail);
 }
 
-// One 32-column chunk of the elementwise step: s (scores) and d (dP) for 32
-// columns c0..c0+31 of this thread's TMEM lane; per column the table entry gives
-// lse, gate, D and visibility.  Returns 16 packed pairs of pg and ds.
-template <bool KEY_ROWS>
-__device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float c, float lse_or_row,
-                                         float gate_row, float dlt_row, int key_or_t, const RowRec* recs, int col0,
-                                         int kv0, uint32_t (&pg)[16], uint32_t (&ds)[16]) {
+// Item of wave v for this CTA.  Items are numbered heaviest first; the waves
+// alternate direction over the CTAs so that every CTA's share of the work
+// comes out nearly even.
+__device__ __forceinline__ int64_t snake_item(int64_t v) {
+    const int64_t G = gridDim.x, c = blockIdx.x;
+    return v * G + ((v & 1) ? (G - 1 - c) : c);
+}
+
+// Of every 16 pairs of exponentials in an unmasked chunk, this many run on
+// the FMA pipe (exp2_poly2) and the rest on the MUFU unit.
+constexpr int kPolyPairs = 4;
+
+__device__ __forceinline__ void exp2_chunk(float (&x)[32], bool masked) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-        float p2[2], q2[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int cc = col0 + 2 * e + h2;
-            float lse, gm, dl;
-            bool vis;
-            if (KEY_ROWS) {  // thread = key (global index key_or_t), column = row cc of the table
-                const RowRec x = recs[cc];  // one 16-byte shared-memory broadcast
-                lse = x.lse;
-                gm = x.gate;
-                dl = x.dlt;
-                vis = x.t >= 0 && key_or_t <= x.t;
-            } else {         // thread = row (position key_or_t), column = key kv0 + cc
-                lse = lse_or_row;
-                gm = gate_row;
-                dl = dlt_row;
-                vis = key_or_t >= 0 && kv0 + cc <= key_or_t;
-            }
-            const float x = __uint_as_float(s[2 * e + h2]) * c - lse;
-            const float p = vis ? fast_exp2(x) : 0.f;
-            p2[h2] = p * gm;
-            q2[h2] = p * (gm * __uint_as_float(dp[2 * e + h2]) - dl);
+        if (!masked && e < kPolyPairs) {
+            up2(exp2_poly2_clamped(x[2 * e], x[2 * e + 1]), x[2 * e], x[2 * e + 1]);
+        } else {
+            x[2 * e] = fast_exp2(x[2 * e]);
+            x[2 * e + 1] = fast_exp2(x[2 * e + 1]);
         }
-        pg[e] = pack_bf16x2(p2[0], p2[1]);
-        ds[e] = pack_bf16x2(q2[0], q2[1]);
+    }
+}
+
+// Exponent phase, thread = routed row: gp = 2^(s c - lse2) for 32 key columns
+// starting at key kv0 (masked: keys after the row's position t give 0).
+__device__ __forceinline__ void exp_row(const uint32_t (&s)[32], float c, float lse2, int t_row, int kv0, bool masked,
+                                        float (&gp)[32]) {
+    const float kNegInf = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const float x = __uint_as_float(s[e]) * c - lse2;
+        gp[e] = (masked && kv0 + e > t_row) ? kNegInf : x;
+    }
+    exp2_chunk(gp, masked);
+}
+
+// Exponent phase, thread = key: gp = 2^(s c - lse2) for 32 row columns starting
+// at column col0 of the table (masked: rows whose position t precedes the key,
+// or padding rows, give 0).
+__device__ __forceinline__ void exp_key(const uint32_t (&s)[32], float c, int key, const TileTab& tab, int col0,
+                                        bool masked, float (&gp)[32]) {
+    const float kNegInf = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 l = *reinterpret_cast<const float4*>(&tab.lse2[col0 + 4 * e4]);
+        gp[4 * e4 + 0] = __uint_as_float(s[4 * e4 + 0]) * c - l.x;
+        gp[4 * e4 + 1] = __uint_as_float(s[4 * e4 + 1]) * c - l.y;
+        gp[4 * e4 + 2] = __uint_as_float(s[4 * e4 + 2]) * c - l.z;
+        gp[4 * e4 + 3] = __uint_as_float(s[4 * e4 + 3]) * c - l.w;
+        if (masked) {
+            const int4 tv = *reinterpret_cast<const int4*>(&tab.t[col0 + 4 * e4]);
+            if (key > tv.x) gp[4 * e4 + 0] = kNegInf;
+            if (key > tv.y) gp[4 * e4 + 1] = kNegInf;
+            if (key > tv.z) gp[4 * e4 + 2] = kNegInf;
+            if (key > tv.w) gp[4 * e4 + 3] = kNegInf;
+        }
+    }
+    exp2_chunk(gp, masked);
+}
+
+__device__ __forceinline__ void pack_chunk(const float (&v)[32], uint32_t (&out)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) out[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+}
+
+// dS phase: ds = gp (dp - dl2), as bf16 pairs; dl2 the thread's row's (thread =
+// row) or per column from the table (thread = key, col0 >= 0).
+__device__ __forceinline__ void ds_row(const float (&gp)[32], const uint32_t (&dp)[32], float dl2,
+                                       uint32_t (&ds)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        ds[e] = pack_bf16x2(gp[2 * e] * (__uint_as_float(dp[2 * e]) - dl2),
+                            gp[2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - dl2));
+}
+__device__ __forceinline__ void ds_key(const float (&gp)[32], const uint32_t (&dp)[32], const TileTab& tab, int col0,
+                                       uint32_t (&ds)[16]) {
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 d = *reinterpret_cast<const float4*>(&tab.dl2[col0 + 4 * e4]);
+        ds[2 * e4] = pack_bf16x2(gp[4 * e4] * (__uint_as_float(dp[4 * e4]) - d.x),
+                                 gp[4 * e4 + 1] * (__uint_as_float(dp[4 * e4 + 1]) - d.y));
+        ds[2 * e4 + 1] = pack_bf16x2(gp[4 * e4 + 2] * (__uint_as_float(dp[4 * e4 + 2]) - d.z),
+                                     gp[4 * e4 + 3] * (__uint_as_float(dp[4 * e4 + 3]) - d.w));
     }
 }
 
@@ -334,7 +372,9 @@ __device__ __forceinline__ void ew_chunk(const uint32_t (&s)[32], const uint32_t
 // table + Q/dO gather, warps 4-11 elementwise + epilogue (thread = row, two
 // warps per row, one per 64-column half).  TMEM: S buffers [0,128) and
 // [128,256), dP [256,384), dQ [384,512); dS (bf16 pairs) overwrites dP's
-// columns a_col(0..7) once dP is in registers.
+// columns a_col(0..7) once dP is in registers.  Per key tile the elementwise
+// warps run the dS phase of tile i, then the exponent phase of tile i+1 (its
+// S is already in TMEM) while the tensor core runs dQ(i) and dP(i+1).
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dO[kTile];
@@ -377,7 +417,9 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             mbar_init(&sm.s_full[i], 1);
         }
         mbar_init(&sm.rows_full, 1);
-        mbar_init(&sm.rows_empty, 2);  // the MMA issuer (operands read) and the elementwise warps (table read)
+        // the MMA issuer's commit after the item's last dQ step, which follows every
+        // elementwise step of the item (and so every read of its table)
+        mbar_init(&sm.rows_empty, 1);
         mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.ew_done, 256);
         mbar_init(&sm.dq_full, 1);
@@ -400,7 +442,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         if (lane == 0) {
             uint32_t kv = 0;
             bool ok = true;
-            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x) {
+            for (int64_t v = 0, it = snake_item(0); it < n_items && ok && !aborted(&sm.abort_flag);
+                 it = snake_item(++v)) {
                 int b, q, w0, nkv;
                 int64_t tile;
                 dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
@@ -468,7 +511,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             auto wait_v = [&](uint32_t x) { return mbar_wait(&sm.kv_full_v[x & 1], (x >> 1) & 1); };
             uint32_t kv = 0, sc = 0, ec = 0, item_no = 0;  // kv tiles, S issued, elementwise steps, items
             bool ok = true;
-            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+            for (int64_t v = 0, it = snake_item(0); it < n_items && ok && !aborted(&sm.abort_flag);
+                 it = snake_item(++v), ++item_no) {
                 int b, q, w0, nkv;
                 int64_t tile;
                 dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
@@ -503,7 +547,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                     umma_commit(&sm.kv_empty_k[x & 1]);  // K(i): read by S(i) and dQ(i)
                     if (i == nkv - 1) {
                         umma_commit(&sm.dq_full);
-                        umma_commit(&sm.rows_empty);  // Q and dO of the item are no longer read
+                        umma_commit(&sm.rows_empty);  // Q, dO and the table of the item are no longer read
                     }
                     if (i + 1 < nkv) {
                         if (!(ok = wait_v(x + 1))) { fail(&sm.abort_flag, p.status, 16); break; }
@@ -527,7 +571,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         // ------------------------------------------------------------ row table + Q / dO gather
         uint32_t item_no = 0;
         bool armed = false;
-        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+        for (int64_t v = 0, it = snake_item(0); it < n_items && !aborted(&sm.abort_flag);
+             it = snake_item(++v), ++item_no) {
             int b, q, w0, nkv;
             int64_t tile;
             dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
@@ -536,7 +581,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 if (lane == 0) fail(&sm.abort_flag, p.status, 20);
                 break;
             }
-            load_tab(p.rec + tile * kBM, p.jtab + tile * kBM, sm.tab);
+            load_tab(p.tabs + tile, sm.tab);
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.rows_full, 2 * kTile);
@@ -551,13 +596,15 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
         if (armed) mbar_wait(&sm.rows_full, (item_no - 1) & 1);
     } else if (warp >= 4) {
         // ------------------------------------------------------------ elementwise + epilogue (thread = row)
-        // Warps 4-7 take columns 0-63 of their rows, warps 8-11 columns 64-127.
+        // Warps 4-7 take key columns 0-63 of their rows, warps 8-11 columns 64-127.
         const int wq = warp & 3;
         const int hh = (warp - 4) >> 2;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        uint32_t sc = 0, item_no = 0;
-        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++item_no) {
+        const uint32_t d_addr = tmem + lane_off + 256 + hh * 64;
+        uint32_t sc = 0, dc = 0, item_no = 0;
+        for (int64_t v = 0, it = snake_item(0); it < n_items && !aborted(&sm.abort_flag);
+             it = snake_item(++v), ++item_no) {
             int b, q, w0, nkv;
             int64_t tile;
             dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
@@ -565,35 +612,52 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 if (lane == 0) fail(&sm.abort_flag, p.status, 30);
                 break;
             }
-            const RowRec rr = sm.tab.rec[r];
-            const int t_row = rr.t;
-            const float lse = rr.lse, gm = rr.gate, dl = rr.dlt;
-            const int j_row = sm.tab.j[r];
+            const int t_row = sm.tab.t[r], j_row = sm.tab.j[r];
+            const float lse2 = sm.tab.lse2[r], dl2 = sm.tab.dl2[r];
+            float gp0[32], gp1[32];
             bool ok = true;
-            for (int i = 0; i < nkv; ++i, ++sc) {
-                const uint32_t sb = sc & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (sc >> 1) & 1) &&
-                                                 mbar_wait(&sm.dp_full, sc & 1))) {
-                    if (lane == 0) fail(&sm.abort_flag, p.status, 31);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t s_addr = tmem + lane_off + sb * 128, d_addr = tmem + lane_off + 256;
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    // chunk cb's bf16 pairs land on columns this warp has already read
-                    uint32_t sv[32], dv[32], pg[16], ds[16];
-                    tmem_ld32(s_addr + hh * 64 + cb * 32, sv);
-                    tmem_ld32(d_addr + hh * 64 + cb * 32, dv);
+            for (int i = 0; i <= nkv; ++i) {
+                if (i > 0) {
+                    // dS phase of key tile i - 1: dS pairs over dP's columns a_col
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.dp_full, dc & 1))) {
+                        if (lane == 0) fail(&sm.abort_flag, p.status, 32);
+                        ok = false;
+                        break;
+                    }
+                    ++dc;
+                    tc_fence_after();
+                    uint32_t d0[32], d1[32], ds[16];
+                    tmem_ld32(d_addr, d0);
+                    tmem_ld32(d_addr + 32, d1);
                     tmem_ld_wait();
-                    ew_chunk<false>(sv, dv, p.scale_log2, lse, gm, dl, t_row, sm.tab.rec, hh * 64 + cb * 32, i * kBM,
-                                    pg, ds);
-                    tmem_st16(d_addr + hh * 64 + cb * 16, ds);
+                    ds_row(gp0, d0, dl2, ds);
+                    tmem_st16(d_addr, ds);
+                    ds_row(gp1, d1, dl2, ds);
+                    tmem_st16(d_addr + 16, ds);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&sm.ew_done);
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.ew_done);
+                if (i < nkv) {
+                    // exponent phase of key tile i (S buffer sc & 1)
+                    const uint32_t sb = sc & 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (sc >> 1) & 1))) {
+                        if (lane == 0) fail(&sm.abort_flag, p.status, 31);
+                        ok = false;
+                        break;
+                    }
+                    ++sc;
+                    tc_fence_after();
+                    const uint32_t s_addr = tmem + lane_off + sb * 128 + hh * 64;
+                    uint32_t s0[32], s1[32];
+                    tmem_ld32(s_addr, s0);
+                    tmem_ld32(s_addr + 32, s1);
+                    tmem_ld_wait();
+                    const bool masked = (i + 1) * kBM > w0;  // the key tile reaches the tile's first position
+                    const int kv0 = i * kBM + hh * 64;
+                    exp_row(s0, p.scale_log2, lse2, t_row, kv0, masked, gp0);
+                    exp_row(s1, p.scale_log2, lse2, t_row, kv0 + 32, masked, gp1);
+                }
             }
             if (!ok) break;
             // epilogue: dQ = (sum_s dS k_s) / sqrt(d), fp32 rows of the routed heads
@@ -614,16 +678,14 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 if (row_ok) {
                     float4* dst = reinterpret_cast<float4*>(drow + cb * 32);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        dst[v] = make_float4(__uint_as_float(o[4 * v]) * p.scale, __uint_as_float(o[4 * v + 1]) * p.scale,
-                                             __uint_as_float(o[4 * v + 2]) * p.scale,
-                                             __uint_as_float(o[4 * v + 3]) * p.scale);
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(o[4 * e]) * p.scale, __uint_as_float(o[4 * e + 1]) * p.scale,
+                                             __uint_as_float(o[4 * e + 2]) * p.scale,
+                                             __uint_as_float(o[4 * e + 3]) * p.scale);
                 }
             }
             tc_fence_before();
             mbar_arrive(&sm.dq_empty);
-            if (warp == 4 && lane == 0) mbar_arrive(&sm.rows_empty);  // this item's table is no longer read
-            // (the MMA issuer's rows_empty commit follows every elementwise step of the item)
         }
     }
     __syncwarp();
@@ -642,14 +704,17 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
 // Q/dO gather (double buffered), warps 4-11 elementwise + epilogue (thread =
 // key, two warps per key, one per 64-column half).  TMEM: dK [0,128), dV
 // [128,256), S^T [256,384), dP^T [384,512); g p and dS (bf16 pairs) overwrite
-// the columns a_col(0..7) of S^T and dP^T.
+// the columns a_col(0..7) of S^T and dP^T.  Per row tile i the tensor core runs
+// dV(i), S^T(i+1), dK(i), dP^T(i+1): the exponent phase of tile i+1 overlaps
+// dK(i) and dP^T(i+1), the dS phase of tile i overlaps dV(i) and S^T(i+1).
 struct KvSmem {
     uint8_t k[kTile];
     uint8_t v[kTile];
     uint8_t q[2][kTile];
     uint8_t dO[2][kTile];
     TileTab tab[2];
-    uint64_t kv_full, kv_empty, rows_full[2], rows_empty[2], st_full, ew_done, acc_full, acc_empty, drain;
+    uint64_t kv_full, kv_empty, rows_full[2], rows_empty[2], st_full, dpt_full, exp_done, ds_done, acc_full,
+        acc_empty, drain;
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -681,10 +746,14 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         mbar_init(&sm.kv_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.rows_full[i], 1);
-            mbar_init(&sm.rows_empty[i], 2);  // MMA issuer (operands) and elementwise warps (table)
+            // the MMA issuer's commit after dK of the tile, which follows both
+            // elementwise phases of the tile (and so every read of its table)
+            mbar_init(&sm.rows_empty[i], 1);
         }
         mbar_init(&sm.st_full, 1);
-        mbar_init(&sm.ew_done, 256);
+        mbar_init(&sm.dpt_full, 1);
+        mbar_init(&sm.exp_done, 256);
+        mbar_init(&sm.ds_done, 256);
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.acc_empty, 256);
         mbar_init(&sm.drain, 1);
@@ -704,7 +773,8 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         // ------------------------------------------------------------ K/V of each item
         if (lane == 0) {
             uint32_t n = 0;
-            for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+            for (int64_t v = 0, it = snake_item(0); it < n_items && !aborted(&sm.abort_flag);
+                 it = snake_item(++v), ++n) {
                 int b, q, kt, tile0, ntiles;
                 kv_item(u, it, b, q, kt, tile0, ntiles);
                 if (!mbar_wait(&sm.kv_empty, (n & 1) ^ 1)) { fail(&sm.abort_flag, p.status, 101); break; }
@@ -728,43 +798,69 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             const uint32_t buf_step = kTile >> 4;  // the second Q / dO buffer, in 16-byte units
             const uint32_t c_dk = tmem, c_dv = tmem + 128, c_st = tmem + 256, c_dpt = tmem + 384;
             auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
+            auto issue_st = [&](uint32_t rb) {  // S^T = K . Q^T
+                const uint32_t qb = qlo0 + rb * buf_step;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                    umma_ss(c_st, desc(klo + off), desc(qb + off), idesc_ss, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.st_full);
+            };
+            auto issue_dpt = [&](uint32_t rb) {  // dP^T = V . dO^T
+                const uint32_t dob = dolo0 + rb * buf_step;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+                    umma_ss(c_dpt, desc(vlo + off), desc(dob + off), idesc_ss, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sm.dpt_full);
+            };
+            auto issue_acc = [&](uint32_t c_acc, uint32_t c_a, uint32_t mlo, bool first) {  // (+)= A . B
+#pragma unroll
+                for (int kk = 0; kk < kBM / 16; ++kk)
+                    umma_ts(c_acc, c_a + a_col(kk), desc(mlo + (uint32_t)((kk * 2048) >> 4)), idesc_acc,
+                            (first && kk == 0) ? 0u : 1u);
+            };
             uint32_t n = 0, rc = 0;  // items, row tiles
             bool ok = true;
-            for (int64_t it = blockIdx.x; it < n_items && ok && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+            for (int64_t v = 0, it = snake_item(0); it < n_items && ok && !aborted(&sm.abort_flag);
+                 it = snake_item(++v), ++n) {
                 int b, q, kt, tile0, ntiles;
                 kv_item(u, it, b, q, kt, tile0, ntiles);
                 if (!mbar_wait(&sm.kv_full, n & 1)) { fail(&sm.abort_flag, p.status, 110); break; }
-                if (!mbar_wait(&sm.acc_empty, (n & 1) ^ 1)) { fail(&sm.abort_flag, p.status, 111); break; }
+                if (!mbar_wait(&sm.rows_full[rc & 1], (rc >> 1) & 1)) { fail(&sm.abort_flag, p.status, 112); break; }
                 tc_fence_after();
+                issue_st(rc & 1);
+                issue_dpt(rc & 1);
+                if (ntiles == 1) umma_commit(&sm.kv_empty);  // K and V are read by S^T and dP^T only
                 for (int i = 0; i < ntiles; ++i, ++rc) {
-                    const uint32_t rb = rc & 1;
-                    if (!(ok = mbar_wait(&sm.rows_full[rb], (rc >> 1) & 1))) { fail(&sm.abort_flag, p.status, 112); break; }
+                    const uint32_t rb = rc & 1, rb1 = (rc + 1) & 1;
+                    if (!(ok = mbar_wait(&sm.exp_done, rc & 1))) { fail(&sm.abort_flag, p.status, 113); break; }
+                    if (i == 0 && !(ok = mbar_wait(&sm.acc_empty, (n & 1) ^ 1))) {
+                        fail(&sm.abort_flag, p.status, 111);
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t qb = qlo0 + rb * buf_step, dob = dolo0 + rb * buf_step;
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {  // S^T = K . Q^T
-                        const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
-                        umma_ss(c_st, desc(klo + off), desc(qb + off), idesc_ss, kk > 0 ? 1u : 0u);
+                    issue_acc(c_dv, c_st, domlo0 + rb * buf_step, i == 0);  // dV += (g p)^T . dO
+                    if (i + 1 < ntiles) {
+                        if (!(ok = mbar_wait(&sm.rows_full[rb1], ((rc + 1) >> 1) & 1))) {
+                            fail(&sm.abort_flag, p.status, 114);
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_st(rb1);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {  // dP^T = V . dO^T
-                        const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
-                        umma_ss(c_dpt, desc(vlo + off), desc(dob + off), idesc_ss, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sm.st_full);
-                    if (!(ok = mbar_wait(&sm.ew_done, rc & 1))) { fail(&sm.abort_flag, p.status, 113); break; }
+                    if (!(ok = mbar_wait(&sm.ds_done, rc & 1))) { fail(&sm.abort_flag, p.status, 115); break; }
                     tc_fence_after();
-                    const uint32_t qmb = qmlo0 + rb * buf_step, domb = domlo0 + rb * buf_step;
-#pragma unroll
-                    for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += (g p)^T . dO ; dK += dS^T . Q
-                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                        umma_ts(c_dv, c_st + a_col(kk), desc(domb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
-                        umma_ts(c_dk, c_dpt + a_col(kk), desc(qmb + (uint32_t)((kk * 2048) >> 4)), idesc_acc, acc);
-                    }
+                    issue_acc(c_dk, c_dpt, qmlo0 + rb * buf_step, i == 0);  // dK += dS^T . Q
                     umma_commit(&sm.rows_empty[rb]);
+                    if (i + 1 < ntiles) {
+                        issue_dpt(rb1);
+                        if (i + 2 == ntiles) umma_commit(&sm.kv_empty);
+                    }
                 }
                 if (!ok) break;
-                umma_commit(&sm.kv_empty);
                 umma_commit(&sm.acc_full);
             }
             umma_commit(&sm.drain);
@@ -774,7 +870,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         // ------------------------------------------------------------ row tables + Q / dO gather
         uint32_t rc = 0;
         int64_t armed = -1;
-        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x) {
+        for (int64_t v = 0, it = snake_item(0); it < n_items && !aborted(&sm.abort_flag); it = snake_item(++v)) {
             int b, q, kt, tile0, ntiles;
             kv_item(u, it, b, q, kt, tile0, ntiles);
             bool ok = true;
@@ -786,7 +882,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     break;
                 }
                 const int64_t tile = ((int64_t)b * u.g + q) * p.ntiles + (tile0 + i);
-                load_tab(p.rec + tile * kBM, p.jtab + tile * kBM, sm.tab[rb]);
+                load_tab(p.tabs + tile, sm.tab[rb]);
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&sm.rows_full[rb], 2 * kTile);
@@ -808,37 +904,62 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         const int hh = (warp - 4) >> 2;
         const int kr = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t st_addr = tmem + lane_off + 256, dpt_addr = tmem + lane_off + 384;
+        const uint32_t st_addr = tmem + lane_off + 256 + hh * 64, dpt_addr = tmem + lane_off + 384 + hh * 64;
+        const int col0 = hh * 64;
         uint32_t n = 0, rc = 0;
-        for (int64_t it = blockIdx.x; it < n_items && !aborted(&sm.abort_flag); it += gridDim.x, ++n) {
+        for (int64_t v = 0, it = snake_item(0); it < n_items && !aborted(&sm.abort_flag);
+             it = snake_item(++v), ++n) {
             int b, q, kt, tile0, ntiles;
             kv_item(u, it, b, q, kt, tile0, ntiles);
             const int key = kt * kBM + kr;
             bool ok = true;
             for (int i = 0; i < ntiles; ++i, ++rc) {
-                const uint32_t rb = rc & 1;
+                const TileTab& tab = sm.tab[rc & 1];
+                // the tile's first position lies before the key tile's end
+                const bool masked = (tile0 + i) * u.W < (kt + 1) * kBM;
+                // exponent phase: g p, kept in fp32, and as bf16 pairs over S^T's columns a_col
                 if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full, rc & 1))) {
                     if (lane == 0) fail(&sm.abort_flag, p.status, 130);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const RowRec* recs = sm.tab[rb].rec;
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    // chunk cb's bf16 pairs land on columns this warp has already read
-                    uint32_t sv[32], dv[32], pg[16], ds[16];
-                    tmem_ld32(st_addr + hh * 64 + cb * 32, sv);
-                    tmem_ld32(dpt_addr + hh * 64 + cb * 32, dv);
+                float gp0[32], gp1[32];
+                {
+                    uint32_t s0[32], s1[32], pk[16];
+                    tmem_ld32(st_addr, s0);
+                    tmem_ld32(st_addr + 32, s1);
                     tmem_ld_wait();
-                    ew_chunk<true>(sv, dv, p.scale_log2, 0.f, 0.f, 0.f, key, recs, hh * 64 + cb * 32, 0, pg, ds);
-                    tmem_st16(st_addr + hh * 64 + cb * 16, pg);
-                    tmem_st16(dpt_addr + hh * 64 + cb * 16, ds);
+                    exp_key(s0, p.scale_log2, key, tab, col0, masked, gp0);
+                    pack_chunk(gp0, pk);
+                    tmem_st16(st_addr, pk);
+                    exp_key(s1, p.scale_log2, key, tab, col0 + 32, masked, gp1);
+                    pack_chunk(gp1, pk);
+                    tmem_st16(st_addr + 16, pk);
+                    tmem_st_wait();
                 }
-                tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sm.ew_done);
-                if (warp == 4 && lane == 0) mbar_arrive(&sm.rows_empty[rb]);  // the table is no longer read
+                mbar_arrive(&sm.exp_done);
+                // dS phase: bf16 pairs over dP^T's columns a_col
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.dpt_full, rc & 1))) {
+                    if (lane == 0) fail(&sm.abort_flag, p.status, 131);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                {
+                    uint32_t d0[32], d1[32], ds[16];
+                    tmem_ld32(dpt_addr, d0);
+                    tmem_ld32(dpt_addr + 32, d1);
+                    tmem_ld_wait();
+                    ds_key(gp0, d0, tab, col0, ds);
+                    tmem_st16(dpt_addr, ds);
+                    ds_key(gp1, d1, tab, col0 + 32, ds);
+                    tmem_st16(dpt_addr + 16, ds);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.ds_done);
             }
             if (!ok) break;
             // epilogue: dK (scaled by 1/sqrt(d)) and dV rows of the item's keys
@@ -861,9 +982,9 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     if (key_ok) {
                         float4* dst = reinterpret_cast<float4*>(dst_row + cb * 32);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * f, __uint_as_float(o[4 * v + 1]) * f,
-                                                 __uint_as_float(o[4 * v + 2]) * f, __uint_as_float(o[4 * v + 3]) * f);
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(o[4 * e]) * f, __uint_as_float(o[4 * e + 1]) * f,
+                                                 __uint_as_float(o[4 * e + 2]) * f, __uint_as_float(o[4 * e + 3]) * f);
                     }
                 }
             }
@@ -889,11 +1010,12 @@ bool attn_backward_tc_supported(const gqe_shape* s) {
 }
 
 namespace {
-// Workspace of the tensor-core backward: gate, D and lse planes [B*T*h] (fp32),
-// o [B*T*h, 128] (fp32), then the packed tiles: records and heads
-// [tiles * 128] and the rows of Q and dO [tiles * 128, 128] (bf16).
+// Workspace of the tensor-core backward: the lse plane [B*T*h] and o
+// [B*T*h, 128] (fp32) that the forward recompute writes when the training
+// forward's are not given, then the packed tiles: tables [tiles] and the rows
+// of Q and dO [tiles * 128, 128] (bf16).
 struct BwdLayout {
-    size_t plane, o32, rec, jtab, rows, total;
+    size_t plane, o32, tabs, rows, total;
     int64_t ntiles, tiles;
 };
 BwdLayout bwd_layout(const gqe_shape* s) {
@@ -906,10 +1028,9 @@ BwdLayout bwd_layout(const gqe_shape* s) {
     L.tiles = (int64_t)s->B * s->g * L.ntiles;
     L.plane = a256(bth * sizeof(float));
     L.o32 = a256(bth * kD * sizeof(float));
-    L.rec = a256((size_t)L.tiles * kBM * sizeof(RowRec));
-    L.jtab = a256((size_t)L.tiles * kBM * sizeof(int32_t));
+    L.tabs = a256((size_t)L.tiles * sizeof(TileTab));
     L.rows = a256((size_t)L.tiles * kBM * kD * 2);
-    L.total = 3 * L.plane + L.o32 + L.rec + L.jtab + 2 * L.rows;
+    L.total = L.plane + L.o32 + L.tabs + 2 * L.rows;
     return L;
 }
 }  // namespace
@@ -921,17 +1042,14 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     const int64_t BT = (int64_t)s.B * s.T;
     const BwdLayout L = bwd_layout(a.s);
     char* base = static_cast<char*>(a.scratch);
-    float* gamma = reinterpret_cast<float*>(base);
-    float* delta = reinterpret_cast<float*>(base + L.plane);
-    float* lse_ws = reinterpret_cast<float*>(base + 2 * L.plane);
-    float* o32_ws = reinterpret_cast<float*>(base + 3 * L.plane);
+    float* lse_ws = reinterpret_cast<float*>(base);
+    float* o32_ws = reinterpret_cast<float*>(base + L.plane);
     const bool saved = a.o32 != nullptr && a.lse != nullptr;
     const float* lse = saved ? a.lse : lse_ws;
     const float* o32 = saved ? a.o32 : o32_ws;
-    RowRec* rec = reinterpret_cast<RowRec*>(base + 3 * L.plane + L.o32);
-    int32_t* jtab = reinterpret_cast<int32_t*>(base + 3 * L.plane + L.o32 + L.rec);
-    __nv_bfloat16* Qc = reinterpret_cast<__nv_bfloat16*>(base + 3 * L.plane + L.o32 + L.rec + L.jtab);
-    __nv_bfloat16* dOc = reinterpret_cast<__nv_bfloat16*>(base + 3 * L.plane + L.o32 + L.rec + L.jtab + L.rows);
+    TileTab* tabs = reinterpret_cast<TileTab*>(base + L.plane + L.o32);
+    __nv_bfloat16* Qc = reinterpret_cast<__nv_bfloat16*>(base + L.plane + L.o32 + L.tabs);
+    __nv_bfloat16* dOc = reinterpret_cast<__nv_bfloat16*>(base + L.plane + L.o32 + L.tabs + L.rows);
     const int64_t rows_total = L.tiles * kBM;
     if (rows_total >= ((int64_t)1 << 31) - 1 || BT * s.h >= ((int64_t)1 << 31) - 1) return cudaErrorNotSupported;
 
@@ -960,14 +1078,6 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
         if (e != cudaSuccess) return e;
     }
 
-    // 1. D, gates, logit gradients, zero dQ of unselected heads
-    const int64_t warps = BT * s.g;
-    bwd_prep_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, a.stream>>>(
-        BT, s.h, s.g, s.k, a.idx, a.gate, (const __nv_bfloat16*)a.dO, o32, gamma, delta, a.dlogits, a.dQ,
-        (uint32_t*)a.status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-
     Params p;
     p.u.B = s.B;
     p.u.T = s.T;
@@ -983,10 +1093,7 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     p.head_offsets = a.head_offsets;
     p.head_pos = a.head_pos;
     p.head_chunk_offsets = a.head_chunk_offsets;
-    p.lse = lse;
-    p.dlt = delta;
-    p.rec = rec;
-    p.jtab = jtab;
+    p.tabs = tabs;
     p.ntiles = (int)L.ntiles;
     p.dQ = a.dQ;
     p.dK = a.dK;
@@ -996,10 +1103,11 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a) {
     p.scale = 1.0f / sqrtf((float)kD);
     p.q_rows = (int)(BT * s.h);
 
-    // 1b. packed tiles (tables, Q and dO rows)
-    bwd_tiles_kernel<<<(unsigned)((L.tiles + 3) / 4), 128, 0, a.stream>>>(
-        p.u, p.ntiles, a.head_offsets, a.head_chunk_offsets, a.head_pos, a.idx, a.gate, lse, delta,
-        (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.dO, rec, jtab, Qc, dOc, (uint32_t*)a.status);
+    // 1. packed tiles (tables, Q and dO rows), logit gradients, dQ of unselected heads
+    bwd_pack_kernel<<<(unsigned)L.tiles, kPackThreads, 0, a.stream>>>(
+        p.u, p.ntiles, a.head_offsets, a.head_chunk_offsets, a.head_pos, a.idx, a.gate, lse, o32,
+        (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.dO, tabs, Qc, dOc, a.dlogits, a.dQ,
+        (uint32_t*)a.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 

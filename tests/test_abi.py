@@ -165,14 +165,13 @@ def test_attn_backward_validation():
     # scratch (gate, D, lse per (b,t,j)) and the router's dW_r partials
     s32 = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_F32)
     assert g.gqe_backward_workspace_bytes(s32) == 256 + max(3 * 2 * 64 * 8 * 4, 64 * 128 * 8 * 4)
-    # bf16 with d_h = 128 (tensor-core backward): the gate, D and lse planes, the
-    # rows' fp32 outputs, then the packed half-window tiles (2*ceil(T/2W) per
-    # (b, group), W = 64 for k = 2): 16-byte row records, heads, Q and dO rows
+    # bf16 with d_h = 128 (tensor-core backward): the lse plane and the rows'
+    # fp32 outputs of the forward recompute, then the packed half-window tiles
+    # (2*ceil(T/2W) per (b, group), W = 64 for k = 2): 2 KB tables, Q and dO rows
     s = g.make_shape(2, 64, 128, 8, 2, 128, 2, g.GQE_BF16)
     need = g.gqe_backward_workspace_bytes(s)
     bth, tiles = 2 * 64 * 8, 2 * 2 * 2
-    attn = 3 * a256(bth * 4) + a256(bth * 128 * 4) + a256(tiles * 128 * 16) + a256(tiles * 128 * 4) \
-        + 2 * a256(tiles * 128 * 128 * 2)
+    attn = a256(bth * 4) + a256(bth * 128 * 4) + a256(tiles * 2048) + 2 * a256(tiles * 128 * 128 * 2)
     assert need == 256 + max(attn, 64 * 128 * 8 * 4)
     call = lambda s, dQ, ws_bytes: g._lib.gqe_attn_prefill_backward(
         ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake, fake, dQ, fake, fake, fake, fake,
