@@ -291,10 +291,12 @@ __device__ __forceinline__ int64_t snake_item(int64_t v) {
 // the FMA pipe (exp2_poly2) and the rest on the MUFU unit.
 constexpr int kPolyPairs = 4;
 
-__device__ __forceinline__ void exp2_chunk(float (&x)[32], bool masked) {
+// The chunk's masked form (a tile on the causal diagonal) runs all on MUFU.
+template <bool MASKED>
+__device__ __forceinline__ void exp2_chunk(float (&x)[32]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-        if (!masked && e < kPolyPairs) {
+        if (!MASKED && e < kPolyPairs) {
             up2(exp2_poly2_clamped(x[2 * e], x[2 * e + 1]), x[2 * e], x[2 * e + 1]);
         } else {
             x[2 * e] = fast_exp2(x[2 * e]);
@@ -304,23 +306,25 @@ __device__ __forceinline__ void exp2_chunk(float (&x)[32], bool masked) {
 }
 
 // Exponent phase, thread = routed row: gp = 2^(s c - lse2) for 32 key columns
-// starting at key kv0 (masked: keys after the row's position t give 0).
-__device__ __forceinline__ void exp_row(const uint32_t (&s)[32], float c, float lse2, int t_row, int kv0, bool masked,
+// starting at key kv0 (MASKED: keys after the row's position t give 0).
+template <bool MASKED>
+__device__ __forceinline__ void exp_row(const uint32_t (&s)[32], float c, float lse2, int t_row, int kv0,
                                         float (&gp)[32]) {
     const float kNegInf = -__int_as_float(0x7f800000);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const float x = __uint_as_float(s[e]) * c - lse2;
-        gp[e] = (masked && kv0 + e > t_row) ? kNegInf : x;
+        gp[e] = (MASKED && kv0 + e > t_row) ? kNegInf : x;
     }
-    exp2_chunk(gp, masked);
+    exp2_chunk<MASKED>(gp);
 }
 
 // Exponent phase, thread = key: gp = 2^(s c - lse2) for 32 row columns starting
-// at column col0 of the table (masked: rows whose position t precedes the key,
+// at column col0 of the table (MASKED: rows whose position t precedes the key,
 // or padding rows, give 0).
+template <bool MASKED>
 __device__ __forceinline__ void exp_key(const uint32_t (&s)[32], float c, int key, const TileTab& tab, int col0,
-                                        bool masked, float (&gp)[32]) {
+                                        float (&gp)[32]) {
     const float kNegInf = -__int_as_float(0x7f800000);
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
@@ -329,7 +333,7 @@ __device__ __forceinline__ void exp_key(const uint32_t (&s)[32], float c, int ke
         gp[4 * e4 + 1] = __uint_as_float(s[4 * e4 + 1]) * c - l.y;
         gp[4 * e4 + 2] = __uint_as_float(s[4 * e4 + 2]) * c - l.z;
         gp[4 * e4 + 3] = __uint_as_float(s[4 * e4 + 3]) * c - l.w;
-        if (masked) {
+        if (MASKED) {
             const int4 tv = *reinterpret_cast<const int4*>(&tab.t[col0 + 4 * e4]);
             if (key > tv.x) gp[4 * e4 + 0] = kNegInf;
             if (key > tv.y) gp[4 * e4 + 1] = kNegInf;
@@ -337,7 +341,7 @@ __device__ __forceinline__ void exp_key(const uint32_t (&s)[32], float c, int ke
             if (key > tv.w) gp[4 * e4 + 3] = kNegInf;
         }
     }
-    exp2_chunk(gp, masked);
+    exp2_chunk<MASKED>(gp);
 }
 
 __device__ __forceinline__ void pack_chunk(const float (&v)[32], uint32_t (&out)[16]) {
@@ -404,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
              const __grid_constant__ CUtensorMap mapQc, const __grid_constant__ CUtensorMap mapdOc, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    DqSmem& sm = *reinterpret_cast<DqSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DqSmem& sm = *smem_align1024<DqSmem>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const UnitGeom& u = p.u;
     const int64_t n_items = dq_items(u);
@@ -653,10 +657,14 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                     tmem_ld32(s_addr, s0);
                     tmem_ld32(s_addr + 32, s1);
                     tmem_ld_wait();
-                    const bool masked = (i + 1) * kBM > w0;  // the key tile reaches the tile's first position
                     const int kv0 = i * kBM + hh * 64;
-                    exp_row(s0, p.scale_log2, lse2, t_row, kv0, masked, gp0);
-                    exp_row(s1, p.scale_log2, lse2, t_row, kv0 + 32, masked, gp1);
+                    if ((i + 1) * kBM > w0) {  // the key tile reaches the tile's first position
+                        exp_row<true>(s0, p.scale_log2, lse2, t_row, kv0, gp0);
+                        exp_row<true>(s1, p.scale_log2, lse2, t_row, kv0 + 32, gp1);
+                    } else {
+                        exp_row<false>(s0, p.scale_log2, lse2, t_row, kv0, gp0);
+                        exp_row<false>(s1, p.scale_log2, lse2, t_row, kv0 + 32, gp1);
+                    }
                 }
             }
             if (!ok) break;
@@ -737,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                const __grid_constant__ CUtensorMap mapQc, const __grid_constant__ CUtensorMap mapdOc, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    KvSmem& sm = *reinterpret_cast<KvSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    KvSmem& sm = *smem_align1024<KvSmem>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const UnitGeom& u = p.u;
     const int64_t n_items = kv_items(u);
@@ -930,10 +938,15 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     tmem_ld32(st_addr, s0);
                     tmem_ld32(st_addr + 32, s1);
                     tmem_ld_wait();
-                    exp_key(s0, p.scale_log2, key, tab, col0, masked, gp0);
+                    if (masked) {
+                        exp_key<true>(s0, p.scale_log2, key, tab, col0, gp0);
+                        exp_key<true>(s1, p.scale_log2, key, tab, col0 + 32, gp1);
+                    } else {
+                        exp_key<false>(s0, p.scale_log2, key, tab, col0, gp0);
+                        exp_key<false>(s1, p.scale_log2, key, tab, col0 + 32, gp1);
+                    }
                     pack_chunk(gp0, pk);
                     tmem_st16(st_addr, pk);
-                    exp_key(s1, p.scale_log2, key, tab, col0 + 32, masked, gp1);
                     pack_chunk(gp1, pk);
                     tmem_st16(st_addr + 16, pk);
                     tmem_st_wait();

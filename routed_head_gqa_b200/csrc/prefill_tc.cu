@@ -142,7 +142,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                   const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQB,
                   const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem& sm = *smem_align1024<Smem>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const UnitGeom& u = p.u;
     const int64_t n_units = u.count();

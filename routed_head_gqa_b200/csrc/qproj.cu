@@ -79,7 +79,7 @@ qproj_kernel(const __grid_constant__ CUtensorMap mapXT, const __grid_constant__ 
     if (mb * kTiles * kM >= n) return;  // the whole CTA leaves before any barrier or TMEM use
 
     extern __shared__ uint8_t smem_raw[];
-    QprojSmem& sm = *reinterpret_cast<QprojSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    QprojSmem& sm = *smem_align1024<QprojSmem>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nk = (d_model + kTK - 1) / kTK;
 

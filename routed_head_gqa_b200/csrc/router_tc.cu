@@ -86,7 +86,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     using Smem = RouterSmem<NB>;
     constexpr int S = Smem::kStages;
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem& sm = *smem_align1024<Smem>(smem_raw);
     constexpr uint32_t kCols = 64 * NB;  // TMEM columns (power of two for NB in {1, 2, 4})
     constexpr int kRows = kTM / KS;      // rows of the tile whose top-k this CTA computes
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(128) umma_tile_kernel(const __grid_constant__ 
                                                         const __nv_bfloat16* __restrict__ A_global,
                                                         float* __restrict__ C, uint32_t* __restrict__ status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align1024<uint8_t>(smem_raw);
     uint8_t* sA = smem;                 // 2 x 16 KB
     uint8_t* sB = smem + 2 * kHalfBytes;  // 2 x 16 KB
     __shared__ __align__(8) uint64_t bar_load, bar_mma;

@@ -15,6 +15,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned address in a dynamic shared-memory buffer, by
+// plain pointer arithmetic (no round trip through an integer), so that the
+// compiler still knows the result points to shared memory and emits shared
+// loads and stores for the accesses through it.
+template <typename T>
+__device__ __forceinline__ T* smem_align1024(uint8_t* raw) {
+    return reinterpret_cast<T*>(raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u));
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
