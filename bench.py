@@ -785,6 +785,7 @@ def main():
                               "shared_head_frac": extras["layer_ops"]["shared_head"]["roofline"]["frac"],
                               "group_slots_frac": extras["layer_ops"]["group_slots"]["roofline"]["frac"],
                               "backward_ms": round(extras["backward"]["ms"], 3),
+                              "backward_frac": extras["backward"]["roofline"]["frac"],
                               "route_backward_ms": round(extras["backward"]["router"]["ms"], 4)}
         print(json.dumps(line))
     if ws > 1:
