@@ -102,13 +102,14 @@ class Oracle:
         lib.oracle_group_slots_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P, P,
                                                 i32]
         lib.oracle_qproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
+        lib.oracle_oproj_rows.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P, i32]
         lib.oracle_decode_paged.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32]
         lib.oracle_attn_backward.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P,
                                              i32]
         lib.oracle_route_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, i32]
         lib.oracle_aux_loss.argtypes = [i64, i32, i32, i32, P, P, P, P]
         for f in (lib.oracle_aux_loss, lib.oracle_route, lib.oracle_compact, lib.oracle_attn_rows, lib.oracle_decode,
-                  lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows,
+                  lib.oracle_shared_rows, lib.oracle_group_slots_rows, lib.oracle_qproj_rows, lib.oracle_oproj_rows,
                   lib.oracle_decode_paged, lib.oracle_attn_backward, lib.oracle_route_backward):
             f.restype = ctypes.c_int
         self.lib = lib
@@ -242,6 +243,30 @@ class Oracle:
                                         ra.shape[0], _ptr(ra), _ptr(out), _threads(n_threads))
         if rc:
             raise ValueError(f"oracle_qproj_rows failed ({rc})")
+        return out
+
+    def oproj_rows(self, O, W_Z, idx, rows=None, n_threads=None):
+        """Routed output projection (float64 [n_rows, d_model]) of token rows
+        b*T + t: the sum over the token's selected heads j = idx[b,t,q,r] of
+        O[b,t,j,:] . W_Z[j*d_h:(j+1)*d_h, :]."""
+        oa, dt = _as_input(O)
+        wa, dw = _as_input(W_Z)
+        if dt != dw:
+            raise TypeError("O and W_Z must share a dtype")
+        B, T, h, d_h = oa.shape
+        ia = np.ascontiguousarray(idx, dtype=np.int32)
+        g, k = ia.shape[2], ia.shape[3]
+        if wa.ndim != 2 or wa.shape[0] != h * d_h:
+            raise ValueError("W_Z must be [h*d_h, d_model]")
+        d_model = wa.shape[1]
+        if rows is None:
+            rows = np.arange(B * T, dtype=np.int64)
+        ra = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+        out = np.empty((ra.shape[0], d_model), np.float64)
+        rc = self.lib.oracle_oproj_rows(B, T, d_model, h, g, d_h, k, dt, _ptr(oa), _ptr(wa), _ptr(ia),
+                                        ra.shape[0], _ptr(ra), _ptr(out), _threads(n_threads))
+        if rc:
+            raise ValueError(f"oracle_oproj_rows failed ({rc})")
         return out
 
     def decode_paged(self, q, K_pages, V_pages, block_table, lengths, idx, gate, n_threads=None):
@@ -405,6 +430,10 @@ def group_slots_rows(*a, **kw):
 
 def qproj_rows(*a, **kw):
     return default().qproj_rows(*a, **kw)
+
+
+def oproj_rows(*a, **kw):
+    return default().oproj_rows(*a, **kw)
 
 
 def decode_paged(*a, **kw):

@@ -51,6 +51,11 @@
  *    query-side computation is conditional on the routing): the query row of
  *    head j is x . W_Q[:, j*d_h : (j+1)*d_h], computed only for the heads a
  *    token selected.
+ *  - Output projection (IBM GQA page: the heads' outputs, concatenated, pass
+ *    through one more linear layer with weight matrix W_Z; GQE page,
+ *    "Activation Conditionnelle": only the selected experts are computed): the
+ *    layer output of a token is the sum, over the heads it selected, of the
+ *    head's (gated) output row times that head's d_h-row block of W_Z.
  *  - Backward (training; the pages state no formula for it): the gradients of
  *    the routed attention, of the gates and of the router's logits, x, W_r and
  *    bias, by the chain rule through the steps above in reverse order.
@@ -419,6 +424,45 @@ int oracle_qproj_rows(int B, int T, int d_model, int h, int g, int d_h, int k, i
                     out[c] = acc;
                 }
             }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Routed output projection for a list of token rows.
+ * O [B, T, h, d_h] (dtype): the gated routed output; W_Z [h*d_h, d_model]
+ * (dtype), head j's block is rows j*d_h .. j*d_h + d_h - 1; idx [B, T, g, k].
+ * Y_rows [n_rows, d_model] out (double):
+ *   Y[bt, n] = sum_q sum_r sum_c O[bt, j, c] * W_Z[j*d_h + c, n],  j = idx[bt, q, r],
+ * the selected heads only (an unselected head's slot does not enter).
+ */
+int oracle_oproj_rows(int B, int T, int d_model, int h, int g, int d_h, int k, int dtype,
+                      const void* O, const void* W_Z, const int32_t* idx,
+                      int64_t n_rows, const int64_t* rows, double* Y_rows, int n_threads) {
+    if (B < 0 || T < 1 || d_model < 1 || h < 1 || g < 1 || h % g != 0 || d_h < 1) return 1;
+    if (k < 1 || k > h / g) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * T) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int e = 0; e < g * k; ++e) {
+            const int j = idx[(size_t)rows[r] * g * k + e];
+            if (j < 0 || j >= h) return 1;
+        }
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t bt = rows[r];
+        double* out = Y_rows + (size_t)r * d_model;
+        for (int n = 0; n < d_model; ++n) {
+            double acc = 0.0;
+            for (int q = 0; q < g; ++q)
+                for (int s = 0; s < k; ++s) {
+                    const int jh = idx[((size_t)bt * g + q) * k + s];
+                    for (int c = 0; c < d_h; ++c)
+                        acc += load_elem(O, ((size_t)bt * h + jh) * d_h + c, dtype) *
+                               load_elem(W_Z, ((size_t)jh * d_h + c) * d_model + n, dtype);
+                }
+            out[n] = acc;
         }
     }
     return 0;

@@ -731,11 +731,58 @@ def check_aux_loss(o):
         assert abs(fd - dl.flat[i]) < 1e-7, f"aux dlogits[{i}]: fd {fd} vs {dl.flat[i]}"
 
 
+# --------------------------------------------------------------------------
+# Routed output projection
+# --------------------------------------------------------------------------
+
+def check_oproj(o):
+    """Block-identity W_Z (d_model = h*d_h): a token's output is its selected
+    heads' slots in place and zeros elsewhere, even where an unselected slot
+    holds values (only the selected experts enter); a one-hot O at one
+    element of a selected head returns that row of W_Z; with zeros in the
+    unselected slots the result is the dense product of the concatenated
+    heads with W_Z (numpy, fp64)."""
+    B, T, h, g, d, k = 2, 3, 4, 2, 4, 1
+    hpg = h // g
+    idx = np.zeros((B, T, g, k), np.int32)
+    for b in range(B):
+        for t in range(T):
+            for q_ in range(g):
+                idx[b, t, q_, 0] = q_ * hpg + (b + 2 * t + q_) % hpg
+    sel = np.zeros((B, T, h), bool)
+    for b in range(B):
+        for t in range(T):
+            sel[b, t, idx[b, t].ravel()] = True
+    O = _f32((B, T, h, d), 90)  # unselected slots deliberately non-zero
+    Y = o.oproj_rows(O, np.eye(h * d, dtype=np.float32), idx).reshape(B, T, h, d)
+    Od = O.astype(np.float64)
+    for b in range(B):
+        for t in range(T):
+            for j in range(h):
+                want = Od[b, t, j] if sel[b, t, j] else np.zeros(d)
+                assert np.array_equal(Y[b, t, j], want), f"identity W_Z ({b},{t},{j})"
+    # one-hot O at element c0 of token (1, 2)'s first selected head: that row of W_Z
+    d_model = 7
+    W = _f32((h * d, d_model), 91)
+    c0 = 3
+    O1 = np.zeros((B, T, h, d), np.float32)
+    j0 = int(idx[1, 2, 1, 0])
+    O1[1, 2, j0, c0] = 1.0
+    Y1 = o.oproj_rows(O1, W, idx).reshape(B, T, d_model)
+    assert np.array_equal(Y1[1, 2], W[j0 * d + c0].astype(np.float64)), "one-hot O picks a W_Z row"
+    assert not Y1[0].any() and not Y1[1, :2].any()
+    # zeros in the unselected slots: the dense product
+    Oz = np.where(sel[..., None], O, 0.0).astype(np.float32)
+    Yz = o.oproj_rows(Oz, W, idx).reshape(B, T, d_model)
+    dense = Oz.reshape(B, T, h * d).astype(np.float64) @ W.astype(np.float64)
+    assert np.allclose(Yz, dense, rtol=0, atol=1e-12), "dense product"
+
+
 ALL_CHECKS = [
     check_router_onehot, check_router_bruteforce, check_router_zero_weights, check_gates,
     check_compact, check_attn_sdpa, check_attn_closed_forms, check_mha_mqa,
     check_prefix_invariance, check_decode, check_group_map_golden, check_active_heads_golden,
     check_shared_head_closed_forms, check_group_slots, check_qproj, check_decode_paged,
     check_backward_sdpa_autograd, check_backward_finite_differences, check_backward_invariants,
-    check_aux_loss,
+    check_aux_loss, check_oproj,
 ]

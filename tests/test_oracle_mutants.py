@@ -39,6 +39,12 @@ MUTANTS = [
      "load_elem(W_Q, (size_t)i * ldw + (size_t)j + c, dtype);"),
     ("qproj_transposed_weight", "load_elem(W_Q, (size_t)i * ldw + (size_t)j * d_h + c, dtype);",
      "load_elem(W_Q, ((size_t)((size_t)j * d_h + c) * d_model + i) % ((size_t)d_model * ldw), dtype);"),
+    ("oproj_head_block_offset", "load_elem(W_Z, ((size_t)jh * d_h + c) * d_model + n, dtype);",
+     "load_elem(W_Z, ((size_t)jh + c) * d_model + n, dtype);"),
+    ("oproj_transposed_weight", "load_elem(W_Z, ((size_t)jh * d_h + c) * d_model + n, dtype);",
+     "load_elem(W_Z, ((size_t)n * h * d_h + (size_t)jh * d_h + c) % ((size_t)h * d_h * d_model), dtype);"),
+    ("oproj_unrouted_heads", "const int jh = idx[((size_t)bt * g + q) * k + s];",
+     "const int jh = q * (h / g) + s;"),
     ("paged_row_offset", "const size_t row = ((pg * page_size + (size_t)(s % page_size)) * g + q) * d_h;",
      "const size_t row = ((pg * page_size + (size_t)((s + 1) % page_size)) * g + q) * d_h;"),
     ("paged_block_lookup", "(size_t)block_table[(size_t)b * max_blocks + s / page_size];",
