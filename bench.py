@@ -357,6 +357,8 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
     Os = torch.empty((w.B, w.T, w.d_h), dtype=w.torch_dtype, device=dev)
     W_Q = gqe_synth.make_qproj_weight(w).to(dev)
     Qp = torch.empty((w.B, w.T, w.h, w.d_h), dtype=w.torch_dtype, device=dev)
+    W_Z = gqe_synth.make_oproj_weight(w).to(dev)
+    Y = torch.empty((w.B, w.T, w.d_model), dtype=w.torch_dtype, device=dev)
     cat = torch.empty((w.B, w.T, w.g, w.k, w.d_h), dtype=w.torch_dtype, device=dev)
     wsum = torch.empty((w.B, w.T, w.g, w.d_h), dtype=w.torch_dtype, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -368,7 +370,10 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
         g.gqe_group_slots(r.shape, r.buf.O, r.buf.idx, r.buf.gate, cat, wsum)
 
     def qproj():
-        g.gqe_routed_qproj(r.shape, r.d["x"], W_Q, r.buf.head_offsets, r.buf.head_pos, Qp, r.buf.workspace)
+        g.gqe_routed_qproj(r.shape, r.d["x"], W_Q, r.buf.idx, r.buf.head_offsets, r.buf.head_pos, Qp, r.buf.workspace)
+
+    def oproj():  # over the prefill's gated output (zeros in the unselected slots)
+        g.gqe_routed_oproj(r.shape, r.buf.O, r.buf.idx, W_Z, Y, r.buf.workspace)
 
     def timed(fn):
         for _ in range(warmup):
@@ -387,6 +392,7 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
     sh_ms = timed(shared)
     sl_ms = timed(slots)
     qp_ms = timed(qproj)
+    op_ms = timed(oproj)
     st = r.buf.status()
     if st != 0:
         raise RuntimeError(f"device status {g.gqe_status_string(st)} in the output construction")
@@ -396,6 +402,9 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
     sl_bytes = float(rows * w.d_h * el * 2 + w.B * w.T * w.g * w.d_h * el + rows * 8)  # O rows in, cat + wsum out
     qp_flops = 2.0 * w.d_model * w.d_h * rows  # routed rows only
     qp_tf = qp_flops / (qp_ms * 1e-3) * 1e-12
+    op_flops = 2.0 * w.d_model * w.d_h * rows  # the selected heads' rows only
+    op_dense = 2.0 * w.d_model * w.d_h * w.B * w.T * w.h  # every head slot, as a dense GEMM would
+    op_tf = op_flops / (op_ms * 1e-3) * 1e-12
     sh_tf = sh_flops / (sh_ms * 1e-3) * 1e-12
     sl_gbs = sl_bytes / (sl_ms * 1e-3) * 1e-9
     del r, flush
@@ -406,6 +415,13 @@ def time_layer_ops(w, steps, warmup, peaks, peak_kind):
                                       "unit": "TFLOP/s", "frac": round(qp_tf / peaks["bf16_tflops"], 4),
                                       "peak_source": f"bf16_tflops burst ({peak_kind})",
                                       "kernel": "gqe_routed_qproj (qproj_kernel)"}},
+        "routed_oproj": {"ms": op_ms, "value": op_tf, "unit": "TFLOP/s", "flops": op_flops,
+                         "roofline": {"bound": "tensor", "achieved": round(op_tf, 1), "peak": peaks["bf16_tflops"],
+                                      "unit": "TFLOP/s", "frac": round(op_tf / peaks["bf16_tflops"], 4),
+                                      "frac_of_dense_equivalent": round(op_dense / (op_ms * 1e-3) * 1e-12
+                                                                        / peaks["bf16_tflops"], 4),
+                                      "peak_source": f"bf16_tflops burst ({peak_kind})",
+                                      "kernel": "gqe_routed_oproj (oproj_kernel)"}},
         "shared_head": {"ms": sh_ms, "value": sh_tf, "unit": "TFLOP/s", "flops": sh_flops,
                         "roofline": {"bound": "tensor", "achieved": round(sh_tf, 1), "peak": peaks["bf16_tflops"],
                                      "unit": "TFLOP/s", "frac": round(sh_tf / peaks["bf16_tflops"], 4),
@@ -782,6 +798,7 @@ def main():
                     json.dump(extras, f)
             line["extras"] = {"paged_decode_frac": extras["paged_decode"]["roofline"]["frac"],
                               "qproj_frac": extras["layer_ops"]["routed_qproj"]["roofline"]["frac"],
+                              "oproj_frac": extras["layer_ops"]["routed_oproj"]["roofline"]["frac"],
                               "shared_head_frac": extras["layer_ops"]["shared_head"]["roofline"]["frac"],
                               "group_slots_frac": extras["layer_ops"]["group_slots"]["roofline"]["frac"],
                               "backward_ms": round(extras["backward"]["ms"], 3),

@@ -181,6 +181,41 @@ def make_qproj_weight(w: Workload):
     return _normal((w.d_model, w.h * w.d_h), gen, std=1.0 / math.sqrt(w.d_model)).to(w.torch_dtype)
 
 
+def make_oproj_weight(w: Workload):
+    """Output projection W_Z [h*d_h, d_model] ~ N(0, 1/sqrt(h*d_h)) in the
+    workload's dtype, from its own seeded generator (seed + 130363)."""
+    gen = torch.Generator().manual_seed(w.seed + 130363)
+    return _normal((w.h * w.d_h, w.d_model), gen, std=1.0 / math.sqrt(w.h * w.d_h)).to(w.torch_dtype)
+
+
+def make_random_routing(w: Workload, seed: int = 777, first_tile_fixed: bool = False):
+    """A seeded routing with the router's structure but no router: for every
+    (b, t, group q) k distinct heads of the group, drawn uniformly, as
+    idx int32 [B, T, g, k].  first_tile_fixed: the first 128 tokens all take
+    the group's first k heads (so a 128-token tile leaves heads unselected)."""
+    gen = torch.Generator().manual_seed(w.seed + seed)
+    hpg = w.h // w.g
+    keys = torch.rand((w.B * w.T, w.g, hpg), generator=gen)
+    pick = keys.argsort(dim=-1)[..., : w.k]
+    if first_tile_fixed:
+        pick[:128] = torch.arange(w.k)
+    idx = pick + (torch.arange(w.g) * hpg)[None, :, None]
+    return idx.to(torch.int32).reshape(w.B, w.T, w.g, w.k)
+
+
+def make_routed_output(w: Workload, idx, seed: int = 991):
+    """A stand-in for the gated routed output O [B, T, h, d_h]: N(0, 1/2) in
+    the slots idx selects and exactly zero in every other slot (the layout the
+    routed prefill writes), in the workload's dtype, from its own seeded
+    generator."""
+    gen = torch.Generator().manual_seed(w.seed + seed)
+    O = _normal((w.B, w.T, w.h, w.d_h), gen, std=0.5)
+    sel = torch.zeros((w.B * w.T, w.h), dtype=torch.bool)
+    sel.scatter_(1, torch.as_tensor(idx).reshape(w.B * w.T, -1).long(), True)
+    O[~sel.reshape(w.B, w.T, w.h)] = 0.0
+    return O.to(w.torch_dtype)
+
+
 def make_output_grad(w: Workload):
     """Incoming gradient dO [B,T,h,d_h] ~ N(0,1) in the workload's dtype (a
     stand-in for the gradient a training step would bring back), from its own

@@ -212,15 +212,52 @@ gqe_status gqe_attn_decode(const gqe_shape* s, const void* q, const void* K_cach
  *
  *   x [B, T, d_model]                  device bf16
  *   W_Q [d_model, h * d_h]             device bf16 (head j's block: columns j*d_h ..)
+ *   idx [B, T, g, k]                   device, 16-byte aligned, as written by gqe_route
  *   head_offsets, head_pos             device, exactly as written by gqe_route
  *   Q [B, T, h, d_h]                   device bf16, out (routed rows)
- *   workspace                          status word only (gqe_workspace_bytes)
+ *   workspace                          the status word; with gqe_workspace_bytes of
+ *                                      room, also 8 bytes per 128-token tile for the
+ *                                      dense path
+ * Two paths, same result.  When the routed share g*k/h is at least 3/10 (and
+ * h <= 64, and the workspace has the tile sets' room) a tiled GEMM over every
+ * token computes the heads of each 128-token x 2-head tile that holds a routed
+ * (t, j) and writes the routed rows only; otherwise a grouped GEMM runs over
+ * each head's routed rows, gathered.
  * Implemented cases: bf16, d_h = 128, d_model % 8 == 0; others return
  * GQE_ERR_UNSUPPORTED.
  */
-gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* head_offsets,
-                            const int32_t* head_pos, void* Q, void* workspace, size_t workspace_bytes,
-                            void* stream);
+gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* idx,
+                            const int32_t* head_offsets, const int32_t* head_pos, void* Q, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * gqe_routed_oproj -- output projection over the routed heads.
+ *
+ * The heads' outputs pass through one more linear layer, the output weight
+ * matrix W_Z (IBM GQA page, multi-head attention mechanics); under GQE only
+ * the selected experts are computed (gist.science summary, "Activation
+ * Conditionnelle"), so a token's output is the sum over the heads it selected:
+ *   Y[b,t,n] = sum_{q, r} sum_c O[b,t,j,c] * W_Z[j*d_h + c, n],   j = idx[b,t,q,r],
+ * accumulated in fp32 on the tensor cores in a fixed order (reproducible) and
+ * rounded to bf16.
+ *
+ *   O [B, T, h, d_h]       device bf16: the gated routed output as
+ *                          gqe_attn_prefill / gqe_attn_decode write it.  The
+ *                          unselected slots must hold zeros: a head that some
+ *                          token of a 128-token tile selected is multiplied in
+ *                          for the whole tile.
+ *   idx [B, T, g, k]       device, 16-byte aligned, as written by gqe_route (an
+ *                          index outside [0, h) is reported in the status word
+ *                          and ignored)
+ *   W_Z [h * d_h, d_model] device bf16 (head j's block: rows j*d_h ..)
+ *   Y [B, T, d_model]      device bf16, out
+ *   workspace              the status word and 8 bytes per 128-token tile
+ *                          (gqe_workspace_bytes covers it)
+ * Implemented cases: bf16, d_h % 64 == 0, h <= 64, d_model % 32 == 0; others
+ * return GQE_ERR_UNSUPPORTED.
+ */
+gqe_status gqe_routed_oproj(const gqe_shape* s, const void* O, const int32_t* idx, const void* W_Z, void* Y,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * gqe_attn_shared_head -- the always-active shared head of the GQE layer.

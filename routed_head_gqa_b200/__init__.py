@@ -29,7 +29,7 @@ GQE_BF16 = 1
 EXPORTED = ["gqe_chunk_count", "gqe_workspace_bytes", "gqe_workspace_init", "gqe_route", "gqe_route_static",
             "gqe_route_static_status",
             "gqe_attn_prefill", "gqe_attn_decode", "gqe_attn_decode_paged", "gqe_attn_shared_head",
-            "gqe_group_slots", "gqe_routed_qproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
+            "gqe_group_slots", "gqe_routed_qproj", "gqe_routed_oproj", "gqe_backward_workspace_bytes", "gqe_attn_prefill_backward",
             "gqe_route_backward", "gqe_route_train", "gqe_aux_loss_workspace_bytes", "gqe_aux_loss",
             "gqe_attn_prefill_train", "gqe_attn_prefill_backward_saved",
             "gqe_get_device_status", "gqe_status_string"]
@@ -73,7 +73,8 @@ def _load():
     lib.gqe_attn_decode.argtypes = [S, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_shared_head.argtypes = [S, _P, _P, _P, _I, _P, _P, _SZ, _P]
     lib.gqe_group_slots.argtypes = [S, _P, _P, _P, _P, _P, _P]
-    lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_routed_qproj.argtypes = [S, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.gqe_routed_oproj.argtypes = [S, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_attn_decode_paged.argtypes = [S, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]
     lib.gqe_backward_workspace_bytes.argtypes = [S]
     lib.gqe_backward_workspace_bytes.restype = _SZ
@@ -90,7 +91,8 @@ def _load():
     lib.gqe_status_string.restype = ctypes.c_char_p
     for f in ("gqe_workspace_init", "gqe_route", "gqe_route_static", "gqe_route_static_status",
               "gqe_attn_prefill", "gqe_attn_decode",
-              "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_attn_decode_paged",
+              "gqe_attn_shared_head", "gqe_group_slots", "gqe_routed_qproj", "gqe_routed_oproj",
+              "gqe_attn_decode_paged",
               "gqe_attn_prefill_backward", "gqe_route_backward", "gqe_get_device_status", "gqe_route_train",
               "gqe_aux_loss", "gqe_attn_prefill_train", "gqe_attn_prefill_backward_saved"):
         getattr(lib, f).restype = _I
@@ -227,10 +229,15 @@ def gqe_attn_decode_paged(shape, q, K_pages, V_pages, page_size, block_table, le
         _stream(stream)))
 
 
-def gqe_routed_qproj(shape, x, W_Q, head_offsets, head_pos, Q, workspace, stream=None) -> None:
-    _check("gqe_routed_qproj", _lib.gqe_routed_qproj(ctypes.byref(shape), _ptr(x), _ptr(W_Q), _ptr(head_offsets),
-                                                     _ptr(head_pos), _ptr(Q), _ptr(workspace), _nbytes(workspace),
-                                                     _stream(stream)))
+def gqe_routed_qproj(shape, x, W_Q, idx, head_offsets, head_pos, Q, workspace, stream=None) -> None:
+    _check("gqe_routed_qproj", _lib.gqe_routed_qproj(ctypes.byref(shape), _ptr(x), _ptr(W_Q), _ptr(idx),
+                                                     _ptr(head_offsets), _ptr(head_pos), _ptr(Q), _ptr(workspace),
+                                                     _nbytes(workspace), _stream(stream)))
+
+
+def gqe_routed_oproj(shape, O, idx, W_Z, Y, workspace, stream=None) -> None:
+    _check("gqe_routed_oproj", _lib.gqe_routed_oproj(ctypes.byref(shape), _ptr(O), _ptr(idx), _ptr(W_Z), _ptr(Y),
+                                                     _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 def gqe_group_slots(shape, O, idx, gate, O_cat, O_wsum, stream=None) -> None:

@@ -22,7 +22,7 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", 
          "--expt-relaxed-constexpr", "-I", os.path.join(os.path.dirname(PKG), "include")]
 
 LIB_SOURCES = ["gqe_api.cu", "router.cu", "router_tc.cu", "prefill_simt.cu", "prefill_tc.cu", "decode.cu",
-               "output.cu", "qproj.cu", "backward.cu", "backward_tc.cu", "route_bwd.cu", "aux_loss.cu"]
+               "output.cu", "qproj.cu", "proj_tc.cu", "backward.cu", "backward_tc.cu", "route_bwd.cu", "aux_loss.cu"]
 SELFTEST_SOURCES = ["selftest.cu"]
 
 

@@ -144,13 +144,31 @@ struct QprojArgs {
     const gqe_shape* s;
     const void* x;               // [B, T, d_model] bf16
     const void* W_Q;             // [d_model, h * 128] bf16
+    const int32_t* idx;          // [B, T, g, k] as written by gqe_route
     const int32_t* head_offsets; // as written by gqe_route
     const int32_t* head_pos;
     void* Q;                     // [B, T, h, 128] bf16, routed rows written
     void* status;
+    void* scratch;               // oproj_scratch_bytes(s) bytes (the dense path's tile sets), or null
     cudaStream_t stream;
 };
 cudaError_t launch_qproj(const QprojArgs& a);
+// The dense path (proj_tc.cu): every head of a token tile with a routed head.
+cudaError_t launch_qproj_dense(const QprojArgs& a);
+
+// Routed output projection (oproj.cu).
+struct OprojArgs {
+    const gqe_shape* s;
+    const void* O;               // [B, T, h, d_h] bf16, zeros in the unselected slots
+    const int32_t* idx;          // [B, T, g, k]
+    const void* W_Z;             // [h * d_h, d_model] bf16
+    void* Y;                     // [B, T, d_model] bf16, out
+    void* status;
+    void* scratch;               // oproj_scratch_bytes(s): the token tiles' active-head sets
+    cudaStream_t stream;
+};
+cudaError_t launch_oproj(const OprojArgs& a);
+size_t oproj_scratch_bytes(const gqe_shape* s);
 
 // Output construction (output.cu).
 struct GroupSlotsArgs {

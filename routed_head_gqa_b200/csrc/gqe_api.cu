@@ -52,6 +52,8 @@ size_t gqe_workspace_bytes(const gqe_shape* s, int Lmax) {
     size_t need = kStatusBytes + route_scratch_bytes(s);
     const size_t shared = kStatusBytes + shared_tables_bytes(s->B, s->T);
     if (shared > need) need = shared;
+    const size_t oproj = kStatusBytes + oproj_scratch_bytes(s);
+    if (oproj > need) need = oproj;
     if (Lmax > 0) {
         const size_t dec = kStatusBytes + align256(decode_partials_bytes(s, Lmax));
         if (dec > need) need = dec;
@@ -256,13 +258,13 @@ gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* 
     return from_cuda(s->dtype == GQE_BF16 ? launch_prefill_tc(a) : launch_prefill_simt(a));
 }
 
-gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* head_offsets,
-                            const int32_t* head_pos, void* Q, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, const int32_t* idx,
+                            const int32_t* head_offsets, const int32_t* head_pos, void* Q, void* workspace,
+                            size_t workspace_bytes, void* stream) {
     gqe_status st = check_shape(s);
     if (st != GQE_OK) return st;
-    if (!x || !W_Q || !head_offsets || !head_pos || !Q) return GQE_ERR_INVALID_ARGUMENT;
-    if (!aligned16(x) || !aligned16(W_Q) || !aligned16(Q)) return GQE_ERR_INVALID_ARGUMENT;
+    if (!x || !W_Q || !idx || !head_offsets || !head_pos || !Q) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(W_Q) || !aligned16(idx) || !aligned16(Q)) return GQE_ERR_INVALID_ARGUMENT;
     if (s->dtype != GQE_BF16 || s->d_h != 128 || s->d_model % 8 != 0) return GQE_ERR_UNSUPPORTED;
     st = check_workspace(workspace, workspace_bytes, kStatusBytes);
     if (st != GQE_OK) return st;
@@ -270,12 +272,38 @@ gqe_status gqe_routed_qproj(const gqe_shape* s, const void* x, const void* W_Q, 
     a.s = s;
     a.x = x;
     a.W_Q = W_Q;
+    a.idx = idx;
     a.head_offsets = head_offsets;
     a.head_pos = head_pos;
     a.Q = Q;
     a.status = workspace;
+    // the dense path's per-tile head sets, when the workspace has room for them
+    a.scratch = workspace_bytes >= kStatusBytes + oproj_scratch_bytes(s)
+                    ? static_cast<void*>(static_cast<char*>(workspace) + kStatusBytes)
+                    : nullptr;
     a.stream = (cudaStream_t)stream;
     return from_cuda(launch_qproj(a));
+}
+
+gqe_status gqe_routed_oproj(const gqe_shape* s, const void* O, const int32_t* idx, const void* W_Z, void* Y,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    gqe_status st = check_shape(s);
+    if (st != GQE_OK) return st;
+    if (!O || !idx || !W_Z || !Y) return GQE_ERR_INVALID_ARGUMENT;
+    if (!aligned16(O) || !aligned16(idx) || !aligned16(W_Z) || !aligned16(Y)) return GQE_ERR_INVALID_ARGUMENT;
+    if (s->dtype != GQE_BF16 || s->d_h % 64 != 0 || s->h > 64 || s->d_model % 32 != 0) return GQE_ERR_UNSUPPORTED;
+    st = check_workspace(workspace, workspace_bytes, kStatusBytes + oproj_scratch_bytes(s));
+    if (st != GQE_OK) return st;
+    OprojArgs a;
+    a.s = s;
+    a.O = O;
+    a.idx = idx;
+    a.W_Z = W_Z;
+    a.Y = Y;
+    a.status = workspace;
+    a.scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.stream = (cudaStream_t)stream;
+    return from_cuda(launch_oproj(a));
 }
 
 gqe_status gqe_group_slots(const gqe_shape* s, const void* O, const int32_t* idx, const float* gate, void* O_cat,

@@ -131,13 +131,35 @@ def test_routed_qproj_validation():
 
     fake = 0x10000
     s = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_BF16)
-    assert g._lib.gqe_routed_qproj(ctypes.byref(s), None, fake, fake, fake, fake, fake, 1 << 20, None) == 1
-    assert g._lib.gqe_routed_qproj(ctypes.byref(s), fake, fake + 4, fake, fake, fake, fake, 1 << 20, None) == 1
+    call = lambda s, x, W, idx: g._lib.gqe_routed_qproj(ctypes.byref(s), x, W, idx, fake, fake, fake, fake, 1 << 20,
+                                                        None)
+    assert call(s, None, fake, fake) == 1
+    assert call(s, fake, fake + 4, fake) == 1
+    assert call(s, fake, fake, None) == 1        # no idx
+    assert call(s, fake, fake, fake + 4) == 1    # misaligned idx
     # tensor-core path only: bf16 with d_h = 128
     s32 = g.make_shape(2, 64, 128, 32, 8, 128, 2, g.GQE_F32)
-    assert g._lib.gqe_routed_qproj(ctypes.byref(s32), fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
+    assert call(s32, fake, fake, fake) == 2
     s64 = g.make_shape(2, 64, 128, 32, 8, 64, 2, g.GQE_BF16)
-    assert g._lib.gqe_routed_qproj(ctypes.byref(s64), fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
+    assert call(s64, fake, fake, fake) == 2
+
+
+def test_routed_oproj_validation():
+    import routed_head_gqa_b200 as g
+
+    fake = 0x10000
+    call = lambda s, O, idx, W, Y, ws=1 << 20: g._lib.gqe_routed_oproj(ctypes.byref(s), O, idx, W, Y, fake, ws,
+                                                                       None)
+    s = g.make_shape(2, 64, 256, 32, 8, 128, 2, g.GQE_BF16)
+    assert call(s, None, fake, fake, fake) == 1          # no O
+    assert call(s, fake, None, fake, fake) == 1          # no idx
+    assert call(s, fake, fake + 4, fake, fake) == 1      # misaligned idx
+    assert call(s, fake, fake, fake + 8, fake) == 1      # misaligned W_Z
+    assert call(s, fake, fake, fake, fake, 16) == 1      # workspace below the status word
+    assert call(g.make_shape(2, 64, 256, 32, 8, 128, 2, g.GQE_F32), fake, fake, fake, fake) == 2  # fp32
+    assert call(g.make_shape(2, 64, 256, 32, 8, 96, 2, g.GQE_BF16), fake, fake, fake, fake) == 2  # d_h 96
+    assert call(g.make_shape(2, 64, 256, 128, 8, 128, 2, g.GQE_BF16), fake, fake, fake, fake) == 2  # h > 64
+    assert call(g.make_shape(2, 64, 200, 32, 8, 128, 2, g.GQE_BF16), fake, fake, fake, fake) == 2  # d_model % 32
 
 
 def test_decode_paged_validation():

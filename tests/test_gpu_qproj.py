@@ -26,7 +26,7 @@ SMALL = [
 SENTINEL = -12288.0  # -1.5 * 2^13: exactly representable in bf16
 
 
-def qproj_parity(w, rows=None, cover=False):
+def qproj_parity(w, rows=None, cover=False, gather=False):
     g = U.gqe()
     inp = gqe_synth.make_inputs(w)
     W_Q = gqe_synth.make_qproj_weight(w)
@@ -34,7 +34,8 @@ def qproj_parity(w, rows=None, cover=False):
     buf = g.Buffers(shape, "cuda")
     buf.route(U.to_dev(inp["x"]), U.to_dev(inp["W_r"]), U.to_dev(inp["bias"]))
     Qp = torch.full((w.B, w.T, w.h, w.d_h), SENTINEL, dtype=w.torch_dtype, device="cuda")
-    g.gqe_routed_qproj(shape, U.to_dev(inp["x"]), U.to_dev(W_Q), buf.head_offsets, buf.head_pos, Qp, buf.workspace)
+    ws = buf.workspace if not gather else buf.workspace[: 256]  # a status-word-only workspace: the gather path
+    g.gqe_routed_qproj(shape, U.to_dev(inp["x"]), U.to_dev(W_Q), buf.idx, buf.head_offsets, buf.head_pos, Qp, ws)
     torch.cuda.synchronize()
     assert buf.status() == 0
     excl, idx_o, _ = U.check_routing(w, inp, buf.idx, buf.gate)
@@ -56,21 +57,27 @@ def qproj_parity(w, rows=None, cover=False):
     return err, len(rows), untouched
 
 
+@pytest.mark.parametrize("gather", [False, True], ids=["auto", "gather"])
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-def test_qproj_small(w):
-    err, n, untouched = qproj_parity(w)
+def test_qproj_small(w, gather):
+    """auto: the dense tiled path where the routed share g*k/h >= 3/10 (all but
+    qp_h32_k1), else the gathered rows; gather: a status-word-only workspace
+    forces the gathered path."""
+    err, n, untouched = qproj_parity(w, gather=gather)
     assert n > 0
     assert err <= U.TOL["bf16"], f"{w.name}: max abs error {err} over {n} rows"
     assert untouched, "rows of unselected heads were written"
 
 
-@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill", "gqe_long"])
-def test_qproj_full_size_covered(name):
+@pytest.mark.parametrize("name,gather", [("dense_gqa", False), ("gqe_prefill", False), ("gqe_long", False),
+                                         ("gqe_prefill", True)])
+def test_qproj_full_size_covered(name, gather):
     """At least 4096 token rows (every routed head of each): whole windows of
     consecutive positions (first, middle and last prefill units of three CTAs,
-    each sequence's last window, the most skewed windows) plus random rows."""
+    each sequence's last window, the most skewed windows) plus random rows; the
+    gathered path once at full size as well."""
     w = W[name]
-    err, n, untouched = qproj_parity(w, cover=True)
+    err, n, untouched = qproj_parity(w, cover=True, gather=gather)
     assert n >= 4096 - 64, f"{name}: only {n} rows compared"
     assert err <= U.TOL["bf16"], f"{name}: max abs error {err} over {n} rows"
     assert untouched
