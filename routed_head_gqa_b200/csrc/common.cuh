@@ -138,6 +138,10 @@ struct PrefillArgs {
     // backward: O and its zero fill are skipped).
     float* o32 = nullptr;
     float* lse = nullptr;
+    // Scratch for split-KV partials (tensor-core prefill): used when the units
+    // would leave SMs idle and split_bytes >= prefill_split_bytes(s); null: no split.
+    void* split_scratch = nullptr;
+    size_t split_bytes = 0;
 };
 // Routed query projection (qproj.cu).
 struct QprojArgs {
@@ -208,6 +212,8 @@ cudaError_t launch_aux_loss(const AuxLossArgs& a);
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a);
+// Scratch the tensor-core prefill uses for split-KV partials on this device (0: no split).
+size_t prefill_split_bytes(const gqe_shape* s);
 
 struct DecodeArgs {
     const gqe_shape* s;

@@ -54,6 +54,14 @@ size_t gqe_workspace_bytes(const gqe_shape* s, int Lmax) {
     if (shared > need) need = shared;
     const size_t oproj = kStatusBytes + oproj_scratch_bytes(s);
     if (oproj > need) need = oproj;
+    const size_t split = kStatusBytes + prefill_split_bytes(s);
+    if (split > need) need = split;
+    gqe_shape one = *s;  // the shared head: identity tables, then its split-KV partials
+    one.h = 1;
+    one.g = 1;
+    one.k = 1;
+    const size_t shared_split = kStatusBytes + shared_tables_bytes(s->B, s->T) + prefill_split_bytes(&one);
+    if (shared_split > need) need = shared_split;
     if (Lmax > 0) {
         const size_t dec = kStatusBytes + align256(decode_partials_bytes(s, Lmax));
         if (dec > need) need = dec;
@@ -211,6 +219,8 @@ gqe_status gqe_attn_prefill(const gqe_shape* s, const void* Q, const void* K, co
     a.stream = (cudaStream_t)stream;
     a.kv_g = s->g;
     a.kv_q0 = 0;
+    a.split_scratch = static_cast<char*>(workspace) + kStatusBytes;
+    a.split_bytes = workspace_bytes - kStatusBytes;
     if (s->dtype == GQE_BF16) {
         if (s->d_h != 128) return GQE_ERR_UNSUPPORTED;
         return from_cuda(launch_prefill_tc(a));
@@ -255,6 +265,9 @@ gqe_status gqe_attn_shared_head(const gqe_shape* s, const void* Qs, const void* 
     a.stream = (cudaStream_t)stream;
     a.kv_g = s->g;
     a.kv_q0 = kv_group;
+    const size_t used = kStatusBytes + shared_tables_bytes(s->B, s->T);
+    a.split_scratch = static_cast<char*>(workspace) + used;
+    a.split_bytes = workspace_bytes - used;
     return from_cuda(s->dtype == GQE_BF16 ? launch_prefill_tc(a) : launch_prefill_simt(a));
 }
 

@@ -72,6 +72,9 @@ struct Smem {
     int32_t abort_flag;
 };
 
+// Split-KV partial of one routed row: o = O/l in fp32 and its log2-sum-exp.
+constexpr int kPartFloats = 132;  // o[128], lse, 3 pad (16-byte records)
+
 struct Params {
     UnitGeom u;
     const __nv_bfloat16* Q;
@@ -87,12 +90,37 @@ struct Params {
     float scale_log2;
     int q_rows;  // B*T*h: rows of Q viewed as [B*T*h, 128]
     int kv_q0;   // KV group of the unit's group 0 in the K/V tensor maps
+    // Split-KV (nsplit > 1): item = unit * nsplit + s covers KV tiles
+    // [s n/nsplit, (s+1) n/nsplit) of the unit's n; each item writes its rows'
+    // partials to part, split 0 also the rows' (position, head, gate) to
+    // part_rows, and prefill_combine_kernel merges them.
+    int nsplit;
+    float* part;         // [items][kQT][kBM][kPartFloats]
+    int32_t* part_rows;  // [units][kQT][kBM][3]
 };
 
 // Keys needed by Q tile t of the unit at window w: 0 .. end-1, end = min(w0 + (t+1)W, T).
-__device__ __forceinline__ int tile_kv_tiles(const UnitGeom& u, int w, int t) {
+__host__ __device__ __forceinline__ int tile_kv_tiles(const UnitGeom& u, int w, int t) {
     const int end = min(w * kQT * u.W + (t + 1) * u.W, u.T);
     return (end + kBN - 1) / kBN;
+}
+
+// Item -> unit, split and the split's KV tiles: the first KV tile kv_lo and
+// each Q tile's count cnt[t] (the tile's own range clipped to the split's).
+// Splits take ceil(n / nsplit) tiles each from the start, so a unit with
+// fewer tiles than splits leaves its last splits empty, never split 0 (which
+// also zero-fills the window and records the rows for the merge).
+__device__ __forceinline__ void item_range(const UnitGeom& u, int nsplit, int64_t item, int64_t& unit, int& split,
+                                           int& b, int& q, int& w, int& kv_lo, int (&cnt)[kQT]) {
+    unit = item / nsplit;
+    split = (int)(item % nsplit);
+    unit_coords(u, unit, b, q, w);
+    const int n_last = tile_kv_tiles(u, w, kQT - 1);
+    const int chunk = (n_last + nsplit - 1) / nsplit;
+    kv_lo = min(split * chunk, n_last);
+    const int kv_hi = min(kv_lo + chunk, n_last);
+#pragma unroll
+    for (int t = 0; t < kQT; ++t) cnt[t] = max(0, min(kv_hi, tile_kv_tiles(u, w, t)) - kv_lo);
 }
 
 // The j-th unit of this CTA: heavy windows first, zig-zag over the CTAs so that
@@ -136,7 +164,9 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
 
 
 // ---------------------------------------------------------------------------
-template <bool kTrain>  // kTrain: also write the training outputs (o32, lse); O only when asked
+// kTrain: also write the training outputs (o32, lse); O only when asked.
+// kSplit: split-KV items (p.nsplit > 1); the plain instance carries none of it.
+template <bool kTrain, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapQB,
@@ -145,7 +175,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     Smem& sm = *smem_align1024<Smem>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const UnitGeom& u = p.u;
-    const int64_t n_units = u.count();
+    const int nsplit = kSplit ? p.nsplit : 1;
+    const int64_t n_units = u.count() * nsplit;  // work items (units when not split)
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -190,24 +221,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             uint32_t kv_it = 0;
             bool k_pending = false;
             for (int64_t j = 0;; ++j) {
-                const int64_t unit = cta_unit(j, n_units);
-                if (unit < 0 || aborted(sm)) break;
-                int b, q, w;
-                unit_coords(u, unit, b, q, w);
-                const int n = tile_kv_tiles(u, w, kQT - 1);
+                const int64_t item = cta_unit(j, n_units);
+                if (item < 0 || aborted(sm)) break;
+                int64_t unit;
+                int split, b, q, w, kv_lo, cnt[kQT];
+                item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+                const int n = cnt[kQT - 1];
                 bool ok = true;
                 for (int i = 0; i < n; ++i, ++kv_it) {
                     const int st = kv_it & 1;
                     const uint32_t par = ((kv_it >> 1) & 1) ^ 1;
                     if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(sm, p, 1); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_k[st], kTileBytes);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, p.kv_q0 + q, i * kBN, b);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, p.kv_q0 + q, i * kBN, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, p.kv_q0 + q, (kv_lo + i) * kBN, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, p.kv_q0 + q, (kv_lo + i) * kBN, b);
                     k_pending = true;
                     if (!mbar_wait(&sm.kv_empty_v[st], par)) { fail(sm, p, 2); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_v[st], kTileBytes);
-                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, p.kv_q0 + q, i * kBN, b);
-                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, p.kv_q0 + q, i * kBN, b);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, p.kv_q0 + q, (kv_lo + i) * kBN, b);
+                    tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st] + kHalf, 64, p.kv_q0 + q, (kv_lo + i) * kBN, b);
                     k_pending = false;
                 }
                 if (!ok) break;
@@ -267,18 +299,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             };
             auto wait_k = [&](uint32_t it) { return mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1); };
             auto wait_v = [&](uint32_t it) { return mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1); };
-            for (int64_t j = 0; ok; ++j, ++u_it) {
-                const int64_t unit = cta_unit(j, n_units);
-                if (unit < 0 || aborted(sm)) break;
-                int b, q, w;
-                unit_coords(u, unit, b, q, w);
-                const int n0 = tile_kv_tiles(u, w, 0), n1 = tile_kv_tiles(u, w, 1);
-                const int qs = u_it & 1;
-                if (!mbar_wait(&sm.q_full[qs], (u_it >> 1) & 1)) { fail(sm, p, 10); break; }
+            for (int64_t j = 0; ok; ++j) {
+                const int64_t item = cta_unit(j, n_units);
+                if (item < 0 || aborted(sm)) break;
+                int64_t unit;
+                int split, b, q, w, kv_lo, cnt[kQT];
+                item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+                const int n0 = cnt[0], n1 = cnt[1];
+                if (n1 == 0) continue;  // an empty split: every role skips it
+                const uint32_t ui = u_it++;
+                const int qs = ui & 1;
+                if (!mbar_wait(&sm.q_full[qs], (ui >> 1) & 1)) { fail(sm, p, 10); break; }
                 tc_fence_after();
                 if (!wait_k(kv_it)) { fail(sm, p, 11); break; }
                 tc_fence_after();
-                issue_s(0, kv_it);
+                if (n0 > 0) issue_s(0, kv_it);
                 issue_s(1, kv_it);
                 umma_commit(&sm.kv_empty_k[kv_it & 1]);
                 if (n1 == 1) umma_commit(&sm.q_empty);
@@ -286,7 +321,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     const uint32_t it = kv_it + i;
                     if (i < n0) {
                         ok = mbar_wait(&sm.p_full[0], (c[0] + i) & 1);
-                        if (ok && i == 0) ok = mbar_wait(&sm.o_empty[0], (u_it & 1) ^ 1);
+                        if (ok && i == 0) ok = mbar_wait(&sm.o_empty[0], (ui & 1) ^ 1);
                         if (ok) ok = wait_v(it);
                         if (!ok) { fail(sm, p, 12); break; }
                         tc_fence_after();
@@ -299,7 +334,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                         }
                     }
                     ok = mbar_wait(&sm.p_full[1], (c[1] + i) & 1);
-                    if (ok && i == 0) ok = mbar_wait(&sm.o_empty[1], (u_it & 1) ^ 1);
+                    if (ok && i == 0) ok = mbar_wait(&sm.o_empty[1], (ui & 1) ^ 1);
                     if (ok) ok = wait_v(it);
                     if (!ok) { fail(sm, p, 14); break; }
                     tc_fence_after();
@@ -328,15 +363,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         uint32_t u_it = 0;
         int64_t armed = -1;  // last unit whose Q loads were issued
         const int32_t total = (int32_t)((int64_t)u.B * u.T * u.g * u.k);
-        for (int64_t j = 0;; ++j, ++u_it) {
-            const int64_t unit = cta_unit(j, n_units);
-            if (unit < 0 || aborted(sm)) break;
-            int b, q, w;
-            unit_coords(u, unit, b, q, w);
-            const int rs = u_it & 1;
+        for (int64_t j = 0;; ++j) {
+            const int64_t item = cta_unit(j, n_units);
+            if (item < 0 || aborted(sm)) break;
+            int64_t unit;
+            int split, b, q, w, kv_lo, cnt[kQT];
+            item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+            if (cnt[kQT - 1] == 0) continue;  // an empty split
+            const uint32_t ui = u_it++;
+            const int rs = ui & 1;
             // The row tables are double buffered: build this unit's while the
             // previous unit still computes, then wait for its Q tiles to be free.
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_free[rs], ((u_it >> 1) & 1) ^ 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_free[rs], ((ui >> 1) & 1) ^ 1))) {
                 if (lane == 0) fail(sm, p, 20);
                 break;
             }
@@ -422,7 +460,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     }
                 }
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_empty, (u_it & 1) ^ 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_empty, (ui & 1) ^ 1))) {
                 if (lane == 0) fail(sm, p, 21);
                 break;
             }
@@ -460,7 +498,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     tma_gather4_2d(&mapQ, &sm.q_full[rs], dst + kHalf, 64, row[0], row[1], row[2], row[3]);
                 }
             }
-            armed = u_it;
+            armed = ui;
         }
         // Drain: the last issued Q loads land before the CTA may exit.
         if (armed >= 0) mbar_wait(&sm.q_full[armed & 1], (armed >> 1) & 1);
@@ -474,10 +512,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         // slots, 16 lanes per slot.
         const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
         for (int64_t j = 0; p.O != nullptr; ++j) {  // a recompute for the backward leaves O alone
-            const int64_t unit = cta_unit(j, n_units);
-            if (unit < 0 || aborted(sm)) break;
+            const int64_t item = cta_unit(j, n_units);
+            if (item < 0 || aborted(sm)) break;
+            if (kSplit && item % nsplit != 0) continue;  // a unit's first split zero-fills its window
             int b, q, w;
-            unit_coords(u, unit, b, q, w);
+            unit_coords(u, item / nsplit, b, q, w);
             for (int half = 0; half < kQT; ++half) {
                 const int w0 = (w * kQT + half) * u.W;
                 const int nt = min(w0 + u.W, u.T) - w0;  // tokens in the half, <= 128
@@ -534,15 +573,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         const uint32_t s_addr = tmem + lane_off + kColS + t * 128;
         const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
         constexpr bool train = kTrain;  // also write R = p - bf16(p) for the exact P.V
-        uint32_t ctile = 0, u_it = 0;
-        for (int64_t j = 0;; ++j, ++u_it) {
-            const int64_t unit = cta_unit(j, n_units);
-            if (unit < 0 || aborted(sm)) break;
-            int b, q, w;
-            unit_coords(u, unit, b, q, w);
-            const int n = tile_kv_tiles(u, w, t);
-            const int rs = u_it & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[rs], (u_it >> 1) & 1))) {
+        uint32_t ctile = 0, u_it = 0, o_it = 0;  // S tiles, items, O_t completions waited
+        for (int64_t j = 0;; ++j) {
+            const int64_t item = cta_unit(j, n_units);
+            if (item < 0 || aborted(sm)) break;
+            int64_t unit;
+            int split, b, q, w, kv_lo, cnt[kQT];
+            item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+            if (cnt[kQT - 1] == 0) continue;  // an empty split
+            const uint32_t ui = u_it++;
+            const int n = cnt[t];
+            const int rs = ui & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[rs], (ui >> 1) & 1))) {
                 if (lane == 0) fail(sm, p, 30);
                 break;
             }
@@ -565,7 +607,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 ld_bind(s[1]);
                 ld_bind(s[2]);
                 ld_bind(s[3]);
-                const int kv0 = i * kBN;
+                const int kv0 = (kv_lo + i) * kBN;
                 const bool need_mask = kv0 + kBN - 1 > lo;
                 if (need_mask) {
 #pragma unroll
@@ -671,13 +713,53 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 mbar_arrive(&sm.p_full[t]);
             }
             if (!ok) break;
+            const int j_row = sm.row_j[rs][t][r];
+            if (kSplit) {
+                // Split-KV: this split's o = O_t / l and log2-sum-exp m + log2(l)
+                // (-inf for a split with no keys for this tile); split 0 also
+                // records the row's position, head and gate for the merge.
+                float* rec = p.part + ((item * kQT + t) * kBM + r) * kPartFloats;
+                if (n > 0) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], o_it & 1))) {
+                        if (lane == 0) fail(sm, p, 35);
+                        break;
+                    }
+                    ++o_it;
+                    tc_fence_after();
+                    const float inv = 1.0f / l;
+#pragma unroll 1
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + cb * 32, o);
+                        ld_wait_bind(o);
+                        float4* dst = reinterpret_cast<float4*>(rec + cb * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                 __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                    }
+                    rec[kD] = m + log2f(l);
+                } else {
+                    rec[kD] = -INFINITY;
+                }
+                if (split == 0) {
+                    int32_t* pr = p.part_rows + ((unit * kQT + t) * kBM + r) * 3;
+                    pr[0] = t_row;
+                    pr[1] = j_row;
+                    pr[2] = __float_as_int(sm.row_gate[rs][t][r]);
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.o_empty[t]);
+                mbar_arrive(&sm.rows_free[rs]);
+                continue;
+            }
             // Epilogue: O_t / l * gate -> bf16 row of O[b, t, j, :].
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], u_it & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.o_full[t], o_it & 1))) {
                 if (lane == 0) fail(sm, p, 34);
                 break;
             }
+            ++o_it;
             tc_fence_after();
-            const int j_row = sm.row_j[rs][t][r];
             const int64_t orow_idx = ((int64_t)b * u.T + (t_row >= 0 ? t_row : 0)) * u.h + j_row;
             if (kTrain) {
                 // Training: the ungated output o = O_t / l in fp32 and the row's
@@ -739,27 +821,122 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     }
 }
 
-}  // namespace
+// Merge of the split-KV partials, one warp per routed row (unit, Q tile, row):
+// O = gate * sum_s 2^(lse_s - LSE) o_s with LSE = log2 sum_s 2^lse_s, over the
+// splits that hold keys for the row's tile, in order (reproducible).  Lane s
+// reads split s's log-sum-exp.
+__global__ void __launch_bounds__(256)
+prefill_combine_kernel(UnitGeom u, int nsplit, const float* __restrict__ part, const int32_t* __restrict__ part_rows,
+                       __nv_bfloat16* __restrict__ O) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (unit * kQT + t) * kBM + r
+    if (row >= u.count() * kQT * kBM) return;
+    const int32_t* pr = part_rows + row * 3;
+    const int t_row = pr[0];
+    if (t_row < 0) return;  // padding
+    const int j_row = pr[1];
+    const float gate = __int_as_float(pr[2]);
+    const int64_t unit = row / (kQT * kBM);
+    const int64_t tr = row % (kQT * kBM);
+    const int t = (int)(tr / kBM);
+    const float* recs = part + (unit * nsplit * (kQT * kBM) + tr) * kPartFloats;
+    const int64_t rstride = (int64_t)kQT * kBM * kPartFloats;  // next split, same row
+    float ls = -INFINITY;
+    if (lane < nsplit) {
+        int64_t un;
+        int sp, b, q, w, kv_lo, cnt[kQT];
+        item_range(u, nsplit, unit * nsplit + lane, un, sp, b, q, w, kv_lo, cnt);
+        if (cnt[t] > 0) ls = recs[lane * rstride + kD];
+    }
+    float m = ls;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+    const float wl = (ls == -INFINITY) ? 0.f : fast_exp2(ls - m);
+    float L = wl;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) L += __shfl_xor_sync(0xffffffffu, L, d);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < nsplit; ++sp) {
+        const float wt = __shfl_sync(0xffffffffu, wl, sp);
+        if (wt == 0.f) continue;
+        const float4 v = reinterpret_cast<const float4*>(recs + sp * rstride)[lane];
+        acc.x += wt * v.x;
+        acc.y += wt * v.y;
+        acc.z += wt * v.z;
+        acc.w += wt * v.w;
+    }
+    const float inv = 1.0f / L;
+    const float4 o = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    int b, q, w;
+    unit_coords(u, unit, b, q, w);
+    const int64_t orow = ((int64_t)b * u.T + t_row) * u.h + j_row;
+    reinterpret_cast<uint2*>(O + orow * kD)[lane] =
+        make_uint2(pack_bf16x2(gate * o.x, gate * o.y), pack_bf16x2(gate * o.z, gate * o.w));
+}
 
-cudaError_t launch_prefill_tc(const PrefillArgs& a) {
-    const gqe_shape& s = *a.s;
-    if (s.k > 4 || s.h / s.g > 32) return cudaErrorNotSupported;
+UnitGeom prefill_geom(const gqe_shape& s) {
     UnitGeom u;
     u.B = s.B; u.T = s.T; u.h = s.h; u.g = s.g; u.k = s.k; u.hpg = s.h / s.g;
     u.W = 32 * (4 / s.k);  // k*W <= 128 rows per tile, W a multiple of the 32-token chunk
     u.nwin = (s.T + kQT * u.W - 1) / (kQT * u.W);
     u.nchunk = gqe_chunk_count(s.T);
+    return u;
+}
+
+// Splits per unit: 1 unless the units would leave at least half of the SMs
+// idle (measured on the shared head: 128 units on 148 SMs ran 16 % slower
+// split, 32 and 64 units 8 % and 1.7x faster), else enough for about two
+// items per SM, with at least two KV tiles per split of the longest unit (an
+// item's fixed cost, its row table and Q tiles, is a few KV tiles' worth), at
+// most 16 (the merge reads one split per lane, at most 32).
+int prefill_splits(const UnitGeom& u, int sms) {
+    const int64_t units = u.count(), target = 2 * (int64_t)sms;
+    if (units <= 0 || 2 * units > sms) return 1;
+    int64_t sp = (target + units - 1) / units;
+    const int n_max = tile_kv_tiles(u, u.nwin - 1, kQT - 1);
+    if (sp > n_max / 2) sp = n_max / 2;
+    if (sp > 16) sp = 16;
+    return sp < 1 ? 1 : (int)sp;
+}
+
+size_t a256b(size_t n) { return (n + 255) & ~size_t(255); }
+size_t split_part_bytes(const UnitGeom& u, int nsplit) {
+    return a256b((size_t)u.count() * nsplit * kQT * kBM * kPartFloats * sizeof(float));
+}
+size_t split_rows_bytes(const UnitGeom& u) { return a256b((size_t)u.count() * kQT * kBM * 3 * sizeof(int32_t)); }
+
+int device_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return sms;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return sms;
+}
+
+}  // namespace
+
+size_t prefill_split_bytes(const gqe_shape* s) {
+    if (s->dtype != GQE_BF16 || s->d_h != kD || s->k > 4 || s->h / s->g > 32) return 0;
+    const UnitGeom u = prefill_geom(*s);
+    const int sp = prefill_splits(u, device_sms());
+    return sp > 1 ? split_part_bytes(u, sp) + split_rows_bytes(u) : 0;
+}
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a) {
+    const gqe_shape& s = *a.s;
+    if (s.k > 4 || s.h / s.g > 32) return cudaErrorNotSupported;
+    const UnitGeom u = prefill_geom(s);
 
     // The setmaxnreg split needs exactly kRegsLaunch registers per thread at
     // launch (a property of the compiled kernel: checked once per process).
     static std::atomic<int> regs_checked{0};
     if (regs_checked.load(std::memory_order_acquire) == 0) {
-        cudaFuncAttributes fa, fb;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel<false>);
-        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fb, prefill_tc_kernel<true>);
+        cudaFuncAttributes fa, fb, fc;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_tc_kernel<false, false>);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fb, prefill_tc_kernel<true, false>);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fc, prefill_tc_kernel<false, true>);
         if (e != cudaSuccess) return e;
-        regs_checked.store((fa.numRegs == kRegsLaunch && fb.numRegs == kRegsLaunch) ? 1 : -1,
-                           std::memory_order_release);
+        const bool all = fa.numRegs == kRegsLaunch && fb.numRegs == kRegsLaunch && fc.numRegs == kRegsLaunch;
+        regs_checked.store(all ? 1 : -1, std::memory_order_release);
     }
     if (regs_checked.load(std::memory_order_acquire) != 1) return cudaErrorNotSupported;
 
@@ -802,14 +979,26 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     p.q_rows = (int)q_rows;
     p.kv_q0 = a.kv_q0;
 
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t units = u.count();
+    const int sms = device_sms();
+    // Split-KV when the units leave SMs idle and the caller's scratch holds the
+    // partials (inference only: the training outputs come from one pass).
+    p.nsplit = 1;
+    p.part = nullptr;
+    p.part_rows = nullptr;
+    if (a.split_scratch != nullptr && a.o32 == nullptr && a.O != nullptr) {
+        const int sp = prefill_splits(u, sms);
+        if (sp > 1 && a.split_bytes >= split_part_bytes(u, sp) + split_rows_bytes(u)) {
+            p.nsplit = sp;
+            p.part = static_cast<float*>(a.split_scratch);
+            p.part_rows = reinterpret_cast<int32_t*>(static_cast<char*>(a.split_scratch) + split_part_bytes(u, sp));
+        }
+    }
+    const int64_t units = u.count() * p.nsplit;
     const int grid = (int)(units < sms ? units : sms);
     const size_t smem = sizeof(Smem) + 1024;
     const bool train = a.o32 != nullptr;
-    auto kern = train ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    auto kern = train ? prefill_tc_kernel<true, false>
+                      : (p.nsplit > 1 ? prefill_tc_kernel<false, true> : prefill_tc_kernel<false, false>);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -822,7 +1011,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mapK, mapV, mapQ, mapQB, p);
+    err = cudaLaunchKernelEx(&cfg, kern, mapK, mapV, mapQ, mapQB, p);
+    if (err != cudaSuccess || p.nsplit == 1) return err;
+    const int64_t rows = u.count() * kQT * kBM;
+    prefill_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, a.stream>>>(
+        u, p.nsplit, p.part, p.part_rows, (__nv_bfloat16*)a.O);
+    return cudaGetLastError();
 }
 
 }  // namespace gqe

@@ -37,6 +37,11 @@ SMALL_BF16 = [
     C("bf16_h64", B=2, T=96, d_model=256, h=64, g=8, d_h=128, k=2, seed=23),
     C("bf16_h128", B=1, T=64, d_model=128, h=128, g=16, d_h=128, k=1, seed=24),
     C("bf16_h256_T40", B=1, T=40, d_model=128, h=256, g=32, d_h=128, k=3, seed=25),
+    # Split-KV: so few units that each is split over its KV tiles and merged by
+    # log-sum-exp (32 units of up to 16 KV tiles -> 8 splits; 5 units over a
+    # ragged T -> 4 splits)
+    C("bf16_splitkv_k2", B=1, T=2048, d_model=64, h=8, g=2, d_h=128, k=2, seed=26),
+    C("bf16_splitkv_ragged", B=1, T=1100, d_model=64, h=4, g=1, d_h=128, k=1, seed=27),
 ]
 SMALL_F32 = [
     W["tiny_f32"],
