@@ -49,7 +49,11 @@ constexpr uint32_t kTileBytes = 2 * kHalf; // [128][128] bf16, 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * tile
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: p <= 2^8 between rescales
-constexpr int kPolyPairs = 4;               // of every 16 element pairs, exp2 on the FMA pipe
+// Of every 16 element pairs of an unmasked tile, exp2 on the FMA pipe
+// (exp2_poly2) for this many, on MUFU for the rest.  A same-box sweep with
+// both softmax warpgroups active measured 0 fastest (gqe_prefill 0.596 ms
+// against 0.607 at 4 and 0.616 at 6; gqe_32k 1.865 against 1.944 ms).
+constexpr int kPolyPairs = 0;
 constexpr uint32_t kWhereTc = 2;            // status "where" id of this kernel
 // Register split (setmaxnreg): 4 control warps at 88, 8 softmax warps at 208.
 // 128*88 + 256*208 = 64512 = 384 * 168, the block's registers at launch.
@@ -651,9 +655,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     l *= alpha;
                 }
                 // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
-                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe (4 of 16
-                // measured fastest with both softmax warpgroups active: MUFU is then
-                // about 80 % busy and the FMA and integer pipes take the rest).
+                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
                 const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);
                 const uint64_t NM2 = pk2(-m_use, -m_use);
                 uint64_t sum2[4] = {0, 0, 0, 0};
