@@ -373,20 +373,24 @@ __device__ __forceinline__ void ds_key(const float (&gp)[32], const uint32_t (&d
 
 // ------------------------------------------------------------------ 2. dQ
 // One CTA per SM; work item = one half-window tile of 128 routed rows.
-// Roles: warp 0 K/V producer (2-stage ring), warp 1 MMA issuer, warp 2 row
-// table + Q/dO gather, warps 4-11 elementwise + epilogue (thread = row, two
+// Roles: warp 0 K/V producer (3-stage K ring, 2-stage V ring), warp 1 MMA
+// issuer, warp 2 Q/dO loads, warps 4-11 elementwise + epilogue (thread = row, two
 // warps per row, one per 64-column half).  TMEM: S buffers [0,128) and
 // [128,256), dP [256,384), dQ [384,512); dS (bf16 pairs) overwrites dP's
 // columns a_col(0..7) once dP is in registers.  Per key tile the elementwise
 // warps run the dS phase of tile i, then the exponent phase of tile i+1 (its
 // S is already in TMEM) while the tensor core runs dQ(i) and dP(i+1).
+// K has three stages: K(i) is read by S(i) early and by dQ(i) late, so with
+// two the load of K(i+2) could only start after dQ(i) and S(i+2) waited for
+// it.  The elementwise warps read their rows' table entries from the
+// workspace (the shared memory is full).
+constexpr int kDqKStages = 3;
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dO[kTile];
-    uint8_t k[2][kTile];
+    uint8_t k[kDqKStages][kTile];
     uint8_t v[2][kTile];
-    TileTab tab;
-    uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
+    uint64_t kv_full_k[kDqKStages], kv_full_v[2], kv_empty_k[kDqKStages], kv_empty_v[2];
     uint64_t rows_full, rows_empty, s_full[2], dp_full, ew_done, dq_full, dq_empty, drain;
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -414,16 +418,17 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
     const UnitGeom& u = p.u;
     const int64_t n_items = dq_items(u);
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kDqKStages; ++i) {
             mbar_init(&sm.kv_full_k[i], 1);
-            mbar_init(&sm.kv_full_v[i], 1);
             mbar_init(&sm.kv_empty_k[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.kv_full_v[i], 1);
             mbar_init(&sm.kv_empty_v[i], 1);
             mbar_init(&sm.s_full[i], 1);
         }
         mbar_init(&sm.rows_full, 1);
-        // the MMA issuer's commit after the item's last dQ step, which follows every
-        // elementwise step of the item (and so every read of its table)
+        // the MMA issuer's commit after the item's last dQ step (Q and dO read)
         mbar_init(&sm.rows_empty, 1);
         mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.ew_done, 256);
@@ -453,12 +458,12 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 int64_t tile;
                 dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
                 for (int i = 0; i < nkv; ++i, ++kv) {
-                    const int st = kv & 1;
-                    const uint32_t par = ((kv >> 1) & 1) ^ 1;
-                    if (!mbar_wait(&sm.kv_empty_k[st], par)) { fail(&sm.abort_flag, p.status, 1); ok = false; break; }
-                    mbar_arrive_expect_tx(&sm.kv_full_k[st], kTile);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st], 0, q, i * kBM, b);
-                    tma_load_4d(&mapK, &sm.kv_full_k[st], sm.k[st] + kHalf, 64, q, i * kBM, b);
+                    const int sk = (int)(kv % kDqKStages), st = kv & 1;
+                    const uint32_t par_k = ((kv / kDqKStages) & 1) ^ 1, par = ((kv >> 1) & 1) ^ 1;
+                    if (!mbar_wait(&sm.kv_empty_k[sk], par_k)) { fail(&sm.abort_flag, p.status, 1); ok = false; break; }
+                    mbar_arrive_expect_tx(&sm.kv_full_k[sk], kTile);
+                    tma_load_4d(&mapK, &sm.kv_full_k[sk], sm.k[sk], 0, q, i * kBM, b);
+                    tma_load_4d(&mapK, &sm.kv_full_k[sk], sm.k[sk] + kHalf, 64, q, i * kBM, b);
                     if (!mbar_wait(&sm.kv_empty_v[st], par)) { fail(&sm.abort_flag, p.status, 2); ok = false; break; }
                     mbar_arrive_expect_tx(&sm.kv_full_v[st], kTile);
                     tma_load_4d(&mapV, &sm.kv_full_v[st], sm.v[st], 0, q, i * kBM, b);
@@ -466,10 +471,10 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                 }
             }
             // every issued load lands before the CTA may exit
-            for (uint32_t back = 1; back <= 2 && back <= kv; ++back) {
+            for (uint32_t back = 1; back <= kDqKStages && back <= kv; ++back) {
                 const uint32_t it = kv - back;
-                mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1);
-                mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1);
+                mbar_wait(&sm.kv_full_k[it % kDqKStages], (it / kDqKStages) & 1);
+                if (back <= 2) mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1);
             }
         }
     } else if (warp == 1) {
@@ -479,14 +484,16 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             const uint32_t idesc_dq = idesc_bf16_f32(kBM, kD, false, true);
             const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
             const uint32_t qlo = smem_desc_lo(smem_u32(sm.q), 16), dolo = smem_desc_lo(smem_u32(sm.dO), 16);
-            const uint32_t klo0 = smem_desc_lo(smem_u32(sm.k[0]), 16), klo1 = smem_desc_lo(smem_u32(sm.k[1]), 16);
-            const uint32_t kmlo0 = smem_desc_lo(smem_u32(sm.k[0]), kHalf), kmlo1 = smem_desc_lo(smem_u32(sm.k[1]), kHalf);
+            // K stage x % 3 sits (x % 3) * kTile bytes past stage 0 (start address in 16-byte units)
+            const uint32_t klo0 = smem_desc_lo(smem_u32(sm.k[0]), 16);
+            const uint32_t kmlo0 = smem_desc_lo(smem_u32(sm.k[0]), kHalf);
+            auto kstage = [&](uint32_t x) { return (x % kDqKStages) * (kTile >> 4); };
             const uint32_t vlo0 = smem_desc_lo(smem_u32(sm.v[0]), 16), vlo1 = smem_desc_lo(smem_u32(sm.v[1]), 16);
             const uint32_t c_s = tmem, c_dp = tmem + 256, c_dq = tmem + 384;
             auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
             // S(kv tile) into S buffer sb: Q . K^T (both K-major).
             auto issue_s = [&](uint32_t kvi, uint32_t sb) {
-                const uint32_t kb = (kvi & 1) ? klo1 : klo0;
+                const uint32_t kb = klo0 + kstage(kvi);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
@@ -506,13 +513,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             };
             // dQ (+)= dS . K (dS bf16 pairs in dP's columns a_col(kk); K MN-major).
             auto issue_dq = [&](uint32_t kvi, bool first) {
-                const uint32_t kb = (kvi & 1) ? kmlo1 : kmlo0;
+                const uint32_t kb = kmlo0 + kstage(kvi);
 #pragma unroll
                 for (int kk = 0; kk < kBM / 16; ++kk)
                     umma_ts(c_dq, c_dp + a_col(kk), desc(kb + (uint32_t)((kk * 2048) >> 4)), idesc_dq,
                             (first && kk == 0) ? 0u : 1u);
             };
-            auto wait_k = [&](uint32_t x) { return mbar_wait(&sm.kv_full_k[x & 1], (x >> 1) & 1); };
+            auto wait_k = [&](uint32_t x) { return mbar_wait(&sm.kv_full_k[x % kDqKStages], (x / kDqKStages) & 1); };
             auto wait_v = [&](uint32_t x) { return mbar_wait(&sm.kv_full_v[x & 1], (x >> 1) & 1); };
             uint32_t kv = 0, sc = 0, ec = 0, item_no = 0;  // kv tiles, S issued, elementwise steps, items
             bool ok = true;
@@ -549,7 +556,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
                     }
                     tc_fence_after();
                     issue_dq(x, i == 0);
-                    umma_commit(&sm.kv_empty_k[x & 1]);  // K(i): read by S(i) and dQ(i)
+                    umma_commit(&sm.kv_empty_k[x % kDqKStages]);  // K(i): read by S(i) and dQ(i)
                     if (i == nkv - 1) {
                         umma_commit(&sm.dq_full);
                         umma_commit(&sm.rows_empty);  // Q, dO and the table of the item are no longer read
@@ -581,13 +588,11 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             int b, q, w0, nkv;
             int64_t tile;
             dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
-            // the previous item's operands and table are free
+            // the previous item's Q and dO are free
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_empty, (item_no & 1) ^ 1))) {
                 if (lane == 0) fail(&sm.abort_flag, p.status, 20);
                 break;
             }
-            load_tab(p.tabs + tile, sm.tab);
-            __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.rows_full, 2 * kTile);
                 const int row0 = (int)(tile * kBM);
@@ -613,12 +618,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ C
             int b, q, w0, nkv;
             int64_t tile;
             dq_item(u, p.ntiles, it, b, q, w0, nkv, tile);
+            const TileTab* tab = p.tabs + tile;  // read-only here: loaded while Q and dO arrive
+            const int t_row = tab->t[r], j_row = tab->j[r];
+            const float lse2 = tab->lse2[r], dl2 = tab->dl2[r];
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.rows_full, item_no & 1))) {
                 if (lane == 0) fail(&sm.abort_flag, p.status, 30);
                 break;
             }
-            const int t_row = sm.tab.t[r], j_row = sm.tab.j[r];
-            const float lse2 = sm.tab.lse2[r], dl2 = sm.tab.dl2[r];
             float gp0[32], gp1[32];
             bool ok = true;
             for (int i = 0; i <= nkv; ++i) {
