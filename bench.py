@@ -48,13 +48,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
+    ("prefill_tc_kernel", "gqe_prefill"): {
+        "sha": "b017cc66fcf82daa", "bytes_per_launch": 1067480000 + 241922304,
+        "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_gqe_prefill.md)"},
+    ("prefill_tc_kernel", "gqe_long"): {
+        "sha": "b017cc66fcf82daa", "bytes_per_launch": 171321344 + 47180800,
+        "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_gqe_long.md)"},
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "a0a298782a4902f5", "bytes_per_launch": 105195008 + 30063872,
-        "note": "ncu --set full, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
+        "sha": "b017cc66fcf82daa", "bytes_per_launch": 105076736 + 29326080,
+        "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
-        "sha": "38d1f07202b92c94", "bytes_per_launch": 2270814604,
-        "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch of the partial kernel: "
-                "dram__bytes.sum.per_second x duration (profiles/decode_partial_kernel_gqe_decode.md)"},
+        "sha": "2ffadcebec633c3d", "bytes_per_launch": 2263625728 + 8142592,
+        "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch of the partial kernel "
+                "(profiles/decode_partial_kernel_gqe_decode.md)"},
 }
 
 
