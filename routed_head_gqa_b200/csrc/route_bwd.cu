@@ -40,9 +40,11 @@ __device__ __forceinline__ void fma4(float a, const float4& b, float4& c) {
     c.w = fmaf(a, b.w, c.w);
 }
 
-// dx[t, i] for a 64-token x 128-column tile; the heads are summed 32 at a time
-// from shared-memory copies of dl (transposed to [head][token]) and W_r
-// (transposed to [head][column]).
+// dx[t, i] for 128-column blocks: a block keeps its columns of W_r (transposed
+// to [head][column]) in shared memory and walks a range of 64-token tiles,
+// loading the next tile's dl (16-byte loads, transposed to [head][token]) into
+// registers while the current tile's FMAs and stores run.
+constexpr int kXTilesPerBlock = 8;
 template <typename T>
 __global__ void __launch_bounds__(kXThreads)
 route_bwd_dx_kernel(int64_t BT, int d_model, int h, const T* __restrict__ W, const float* __restrict__ dl,
@@ -53,46 +55,84 @@ route_bwd_dx_kernel(int64_t BT, int d_model, int h, const T* __restrict__ W, con
     __shared__ __align__(16) float WT[kHc][kXCol + 4];
     const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
     const int i0 = blockIdx.x * kXCol, c0 = tx * 4;
-    const int64_t t0 = (int64_t)blockIdx.y * kXTok;
-    float4 acc[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t n_tiles = (BT + kXTok - 1) / kXTok;
+    const int64_t tile_lo = (int64_t)blockIdx.y * kXTilesPerBlock;
+    const int64_t tile_hi = min(n_tiles, tile_lo + kXTilesPerBlock);
+    constexpr int kDV = kXTok * kHc / 4 / kXThreads;  // float4 of dl per thread per tile
+    const bool vec_dl = (h % 4) == 0;
     for (int j0 = 0; j0 < h; j0 += kHc) {
         __syncthreads();
-        for (int c = threadIdx.x; c < kXTok * kHc; c += kXThreads) {
-            const int t = c / kHc, jj = c % kHc;
-            dlT[jj][t] = (t0 + t < BT && j0 + jj < h) ? dl[(t0 + t) * h + j0 + jj] : 0.f;
-        }
         for (int c = threadIdx.x; c < kXCol * kHc; c += kXThreads) {
             const int col = c / kHc, jj = c % kHc;
             WT[jj][col] = (i0 + col < d_model && j0 + jj < h) ? ld<T>(W + (int64_t)(i0 + col) * h + j0 + jj) : 0.f;
         }
-        __syncthreads();
-#pragma unroll 4
-        for (int jj = 0; jj < kHc; ++jj) {
-            const float4 w = *reinterpret_cast<const float4*>(&WT[jj][c0]);
-            const float4 a = *reinterpret_cast<const float4*>(&dlT[jj][ty * 8]);
-            const float4 b = *reinterpret_cast<const float4*>(&dlT[jj][ty * 8 + 4]);
-            fma4(a.x, w, acc[0]);
-            fma4(a.y, w, acc[1]);
-            fma4(a.z, w, acc[2]);
-            fma4(a.w, w, acc[3]);
-            fma4(b.x, w, acc[4]);
-            fma4(b.y, w, acc[5]);
-            fma4(b.z, w, acc[6]);
-            fma4(b.w, w, acc[7]);
-        }
-    }
+        float4 dr[kDV];
+        auto fetch = [&](int64_t tile) {
+            const int64_t t0 = tile * kXTok;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t t = t0 + ty * 8 + r;
-        if (t >= BT) break;
-        float* out = dx + t * d_model + i0 + c0;
-        if (i0 + c0 + 3 < d_model && (d_model & 3) == 0) {
-            *reinterpret_cast<float4*>(out) = acc[r];
-        } else {
-            const float v[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
-            for (int e = 0; e < 4 && i0 + c0 + e < d_model; ++e) out[e] = v[e];
+            for (int v = 0; v < kDV; ++v) {
+                const int c = threadIdx.x + v * kXThreads;  // (token, 4 heads)
+                const int t = c / (kHc / 4), jq = (c % (kHc / 4)) * 4;
+                const int64_t row = t0 + t;
+                if (row < BT && vec_dl && j0 + jq + 3 < h) {
+                    dr[v] = *reinterpret_cast<const float4*>(dl + row * h + j0 + jq);
+                } else {
+                    float e[4];
+                    for (int q = 0; q < 4; ++q) e[q] = (row < BT && j0 + jq + q < h) ? dl[row * h + j0 + jq + q] : 0.f;
+                    dr[v] = make_float4(e[0], e[1], e[2], e[3]);
+                }
+            }
+        };
+        if (tile_lo < tile_hi) fetch(tile_lo);
+        for (int64_t tile = tile_lo; tile < tile_hi; ++tile) {
+            __syncthreads();
+#pragma unroll
+            for (int v = 0; v < kDV; ++v) {
+                const int c = threadIdx.x + v * kXThreads, t = c / (kHc / 4), jq = (c % (kHc / 4)) * 4;
+                dlT[jq][t] = dr[v].x;
+                dlT[jq + 1][t] = dr[v].y;
+                dlT[jq + 2][t] = dr[v].z;
+                dlT[jq + 3][t] = dr[v].w;
+            }
+            __syncthreads();
+            if (tile + 1 < tile_hi) fetch(tile + 1);
+            float4 acc[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int jj = 0; jj < kHc; ++jj) {
+                const float4 w = *reinterpret_cast<const float4*>(&WT[jj][c0]);
+                const float4 a = *reinterpret_cast<const float4*>(&dlT[jj][ty * 8]);
+                const float4 b = *reinterpret_cast<const float4*>(&dlT[jj][ty * 8 + 4]);
+                fma4(a.x, w, acc[0]);
+                fma4(a.y, w, acc[1]);
+                fma4(a.z, w, acc[2]);
+                fma4(a.w, w, acc[3]);
+                fma4(b.x, w, acc[4]);
+                fma4(b.y, w, acc[5]);
+                fma4(b.z, w, acc[6]);
+                fma4(b.w, w, acc[7]);
+            }
+            const int64_t t0 = tile * kXTok;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int64_t t = t0 + ty * 8 + r;
+                if (t >= BT) break;
+                float* out = dx + t * d_model + i0 + c0;
+                if (i0 + c0 + 3 < d_model && (d_model & 3) == 0) {
+                    if (j0 > 0) {  // heads past the first 32: add to the earlier passes' sums
+                        const float4 o = *reinterpret_cast<const float4*>(out);
+                        acc[r].x += o.x;
+                        acc[r].y += o.y;
+                        acc[r].z += o.z;
+                        acc[r].w += o.w;
+                    }
+                    *reinterpret_cast<float4*>(out) = acc[r];
+                } else {
+                    const float v[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+                    for (int e = 0; e < 4 && i0 + c0 + e < d_model; ++e) out[e] = (j0 > 0 ? out[e] : 0.f) + v[e];
+                }
+            }
         }
     }
 }
@@ -112,17 +152,62 @@ route_bwd_dw_kernel(int64_t BT, int d_model, int h, int64_t per_split, const T* 
     float4 acc[8];  // acc[jj] holds heads j0 + ty*8 + jj for columns tx*4 .. tx*4+3
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) acc[jj] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // The next stage's x and dl are loaded into registers while the current
+    // stage's FMAs run (16-byte loads of 8 bf16 or 4 fp32 where the row allows).
+    constexpr int kEV = 16 / sizeof(T);                             // elements per 16-byte vector
+    constexpr int kXV = kWStage * kWCol / kEV / kWThreads;          // x vectors per thread per stage
+    constexpr int kDV = kWStage * kHc / kWThreads;                  // dl values per thread per stage
+    const bool vec_ok = (d_model % kEV) == 0 && i0 + kWCol <= d_model;
+    float xr[kXV][kEV], dr[kDV];
+    auto fetch = [&](int64_t s0) {
+#pragma unroll
+        for (int v = 0; v < kXV; ++v) {
+            const int c = (threadIdx.x + v * kWThreads) * kEV;  // element index in the [kWStage][kWCol] stage
+            const int t = c / kWCol, col = c % kWCol;
+            const int64_t row = s0 + t;
+            if (row < b1 && vec_ok) {
+                const uint4 q = *reinterpret_cast<const uint4*>(x + row * d_model + i0 + col);
+                if constexpr (sizeof(T) == 2) {
+                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        xr[v][2 * e] = __uint_as_float(w[e] << 16);
+                        xr[v][2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                    }
+                } else {
+                    xr[v][0] = __uint_as_float(q.x);
+                    xr[v][1] = __uint_as_float(q.y);
+                    xr[v][2] = __uint_as_float(q.z);
+                    xr[v][3] = __uint_as_float(q.w);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < kEV; ++e)
+                    xr[v][e] = (row < b1 && i0 + col + e < d_model) ? ld<T>(x + row * d_model + i0 + col + e) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < kDV; ++v) {
+            const int c = threadIdx.x + v * kWThreads, t = c / kHc, jj = c % kHc;
+            dr[v] = (s0 + t < b1 && j0 + jj < h) ? dl[(s0 + t) * h + j0 + jj] : 0.f;
+        }
+    };
+    fetch(b0);
     for (int64_t s0 = b0; s0 < b1; s0 += kWStage) {
         __syncthreads();
-        for (int c = threadIdx.x; c < kWStage * kWCol; c += kWThreads) {
-            const int t = c / kWCol, col = c % kWCol;
-            xs[t][col] = (s0 + t < b1 && i0 + col < d_model) ? ld<T>(x + (s0 + t) * d_model + i0 + col) : 0.f;
+#pragma unroll
+        for (int v = 0; v < kXV; ++v) {
+            const int c = (threadIdx.x + v * kWThreads) * kEV, t = c / kWCol, col = c % kWCol;
+#pragma unroll
+            for (int e = 0; e < kEV; ++e) xs[t][col + e] = xr[v][e];
         }
-        for (int c = threadIdx.x; c < kWStage * kHc; c += kWThreads) {
-            const int t = c / kHc, jj = c % kHc;
-            dls[t][jj] = (s0 + t < b1 && j0 + jj < h) ? dl[(s0 + t) * h + j0 + jj] : 0.f;
+#pragma unroll
+        for (int v = 0; v < kDV; ++v) {
+            const int c = threadIdx.x + v * kWThreads;
+            dls[c / kHc][c % kHc] = dr[v];
         }
         __syncthreads();
+        if (s0 + kWStage < b1) fetch(s0 + kWStage);
 #pragma unroll 4
         for (int t = 0; t < kWStage; ++t) {
             const float4 xv = *reinterpret_cast<const float4*>(&xs[t][tx * 4]);
@@ -191,7 +276,8 @@ template <typename T>
 cudaError_t launch_typed(const RouteBwdArgs& a) {
     const gqe_shape& s = *a.s;
     const int64_t BT = (int64_t)s.B * s.T;
-    const dim3 gx((unsigned)((s.d_model + kXCol - 1) / kXCol), (unsigned)((BT + kXTok - 1) / kXTok));
+    const int64_t x_tiles = (BT + kXTok - 1) / kXTok;
+    const dim3 gx((unsigned)((s.d_model + kXCol - 1) / kXCol), (unsigned)((x_tiles + kXTilesPerBlock - 1) / kXTilesPerBlock));
     route_bwd_dx_kernel<T><<<gx, kXThreads, 0, a.stream>>>(BT, s.d_model, s.h, (const T*)a.W_r, a.dlogits, a.dx);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

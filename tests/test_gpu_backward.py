@@ -98,11 +98,19 @@ def gpu_route_backward(w, inp, dlogits):
     return [t.cpu().numpy().astype(np.float64) for t in (dx, dW, db)]
 
 
-@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill"])
+ROUTE_BWD_SMALL = [
+    # two 32-head passes (dx summed over them), a ragged column block and token tile
+    C("rb_h64_ragged", B=1, T=300, d_model=200, h=64, g=8, d_h=128, k=2, seed=97),
+    C("rb_f32_h40", B=2, T=70, d_model=36, h=40, g=4, d_h=64, k=3, dtype="f32", seed=98),
+]
+
+
+@pytest.mark.parametrize("name", ["dense_gqa", "gqe_prefill"] + [w.name for w in ROUTE_BWD_SMALL])
 def test_route_backward_full_size(name):
-    """Router gradients at full size from a seeded gate gradient: the oracle's
-    logit gradients go in, dx, dW_r and dbias are compared in full."""
-    w = W[name]
+    """Router gradients from a seeded gate gradient: the oracle's logit
+    gradients go in, dx, dW_r and dbias are compared in full (at full size,
+    and on small shapes with more than 32 heads and ragged tiles)."""
+    w = W[name] if name in W else next(x for x in ROUTE_BWD_SMALL if x.name == name)
     inp = gqe_synth.make_inputs(w)
     idx_o, gate_o, _, _ = U.oracle_route(w, inp)
     dgate = np.random.default_rng(w.seed + 7).standard_normal(idx_o.shape)
