@@ -15,17 +15,22 @@
 //
 // Roles (384 threads, one persistent CTA per SM):
 //   warp 0      TMA producer for K/V tiles; owns the TMEM allocation
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V on tcgen05
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T on tcgen05 (the training
+//               instance issues O_t += P_t V here too)
 //   warp 2      row tables and Q tiles: one TMA box per head and half when every
 //               token of the half-window selected every head of the group (dense
 //               GQA), TMA tile::gather4 of the routed rows otherwise (128B-swizzled)
-//   warp 3      zero fill of the window's unselected output slots
-//   warps 4-7   softmax + epilogue of Q tile 0 (one row per thread)
-//   warps 8-11  softmax + epilogue of Q tile 1
-// The two softmax warpgroups alternate with the tensor core: while one turns
-// S into P, the tensor core runs the other tile's P.V and next QK^T.
-// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512); P_t (bf16
-// pairs) overwrites the first 64 columns of S_t once S_t is in registers.
+//   warp 3      MMA issuer (one thread): O_t += P_t V (inference instances)
+//   warps 4-7   softmax + epilogue of Q tile 0 (one row per thread), and the zero
+//               fill of its half-window's unselected output slots
+//   warps 8-11  the same for Q tile 1
+// TMEM columns (inference instances): one S buffer [0,128) that the tiles take
+// in turn, P_0 [128,192) and P_1 [192,256) (bf16 pairs), O_0 [256,384), O_1
+// [384,512).  A softmax warpgroup reads S into registers and hands the buffer
+// back at once, so the next S is computed while it exponentiates; with P in its
+// own slot the next S does not wait for this tile's P.V either.  The training
+// instance keeps S_t in [128 t, 128 t + 128) with P_t (and R = p - bf16(p))
+// overwriting it, because its P and R need 128 columns per tile.
 #include <atomic>
 #include <climits>
 
@@ -48,6 +53,10 @@ constexpr uint32_t kHalf = 128 * 64 * 2;   // one [128][64] bf16 box, 16 KB
 constexpr uint32_t kTileBytes = 2 * kHalf; // [128][128] bf16, 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * tile
+// Inference instances: one S buffer that the two tiles take in turn and a P
+// slot per tile (bf16 pairs, P_t at kColP + 64 * tile), so a tile's next S is
+// computed while its softmax still turns the current one into P.
+constexpr uint32_t kColSbuf = 0, kColP = 128;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: p <= 2^8 between rescales
 // Of every 16 element pairs of an unmasked tile, exp2 on the FMA pipe
 // (exp2_poly2) for this many, on MUFU for the rest.  A same-box sweep with
@@ -71,7 +80,8 @@ struct Smem {
     int32_t cut_prefix[2][kQT][33];
     uint64_t kv_full_k[2], kv_full_v[2], kv_empty_k[2], kv_empty_v[2];
     uint64_t s_full[kQT], p_full[kQT], o_full[kQT], o_empty[kQT];
-    uint64_t q_full[2], q_empty, rows_free[2], mma_drain;
+    uint64_t s_free, p_empty[kQT];  // shared-S layout: S buffer read out, P slot consumed
+    uint64_t q_full[2], q_empty, rows_free[2], mma_drain, mma_drain2;
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -168,6 +178,64 @@ __device__ __forceinline__ void ld_bind(uint32_t (&r)[32]) {
 
 
 // ---------------------------------------------------------------------------
+// TMEM columns of S_t and P_t.  The training instance keeps S_t and P_t (with
+// R = p - bf16(p) in columns 64-127) in the tile's own 128 columns; the others
+// use one S buffer that the tiles take in turn, and a 64-column P slot per tile.
+template <bool kSB>
+__device__ __forceinline__ uint32_t s_col(int t) { return kSB ? kColSbuf : kColS + 128u * t; }
+template <bool kSB>
+__device__ __forceinline__ uint32_t p_col(int t) { return kSB ? kColP + 64u * t : kColS + 128u * t; }
+
+// The issuing thread's view of the two GEMMs.  Shared-memory descriptors are
+// built once: a K step only moves the start address (16-byte units in the low
+// word), so each MMA adds a compile-time offset instead of rebuilding the
+// descriptor (the issuing thread's scalar work would otherwise outlast the
+// MMAs).  The high word (stride offset 1024, 128-byte swizzle) is shared by
+// every operand here.
+template <bool kSB, bool kTrain>
+struct MmaIssue {
+    // scalars, not arrays: a runtime index into a member array would put it in local memory
+    uint32_t tmem, dhi, qlo0, qlo1, klo0, klo1, vlo0, vlo1, idesc_s, idesc_pv;
+    __device__ MmaIssue(Smem& sm, uint32_t tmem_base)
+        : tmem(tmem_base),
+          dhi(smem_desc_hi(1024, kSwizzle128B)),
+          qlo0(smem_desc_lo(smem_u32(sm.q[0]), 16)),
+          qlo1(smem_desc_lo(smem_u32(sm.q[1]), 16)),
+          klo0(smem_desc_lo(smem_u32(sm.k[0]), 16)),
+          klo1(smem_desc_lo(smem_u32(sm.k[1]), 16)),
+          vlo0(smem_desc_lo(smem_u32(sm.v[0]), kHalf)),
+          vlo1(smem_desc_lo(smem_u32(sm.v[1]), kHalf)),
+          idesc_s(idesc_bf16_f32(kBM, kBN, false, false)),
+          idesc_pv(idesc_bf16_f32(kBM, kD, false, true)) {}
+    __device__ __forceinline__ uint64_t desc(uint32_t lo) const { return smem_desc_join(lo, dhi); }
+    // S_t = Q_t K(it)^T into S_t's columns
+    __device__ __forceinline__ void s(int t, uint32_t it) const {
+        const uint32_t a0 = t ? qlo1 : qlo0, b0 = (it & 1) ? klo1 : klo0;
+        const uint32_t d = tmem + s_col<kSB>(t);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+            umma_ss(d, desc(a0 + off), desc(b0 + off), idesc_s, kk > 0 ? 1u : 0u);
+        }
+    }
+    // O_t += P_t V(it).  For the training outputs P.V runs over [P | R] against
+    // V twice: R holds p - bf16(p), so o is accurate far beyond bf16 P (the
+    // backward's D = g dO . o needs it).
+    __device__ __forceinline__ void pv(int t, uint32_t it, bool first) const {
+        const uint32_t b0 = (it & 1) ? vlo1 : vlo0;
+        const uint32_t d = tmem + kColO + t * 128, a = tmem + p_col<kSB>(t);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(d, a + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        if (kTrain) {
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+                umma_ts(d, a + 64 + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, 1u);
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
 // kTrain: also write the training outputs (o32, lse); O only when asked.
 // kSplit: split-KV items (p.nsplit > 1); the plain instance carries none of it.
 template <bool kTrain, bool kSplit>
@@ -181,6 +249,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     const UnitGeom& u = p.u;
     const int nsplit = kSplit ? p.nsplit : 1;
     const int64_t n_units = u.count() * nsplit;  // work items (units when not split)
+    // TMEM layout: the training instance keeps S_t and P_t (with R = p - bf16(p))
+    // in the tile's own 128 columns; the others use the shared S buffer.
+    constexpr bool kSB = !kTrain;
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -196,9 +267,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             mbar_init(&sm.p_full[t], 128);
             mbar_init(&sm.o_full[t], 1);
             mbar_init(&sm.o_empty[t], 128);
+            mbar_init(&sm.p_empty[t], 1);
         }
+        mbar_init(&sm.s_free, 4);  // one arrive per warp of the tile's warpgroup
         mbar_init(&sm.q_empty, 1);
         mbar_init(&sm.mma_drain, 1);
+        mbar_init(&sm.mma_drain2, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
     }
@@ -258,104 +332,105 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         }
     } else if (warp == 1) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ MMA issuer (S; all MMAs when training)
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
-            const uint32_t idesc_pv = idesc_bf16_f32(kBM, kD, false, true);
+            const MmaIssue<kSB, kTrain> mma(sm, tmem);
             uint32_t kv_it = 0, u_it = 0, c[kQT] = {0, 0};
             bool ok = true;
-            // Shared-memory descriptors are built once: a K step only moves the
-            // start address (16-byte units in the low word), so each MMA adds a
-            // compile-time offset instead of rebuilding the descriptor (the
-            // single issuing thread's scalar work would otherwise outlast the
-            // MMAs).  The high word (stride offset 1024, 128-byte swizzle) is
-            // shared by every operand here.
-            const uint32_t dhi = smem_desc_hi(1024, kSwizzle128B);
-            const uint32_t qlo0 = smem_desc_lo(smem_u32(sm.q[0]), 16), qlo1 = smem_desc_lo(smem_u32(sm.q[1]), 16);
-            const uint32_t klo0 = smem_desc_lo(smem_u32(sm.k[0]), 16), klo1 = smem_desc_lo(smem_u32(sm.k[1]), 16);
-            const uint32_t vlo0 = smem_desc_lo(smem_u32(sm.v[0]), kHalf), vlo1 = smem_desc_lo(smem_u32(sm.v[1]), kHalf);
-            auto desc = [&](uint32_t lo) { return smem_desc_join(lo, dhi); };
-            auto issue_s = [&](int t, uint32_t it) {
-                const uint32_t a0 = t ? qlo1 : qlo0, b0 = (it & 1) ? klo1 : klo0;
-                const uint32_t d = tmem + kColS + t * 128;
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (uint32_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
-                    umma_ss(d, desc(a0 + off), desc(b0 + off), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&sm.s_full[t]);
-            };
-            // For the training outputs P.V runs over [P | R] against V twice: R (in
-            // S's columns 64-127) holds p - bf16(p), so o is accurate far beyond
-            // bf16 P (the backward's D = g dO . o needs it).
-            constexpr bool train = kTrain;
-            auto issue_pv = [&](int t, uint32_t it, bool first) {
-                const uint32_t b0 = (it & 1) ? vlo1 : vlo0;
-                const uint32_t d = tmem + kColO + t * 128, a = tmem + kColS + t * 128;
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    umma_ts(d, a + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
-                if (train) {
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        umma_ts(d, a + 64 + kk * 8, desc(b0 + (uint32_t)((kk * 2048) >> 4)), idesc_pv, 1u);
-                }
-            };
             auto wait_k = [&](uint32_t it) { return mbar_wait(&sm.kv_full_k[it & 1], (it >> 1) & 1); };
             auto wait_v = [&](uint32_t it) { return mbar_wait(&sm.kv_full_v[it & 1], (it >> 1) & 1); };
-            for (int64_t j = 0; ok; ++j) {
-                const int64_t item = cta_unit(j, n_units);
-                if (item < 0 || aborted(sm)) break;
-                int64_t unit;
-                int split, b, q, w, kv_lo, cnt[kQT];
-                item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
-                const int n0 = cnt[0], n1 = cnt[1];
-                if (n1 == 0) continue;  // an empty split: every role skips it
-                const uint32_t ui = u_it++;
-                const int qs = ui & 1;
-                if (!mbar_wait(&sm.q_full[qs], (ui >> 1) & 1)) { fail(sm, p, 10); break; }
-                tc_fence_after();
-                if (!wait_k(kv_it)) { fail(sm, p, 11); break; }
-                tc_fence_after();
-                if (n0 > 0) issue_s(0, kv_it);
-                issue_s(1, kv_it);
-                umma_commit(&sm.kv_empty_k[kv_it & 1]);
-                if (n1 == 1) umma_commit(&sm.q_empty);
-                for (int i = 0; i < n1; ++i) {
-                    const uint32_t it = kv_it + i;
-                    if (i < n0) {
-                        ok = mbar_wait(&sm.p_full[0], (c[0] + i) & 1);
-                        if (ok && i == 0) ok = mbar_wait(&sm.o_empty[0], (ui & 1) ^ 1);
-                        if (ok) ok = wait_v(it);
-                        if (!ok) { fail(sm, p, 12); break; }
-                        tc_fence_after();
-                        issue_pv(0, it, i == 0);
-                        if (i == n0 - 1) umma_commit(&sm.o_full[0]);
-                        if (i + 1 < n0) {
-                            if (!wait_k(it + 1)) { fail(sm, p, 13); ok = false; break; }
+            if constexpr (kSB) {
+                // S_t(i) of every step, tile 0 first, into the shared S buffer:
+                // each waits until the previous S has been read out by its
+                // softmax (s_free), so S of the next step is computed while the
+                // softmax warps still work on the current one.  P.V is issued by
+                // warp 3.
+                uint32_t s_cnt = 0;
+                for (int64_t j = 0; ok; ++j) {
+                    const int64_t item = cta_unit(j, n_units);
+                    if (item < 0 || aborted(sm)) break;
+                    int64_t unit;
+                    int split, b, q, w, kv_lo, cnt[kQT];
+                    item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+                    const int n0 = cnt[0], n1 = cnt[1];
+                    if (n1 == 0) continue;  // an empty split: every role skips it
+                    const uint32_t ui = u_it++;
+                    if (!mbar_wait(&sm.q_full[ui & 1], (ui >> 1) & 1)) { fail(sm, p, 10); break; }
+                    for (int i = 0; i < n1 && ok; ++i, ++kv_it) {
+                        if (!wait_k(kv_it)) { fail(sm, p, 11); ok = false; break; }
+                        for (int t = (i < n0) ? 0 : 1; t < kQT; ++t) {
+                            if (s_cnt > 0 && !mbar_wait(&sm.s_free, (s_cnt - 1) & 1)) { fail(sm, p, 12); ok = false; break; }
                             tc_fence_after();
-                            issue_s(0, it + 1);
+                            mma.s(t, kv_it);
+                            umma_commit(&sm.s_full[t]);
+                            ++s_cnt;
                         }
-                    }
-                    ok = mbar_wait(&sm.p_full[1], (c[1] + i) & 1);
-                    if (ok && i == 0) ok = mbar_wait(&sm.o_empty[1], (ui & 1) ^ 1);
-                    if (ok) ok = wait_v(it);
-                    if (!ok) { fail(sm, p, 14); break; }
-                    tc_fence_after();
-                    issue_pv(1, it, i == 0);
-                    umma_commit(&sm.kv_empty_v[it & 1]);
-                    if (i == n1 - 1) umma_commit(&sm.o_full[1]);
-                    if (i + 1 < n1) {
-                        if (!wait_k(it + 1)) { fail(sm, p, 15); ok = false; break; }
-                        tc_fence_after();
-                        issue_s(1, it + 1);
-                        umma_commit(&sm.kv_empty_k[(it + 1) & 1]);
-                        if (i + 1 == n1 - 1) umma_commit(&sm.q_empty);
+                        if (!ok) break;
+                        umma_commit(&sm.kv_empty_k[kv_it & 1]);
+                        if (i == n1 - 1) umma_commit(&sm.q_empty);
                     }
                 }
-                kv_it += n1;
-                c[0] += n0;
-                c[1] += n1;
+            } else {
+                for (int64_t j = 0; ok; ++j) {
+                    const int64_t item = cta_unit(j, n_units);
+                    if (item < 0 || aborted(sm)) break;
+                    int64_t unit;
+                    int split, b, q, w, kv_lo, cnt[kQT];
+                    item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+                    const int n0 = cnt[0], n1 = cnt[1];
+                    if (n1 == 0) continue;  // an empty split: every role skips it
+                    const uint32_t ui = u_it++;
+                    const int qs = ui & 1;
+                    if (!mbar_wait(&sm.q_full[qs], (ui >> 1) & 1)) { fail(sm, p, 10); break; }
+                    tc_fence_after();
+                    if (!wait_k(kv_it)) { fail(sm, p, 11); break; }
+                    tc_fence_after();
+                    if (n0 > 0) {
+                        mma.s(0, kv_it);
+                        umma_commit(&sm.s_full[0]);
+                    }
+                    mma.s(1, kv_it);
+                    umma_commit(&sm.s_full[1]);
+                    umma_commit(&sm.kv_empty_k[kv_it & 1]);
+                    if (n1 == 1) umma_commit(&sm.q_empty);
+                    for (int i = 0; i < n1; ++i) {
+                        const uint32_t it = kv_it + i;
+                        if (i < n0) {
+                            ok = mbar_wait(&sm.p_full[0], (c[0] + i) & 1);
+                            if (ok && i == 0) ok = mbar_wait(&sm.o_empty[0], (ui & 1) ^ 1);
+                            if (ok) ok = wait_v(it);
+                            if (!ok) { fail(sm, p, 12); break; }
+                            tc_fence_after();
+                            mma.pv(0, it, i == 0);
+                            if (i == n0 - 1) umma_commit(&sm.o_full[0]);
+                            if (i + 1 < n0) {
+                                if (!wait_k(it + 1)) { fail(sm, p, 13); ok = false; break; }
+                                tc_fence_after();
+                                mma.s(0, it + 1);
+                                umma_commit(&sm.s_full[0]);
+                            }
+                        }
+                        ok = mbar_wait(&sm.p_full[1], (c[1] + i) & 1);
+                        if (ok && i == 0) ok = mbar_wait(&sm.o_empty[1], (ui & 1) ^ 1);
+                        if (ok) ok = wait_v(it);
+                        if (!ok) { fail(sm, p, 14); break; }
+                        tc_fence_after();
+                        mma.pv(1, it, i == 0);
+                        umma_commit(&sm.kv_empty_v[it & 1]);
+                        if (i == n1 - 1) umma_commit(&sm.o_full[1]);
+                        if (i + 1 < n1) {
+                            if (!wait_k(it + 1)) { fail(sm, p, 15); ok = false; break; }
+                            tc_fence_after();
+                            mma.s(1, it + 1);
+                            umma_commit(&sm.s_full[1]);
+                            umma_commit(&sm.kv_empty_k[(it + 1) & 1]);
+                            if (i + 1 == n1 - 1) umma_commit(&sm.q_empty);
+                        }
+                    }
+                    kv_it += n1;
+                    c[0] += n0;
+                    c[1] += n1;
+                }
             }
             // Drain: all issued MMAs complete before TMEM is released.
             umma_commit(&sm.mma_drain);
@@ -508,63 +583,41 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         if (armed >= 0) mbar_wait(&sm.q_full[armed & 1], (armed >> 1) & 1);
     } else if (warp == 3) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
-        // ------------------------------------------------------------ zero fill of unselected slots
-        // The unit's window [w0, w0 + 2W) x heads of group q, one W-position half
-        // at a time: slots whose head the token did not select are written as
-        // zeros.  Each lane owns up to 4 of the half's tokens and loads their k
-        // selections at once; the warp then zeroes the unselected 256-byte
-        // slots, 16 lanes per slot.
-        const uint32_t group_mask = (u.hpg >= 32) ? 0xffffffffu : ((1u << u.hpg) - 1u);
-        for (int64_t j = 0; p.O != nullptr; ++j) {  // a recompute for the backward leaves O alone
-            const int64_t item = cta_unit(j, n_units);
-            if (item < 0 || aborted(sm)) break;
-            if (kSplit && item % nsplit != 0) continue;  // a unit's first split zero-fills its window
-            int b, q, w;
-            unit_coords(u, item / nsplit, b, q, w);
-            for (int half = 0; half < kQT; ++half) {
-                const int w0 = (w * kQT + half) * u.W;
-                const int nt = min(w0 + u.W, u.T) - w0;  // tokens in the half, <= 128
-                if (nt <= 0) break;
-                int sj[kBM / 32][4];
-#pragma unroll
-                for (int i = 0; i < kBM / 32; ++i) {
-                    const int tt = lane + 32 * i;
-                    const int64_t sel = (((int64_t)b * u.T + w0 + tt) * u.g + q) * u.k;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) sj[i][s] = (tt < nt && s < u.k) ? p.idx[sel + s] : -1;
-                }
-                uint32_t unsel[kBM / 32];
-                bool any = false;
-#pragma unroll
-                for (int i = 0; i < kBM / 32; ++i) {
-                    uint32_t m = 0;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const int a = sj[i][s] - q * u.hpg;  // head within the group
-                        if (a >= 0 && a < u.hpg) m |= 1u << a;
-                    }
-                    unsel[i] = (lane + 32 * i < nt) ? (~m & group_mask) : 0u;
-                    any |= unsel[i] != 0u;
-                }
-                if (!__any_sync(0xffffffffu, any)) continue;
-                for (int tt = 0; tt < nt; ++tt) {
-                    uint32_t un = __shfl_sync(0xffffffffu, unsel[0], tt & 31);
-#pragma unroll
-                    for (int i = 1; i < kBM / 32; ++i) {
-                        const uint32_t v = __shfl_sync(0xffffffffu, unsel[i], tt & 31);
-                        if ((tt >> 5) == i) un = v;
-                    }
-                    __nv_bfloat16* orow = p.O + (((int64_t)b * u.T + w0 + tt) * u.h + q * u.hpg) * kD;
-                    while (un != 0u) {
-                        // two slots per pass: the lowest set bit for lanes 0-15, the next for 16-31
-                        const int a0 = __ffs(un) - 1;
-                        un &= un - 1u;
-                        const int a1 = (un != 0u) ? __ffs(un) - 1 : -1;
-                        if (a1 >= 0) un &= un - 1u;
-                        const int a = (lane < 16) ? a0 : a1;
-                        if (a >= 0) reinterpret_cast<uint4*>(orow + (int64_t)a * kD)[lane & 15] = make_uint4(0, 0, 0, 0);
+        if constexpr (kSB) {
+            // -------------------------------------------------------- MMA issuer (P.V)
+            // O_t += P_t(i) V(i) once the softmax has written P_t(i) to the
+            // tile's P slot; each completion hands the slot back (p_empty).
+            if (lane == 0) {
+                const MmaIssue<kSB, kTrain> mma(sm, tmem);
+                uint32_t kv_it = 0, u_it = 0, c[kQT] = {0, 0};
+                bool ok = true;
+                for (int64_t j = 0; ok; ++j) {
+                    const int64_t item = cta_unit(j, n_units);
+                    if (item < 0 || aborted(sm)) break;
+                    int64_t unit;
+                    int split, b, q, w, kv_lo, cnt[kQT];
+                    item_range(u, nsplit, item, unit, split, b, q, w, kv_lo, cnt);
+                    const int n0 = cnt[0], n1 = cnt[1];
+                    if (n1 == 0) continue;  // an empty split
+                    const uint32_t ui = u_it++;
+                    for (int i = 0; i < n1 && ok; ++i, ++kv_it) {
+                        if (!mbar_wait(&sm.kv_full_v[kv_it & 1], (kv_it >> 1) & 1)) { fail(sm, p, 17); ok = false; break; }
+                        for (int t = (i < n0) ? 0 : 1; t < kQT; ++t) {
+                            ok = mbar_wait(&sm.p_full[t], c[t] & 1);
+                            if (ok && i == 0) ok = mbar_wait(&sm.o_empty[t], (ui & 1) ^ 1);
+                            if (!ok) { fail(sm, p, 18); break; }
+                            tc_fence_after();
+                            mma.pv(t, kv_it, i == 0);
+                            umma_commit(&sm.p_empty[t]);
+                            ++c[t];
+                            if (i == (t ? n1 : n0) - 1) umma_commit(&sm.o_full[t]);
+                        }
+                        if (!ok) break;
+                        umma_commit(&sm.kv_empty_v[kv_it & 1]);
                     }
                 }
+                umma_commit(&sm.mma_drain2);
+                mbar_wait(&sm.mma_drain2, 0);
             }
         }
     } else {
@@ -574,7 +627,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         const int wq = warp & 3;           // TMEM lane quarter of this warp
         const int r = wq * 32 + lane;      // routed row owned by this thread
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t s_addr = tmem + lane_off + kColS + t * 128;
+        const uint32_t s_addr = tmem + lane_off + s_col<kSB>(t);
+        const uint32_t p_addr = tmem + lane_off + p_col<kSB>(t);
         const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
         constexpr bool train = kTrain;  // also write R = p - bf16(p) for the exact P.V
         uint32_t ctile = 0, u_it = 0, o_it = 0;  // S tiles, items, O_t completions waited
@@ -588,6 +642,38 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             const uint32_t ui = u_it++;
             const int n = cnt[t];
             const int rs = ui & 1;
+            // Zero fill of the tile's half-window [lo, lo + W): every slot whose
+            // head the token did not select is written as zeros (a unit's first
+            // split does it; a recompute for the backward leaves O alone).  It
+            // needs neither Q nor S, so it runs while the unit's Q tiles load.
+            // Each token has 128 / W threads; thread r takes every (128 / W)-th
+            // head of the token's complement.
+            if (p.O != nullptr && (!kSplit || split == 0)) {
+                const int lo = (w * kQT + t) * u.W;
+                const int tpt = kBM / u.W;  // threads per token: 1, 2 or 4
+                const int tok = lo + r / tpt;
+                if (tok < min(lo + u.W, u.T)) {
+                    const int64_t sel = (((int64_t)b * u.T + tok) * u.g + q) * u.k;
+                    uint64_t chosen = 0;
+#pragma unroll
+                    for (int s2 = 0; s2 < 4; ++s2) {
+                        if (s2 < u.k) {
+                            const int a = p.idx[sel + s2] - q * u.hpg;  // head within the group
+                            if (a >= 0 && a < u.hpg) chosen |= 1ull << a;
+                        }
+                    }
+                    uint64_t un = ~chosen & ((u.hpg >= 64) ? ~0ull : ((1ull << u.hpg) - 1ull));
+                    uint4* orow = reinterpret_cast<uint4*>(p.O + (((int64_t)b * u.T + tok) * u.h + q * u.hpg) * kD);
+                    for (int c = 0; un != 0ull; ++c) {
+                        const int a = __ffsll((long long)un) - 1;
+                        un &= un - 1ull;
+                        if (c % tpt != r % tpt) continue;
+                        uint4* dst = orow + (int64_t)a * (kD * 2 / 16);
+#pragma unroll
+                        for (int v = 0; v < kD * 2 / 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full[rs], (ui >> 1) & 1))) {
                 if (lane == 0) fail(sm, p, 30);
                 break;
@@ -604,65 +690,62 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                     break;
                 }
                 tc_fence_after();
+                // The tile's scores, four 32-column chunks.  On an unmasked tile
+                // after the first, the exponentials are taken against the running
+                // max m while the tile's row max is formed alongside: when no row
+                // of the warp grew its max by more than the rescale threshold (the
+                // usual case) P is final, else the general path below redoes the
+                // tile from the scores, which stay in registers.  The first
+                // chunk's exponentials start while the other three load.
                 uint32_t s[4][32];
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tmem_ld32(s_addr + cb * 32, s[cb]);
-                ld_wait_bind(s[0]);
-                ld_bind(s[1]);
-                ld_bind(s[2]);
-                ld_bind(s[3]);
                 const int kv0 = (kv_lo + i) * kBN;
                 const bool need_mask = kv0 + kBN - 1 > lo;
-                if (need_mask) {
-#pragma unroll
-                    for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (kv0 + cb * 32 + e > t_eff) s[cb][e] = __float_as_uint(-INFINITY);
-                }
-                // row max of the raw scores: four independent 3-input max chains
-                float mq[4];
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    float a0 = __uint_as_float(s[cb][0]);
-#pragma unroll
-                    for (int e = 1; e < 31; e += 2)
-                        a0 = fmax3(a0, __uint_as_float(s[cb][e]), __uint_as_float(s[cb][e + 1]));
-                    mq[cb] = fmaxf(a0, __uint_as_float(s[cb][31]));
-                }
-                const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
-                // Lazy rescaling: keep the running max unless it grows by more than the threshold.
-                float m_use = m;
-                bool rescale = false;
-                if (mx > m + kRescaleThreshold || m == -INFINITY) {
-                    m_use = mx;
-                    rescale = (i > 0);
-                }
-                // S_t of this tile is complete, so O_t already holds P.V of every
-                // earlier tile (the commit that signalled s_full covers them).
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float alpha = rescale ? fast_exp2(m - m_use) : 1.0f;
-#pragma unroll 1
-                    for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t o[32];
-                        tmem_ld32(o_addr + cb * 32, o);
-                        ld_wait_bind(o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st16(o_addr + cb * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-                        tmem_st16(o_addr + cb * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
-                    }
-                    l *= alpha;
-                }
-                // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
-                // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
+                const bool spec = !need_mask && i > 0;  // the same for the whole warp
                 const uint64_t C2 = pk2(p.scale_log2, p.scale_log2);
-                const uint64_t NM2 = pk2(-m_use, -m_use);
                 uint64_t sum2[4] = {0, 0, 0, 0};
-                if (need_mask) {
+                float m_use = m;
+                bool rescale = false, done = false, slot_ok = true;
+                // Shared S buffer: read it out whole and hand it back to the next S.
+                if constexpr (kSB) {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) tmem_ld32(s_addr + cb * 32, s[cb]);
+                    ld_wait_bind(s[0]);
+                    ld_bind(s[1]);
+                    ld_bind(s[2]);
+                    ld_bind(s[3]);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.s_free);
+                }
+                // P slot of this tile: free once the tile's previous P.V has
+                // completed (which also completes O_t up to the previous tile).
+                auto wait_slot = [&]() {
+                    if (ctile > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.p_empty[t], (ctile - 1) & 1)))
+                        slot_ok = false;
+                    tc_fence_after();
+                };
+                if (spec) {
+                    if constexpr (!kSB) {
+                        tmem_ld32(s_addr, s[0]);
+                        ld_wait_bind(s[0]);
+#pragma unroll
+                        for (int cb = 1; cb < 4; ++cb) tmem_ld32(s_addr + cb * 32, s[cb]);
+                    }
+                    const uint64_t NM2 = pk2(-m, -m);
+                    float mq[4];
+                    uint32_t pk[4][16], rk[4][16];
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t pk[16], rk[16];
+                        if (!kSB && cb == 1) {
+                            ld_wait_bind(s[1]);
+                            ld_bind(s[2]);
+                            ld_bind(s[3]);
+                        }
+                        float a0 = __uint_as_float(s[cb][0]);
+#pragma unroll
+                        for (int e = 1; e < 31; e += 2)
+                            a0 = fmax3(a0, __uint_as_float(s[cb][e]), __uint_as_float(s[cb][e + 1]));
+                        mq[cb] = fmaxf(a0, __uint_as_float(s[cb][31]));
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             float x0, x1;
@@ -670,39 +753,129 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                                 x0, x1);
                             const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                             sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
-                            pk[e] = pack_bf16x2(p0, p1);
-                            if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
-                                                           p1 - __uint_as_float(pk[e] & 0xffff0000u));
+                            pk[cb][e] = pack_bf16x2(p0, p1);
+                            if (train) rk[cb][e] = pack_bf16x2(p0 - __uint_as_float(pk[cb][e] << 16),
+                                                               p1 - __uint_as_float(pk[cb][e] & 0xffff0000u));
                         }
-                        tmem_st16(s_addr + cb * 16, pk);
-                        if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
+                        if constexpr (kSB) {
+                            // the first two chunks wait in registers for the slot
+                            if (cb == 1) {
+                                wait_slot();
+                                tmem_st16(p_addr, pk[0]);
+                                tmem_st16(p_addr + 16, pk[1]);
+                            } else if (cb > 1) {
+                                tmem_st16(p_addr + cb * 16, pk[cb]);
+                            }
+                        } else {
+                            tmem_st16(p_addr + cb * 16, pk[cb]);
+                            if (train) tmem_st16(s_addr + 64 + cb * 16, rk[cb]);
+                        }
                     }
-                } else {
+                    const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
+                    done = __all_sync(0xffffffffu, mx <= m + kRescaleThreshold);
+                    if (!done) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sum2[e] = 0;
+                    }
+                } else if constexpr (!kSB) {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) tmem_ld32(s_addr + cb * 32, s[cb]);
+                    ld_wait_bind(s[0]);
+                    ld_bind(s[1]);
+                    ld_bind(s[2]);
+                    ld_bind(s[3]);
+                }
+                if (!done) {
+                    if (need_mask) {
+#pragma unroll
+                        for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (kv0 + cb * 32 + e > t_eff) s[cb][e] = __float_as_uint(-INFINITY);
+                    }
+                    // row max of the raw scores: four independent 3-input max chains
+                    float mq[4];
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
-                        uint32_t pk[16], rk[16];
+                        float a0 = __uint_as_float(s[cb][0]);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const uint64_t x2 =
-                                ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2);
-                            float p0, p1;
-                            if (e < kPolyPairs) {
-                                float x0, x1;
-                                up2(x2, x0, x1);
-                                up2(exp2_poly2_clamped(x0, x1), p0, p1);
-                            } else {
-                                float x0, x1;
-                                up2(x2, x0, x1);
-                                p0 = fast_exp2(x0);
-                                p1 = fast_exp2(x1);
-                            }
-                            sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
-                            pk[e] = pack_bf16x2(p0, p1);
-                            if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
-                                                           p1 - __uint_as_float(pk[e] & 0xffff0000u));
+                        for (int e = 1; e < 31; e += 2)
+                            a0 = fmax3(a0, __uint_as_float(s[cb][e]), __uint_as_float(s[cb][e + 1]));
+                        mq[cb] = fmaxf(a0, __uint_as_float(s[cb][31]));
+                    }
+                    const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
+                    // Lazy rescaling: keep the running max unless it grows by more than the threshold.
+                    if (mx > m + kRescaleThreshold || m == -INFINITY) {
+                        m_use = mx;
+                        rescale = (i > 0);
+                    }
+                    // O_t must hold P.V of every earlier tile: in the shared-S layout
+                    // the tile's previous P.V has completed once the slot is free; in
+                    // the other, S_t's completion covers it (the same commit).
+                    if constexpr (kSB) wait_slot();
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        const float alpha = rescale ? fast_exp2(m - m_use) : 1.0f;
+#pragma unroll 1
+                        for (int cb = 0; cb < 4; ++cb) {
+                            uint32_t o[32];
+                            tmem_ld32(o_addr + cb * 32, o);
+                            ld_wait_bind(o);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st16(o_addr + cb * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+                            tmem_st16(o_addr + cb * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
                         }
-                        tmem_st16(s_addr + cb * 16, pk);
-                        if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
+                        l *= alpha;
+                    }
+                    // p = 2^(s*c - m): one packed FMA per pair; exp2 on MUFU, or for
+                    // kPolyPairs of every 16 pairs of an unmasked tile on the FMA pipe.
+                    const uint64_t NM2 = pk2(-m_use, -m_use);
+                    if (need_mask) {
+#pragma unroll
+                        for (int cb = 0; cb < 4; ++cb) {
+                            uint32_t pk[16], rk[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                float x0, x1;
+                                up2(ffma2(pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2,
+                                          NM2),
+                                    x0, x1);
+                                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                                sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
+                                pk[e] = pack_bf16x2(p0, p1);
+                                if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
+                                                               p1 - __uint_as_float(pk[e] & 0xffff0000u));
+                            }
+                            tmem_st16(p_addr + cb * 16, pk);
+                            if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
+                        }
+                    } else {
+#pragma unroll
+                        for (int cb = 0; cb < 4; ++cb) {
+                            uint32_t pk[16], rk[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const uint64_t x2 = ffma2(
+                                    pk2(__uint_as_float(s[cb][2 * e]), __uint_as_float(s[cb][2 * e + 1])), C2, NM2);
+                                float p0, p1;
+                                if (e < kPolyPairs) {
+                                    float x0, x1;
+                                    up2(x2, x0, x1);
+                                    up2(exp2_poly2_clamped(x0, x1), p0, p1);
+                                } else {
+                                    float x0, x1;
+                                    up2(x2, x0, x1);
+                                    p0 = fast_exp2(x0);
+                                    p1 = fast_exp2(x1);
+                                }
+                                sum2[e & 3] = fadd2(sum2[e & 3], pk2(p0, p1));
+                                pk[e] = pack_bf16x2(p0, p1);
+                                if (train) rk[e] = pack_bf16x2(p0 - __uint_as_float(pk[e] << 16),
+                                                               p1 - __uint_as_float(pk[e] & 0xffff0000u));
+                            }
+                            tmem_st16(p_addr + cb * 16, pk);
+                            if (train) tmem_st16(s_addr + 64 + cb * 16, rk);
+                        }
                     }
                 }
                 float sa, sb;
@@ -713,6 +886,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&sm.p_full[t]);
+                if (!slot_ok) {
+                    if (lane == 0) fail(sm, p, 36);
+                    ok = false;
+                    break;
+                }
             }
             if (!ok) break;
             const int j_row = sm.row_j[rs][t][r];
@@ -790,27 +968,57 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
             }
             const float f = (t_row >= 0) ? sm.row_gate[rs][t][r] / l : 0.f;
             __nv_bfloat16* orow = p.O + orow_idx * kD;
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t o[32];
-                tmem_ld32(o_addr + cb * 32, o);
-                ld_wait_bind(o);
-                if (t_row >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+            if constexpr (kSB) {
+                // O_t whole into registers; O_t and the row table go back to the
+                // next unit before the global stores.
+                uint32_t o[4][32];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * f, __uint_as_float(o[8 * v + 1]) * f);
-                        pk.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * f, __uint_as_float(o[8 * v + 3]) * f);
-                        pk.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * f, __uint_as_float(o[8 * v + 5]) * f);
-                        pk.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * f, __uint_as_float(o[8 * v + 7]) * f);
-                        dst[v] = pk;
+                for (int cb = 0; cb < 4; ++cb) tmem_ld32(o_addr + cb * 32, o[cb]);
+                ld_wait_bind(o[0]);
+                ld_bind(o[1]);
+                ld_bind(o[2]);
+                ld_bind(o[3]);
+                tc_fence_before();
+                mbar_arrive(&sm.o_empty[t]);
+                mbar_arrive(&sm.rows_free[rs]);
+                if (t_row >= 0) {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(__uint_as_float(o[cb][8 * v + 0]) * f, __uint_as_float(o[cb][8 * v + 1]) * f);
+                            pk.y = pack_bf16x2(__uint_as_float(o[cb][8 * v + 2]) * f, __uint_as_float(o[cb][8 * v + 3]) * f);
+                            pk.z = pack_bf16x2(__uint_as_float(o[cb][8 * v + 4]) * f, __uint_as_float(o[cb][8 * v + 5]) * f);
+                            pk.w = pack_bf16x2(__uint_as_float(o[cb][8 * v + 6]) * f, __uint_as_float(o[cb][8 * v + 7]) * f);
+                            dst[v] = pk;
+                        }
                     }
                 }
+            } else {
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cb * 32, o);
+                    ld_wait_bind(o);
+                    if (t_row >= 0) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 pk;
+                            pk.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * f, __uint_as_float(o[8 * v + 1]) * f);
+                            pk.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * f, __uint_as_float(o[8 * v + 3]) * f);
+                            pk.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * f, __uint_as_float(o[8 * v + 5]) * f);
+                            pk.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * f, __uint_as_float(o[8 * v + 7]) * f);
+                            dst[v] = pk;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.o_empty[t]);
+                mbar_arrive(&sm.rows_free[rs]);
             }
-            tc_fence_before();
-            mbar_arrive(&sm.o_empty[t]);
-            mbar_arrive(&sm.rows_free[rs]);
         }
     }
 
