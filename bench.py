@@ -49,13 +49,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # source they were taken on (sha256 of the listed files).  See profiles/.
 NCU_TRAFFIC = {
     ("prefill_tc_kernel", "gqe_prefill"): {
-        "sha": "b017cc66fcf82daa", "bytes_per_launch": 1067480000 + 241922304,
+        "sha": "f93b2665924b3811", "bytes_per_launch": 1060030000 + 231494144,
         "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_gqe_prefill.md)"},
     ("prefill_tc_kernel", "gqe_long"): {
-        "sha": "b017cc66fcf82daa", "bytes_per_launch": 171321344 + 47180800,
+        "sha": "f93b2665924b3811", "bytes_per_launch": 169284608 + 37322752,
         "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_gqe_long.md)"},
     ("prefill_tc_kernel", "dense_gqa"): {
-        "sha": "b017cc66fcf82daa", "bytes_per_launch": 105076736 + 29326080,
+        "sha": "f93b2665924b3811", "bytes_per_launch": 104842752 + 30646272,
         "note": "ncu SpeedOfLight + MemoryWorkloadAnalysis, one launch (profiles/prefill_tc_kernel_dense_gqa.md)"},
     ("decode_partial_kernel", "gqe_decode"): {
         "sha": "2ffadcebec633c3d", "bytes_per_launch": 2263625728 + 8142592,
