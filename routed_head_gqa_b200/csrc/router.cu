@@ -164,12 +164,15 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
     // of the batch's T*g*k entries: sums are clamped to that range here and
     // every scatter index is checked below.
     const long long per_batch = (long long)T * g * k;
+    // Sums in 32 bits: each clamped count is at most 32, so a head's total is
+    // at most 32 * nchunk < T + 32.  Lanes stride over the chunks (coalesced).
     for (int j = warp; j < h; j += nwarps) {
-        long long tot = 0, pre = 0;
+        const int32_t* row = cnt + (int64_t)j * nchunk;
+        int tot = 0, pre = 0;
         for (int cc = lane; cc < nchunk; cc += 32) {
-            const long long v = min(max(cnt[(int64_t)j * nchunk + cc], 0), kChunk);
+            const int v = min(max(row[cc], 0), kChunk);
             tot += v;
-            if (cc < c) pre += v;
+            pre += (cc < c) ? v : 0;
         }
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) {
@@ -177,8 +180,8 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
             pre += __shfl_xor_sync(0xffffffffu, pre, d);
         }
         if (lane == 0) {
-            total[j] = (int32_t)min(tot, (long long)per_batch);
-            before[j] = (int32_t)min(pre, (long long)per_batch);
+            total[j] = (int32_t)min((long long)tot, per_batch);
+            before[j] = (int32_t)min((long long)pre, per_batch);
         }
     }
     __syncthreads();
@@ -210,12 +213,24 @@ __global__ void compact_scan_scatter_kernel(const int32_t* __restrict__ idx, int
     const int t = c * kChunk + lane;
     const unsigned below = (1u << lane) - 1u;
     for (int q = warp; q < g; q += nwarps) {
-        int sel[16];
-        for (int s = 0; s < k; ++s) sel[s] = (t < T) ? idx[(((int64_t)b * T + t) * g + q) * k + s] : -1;
+        // the token's selections in group q as a bit mask of heads within the
+        // group (groups of more than 64 heads compare against idx directly)
+        const int32_t* sel = idx + (((int64_t)b * T + (t < T ? t : 0)) * g + q) * k;
+        uint64_t chosen = 0;
+        if (t < T && hpg <= 64) {
+            for (int s = 0; s < k; ++s) {
+                const int a = sel[s] - q * hpg;
+                if (a >= 0 && a < hpg) chosen |= 1ull << a;
+            }
+        }
         for (int jj = 0; jj < hpg; ++jj) {
             const int j = q * hpg + jj;
             bool hit = false;
-            for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
+            if (hpg <= 64) {
+                hit = (chosen >> jj) & 1ull;
+            } else if (t < T) {
+                for (int s = 0; s < k; ++s) hit |= (sel[s] == j);
+            }
             const unsigned ball = __ballot_sync(0xffffffffu, hit);
             if (hit) {
                 const long long e = (long long)total[j] + before[j] + __popc(ball & below);
