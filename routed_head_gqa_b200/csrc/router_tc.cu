@@ -36,9 +36,13 @@ constexpr uint32_t kXBytes = kTM * kTK * 2;  // 16 KB
 constexpr uint32_t kWBlock = kTK * 64 * 2;   // [64 k][64 heads] = 8 KB
 constexpr uint32_t kWhereRouter = 3;
 
-// Pipeline depth: about 192 KB of stages whatever the head count.
+// Pipeline depth.  With up to 64 heads a CTA keeps 4 stages (96 KB), so two
+// CTAs share an SM: all tiles of a launch of up to 2 x 148 tiles stream at
+// once, instead of a second, partial wave of one-CTA-per-SM tiles (gqe_prefill
+// shapes, 256 tiles: route 0.093 -> 0.083 ms).  Wider W_r blocks keep about
+// 192 KB of stages in one CTA.
 template <int NB>
-constexpr int router_stages() { return NB == 1 ? 8 : (NB == 2 ? 6 : 4); }
+constexpr int router_stages() { return NB == 1 ? 4 : (NB == 2 ? 6 : 4); }
 
 template <int NB>  // number of 64-head blocks: N = 64 * NB
 struct RouterSmem {
