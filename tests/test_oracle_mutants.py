@@ -65,6 +65,15 @@ MUTANTS = [
     ("aux_fraction_per_token", "f[j] += 1.0 / ((double)N * k);", "f[j] += 1.0 / (double)N;"),
     ("aux_no_group_size_factor", "L += (double)hpg * s / (double)g;", "L += s / (double)g;"),
     ("aux_grad_drops_mean", "c * p[jj] * (f[q * hpg + jj] - pf);", "c * p[jj] * f[q * hpg + jj];"),
+    ("query_row_from_slot_not_head", "const size_t q_off = ((size_t)bt * h + j) * d_h;",
+     "const size_t q_off = ((size_t)bt * h + q * hpg + s) * d_h;"),
+    ("kv_group_strided", "const size_t kv_base = ((size_t)b * T * g + q) * d_h;",
+     "const size_t kv_base = ((size_t)b * T * g + j % g) * d_h;"),
+    ("values_read_from_keys", "o[d] += w * load_elem(V, vr + d, dtype);", "o[d] += w * load_elem(K, vr + d, dtype);"),
+    ("decode_output_in_slot_order", "O[((size_t)b * h + j) * d_h + d] = gate[sel] * o[d];",
+     "O[((size_t)b * h + q * hpg + s) * d_h + d] = gate[sel] * o[d];"),
+    ("decode_kv_group_strided", "const size_t kv_base = ((size_t)b * Lmax * g + q) * d_h;",
+     "const size_t kv_base = ((size_t)b * Lmax * g + j % g) * d_h;"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
