@@ -6,6 +6,7 @@ process (a broken copy may crash)."""
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -74,6 +75,30 @@ MUTANTS = [
      "O[((size_t)b * h + q * hpg + s) * d_h + d] = gate[sel] * o[d];"),
     ("decode_kv_group_strided", "const size_t kv_base = ((size_t)b * Lmax * g + q) * d_h;",
      "const size_t kv_base = ((size_t)b * Lmax * g + j % g) * d_h;"),
+    ("topk_picks_smallest", "if (lg[prev] < lg[a]) {", "if (lg[prev] > lg[a]) {"),
+    ("margin_from_top_logit", "(double)lg[order[k - 1]] - (double)lg[order[k]]", "(double)lg[order[0]] - (double)lg[order[k]]"),
+    ("compact_first_slot_only", "for (int s = 0; s < k; ++s) hit |= (sel[s] == j);",
+     "for (int s = 0; s < 1; ++s) hit |= (sel[s] == j);"),
+    ("compact_drops_last_position", "for (int t = 0; t < T; ++t) {\n                const int32_t* sel",
+     "for (int t = 0; t < T - 1; ++t) {\n                const int32_t* sel"),
+    ("slots_query_from_slot_not_head", "attend_one(Q, ((size_t)bt * h + j) * d_h, K, V",
+     "attend_one(Q, ((size_t)bt * h + q * hpg + s) * d_h, K, V"),
+    ("weighted_sum_first_gate", "for (int d = 0; d < d_h; ++d) ws[d] += gate[sel] * slot[d];",
+     "for (int d = 0; d < d_h; ++d) ws[d] += gate[sel - s] * slot[d];"),
+    ("oproj_reads_slot_not_head", "load_elem(O, ((size_t)bt * h + jh) * d_h + c, dtype)",
+     "load_elem(O, ((size_t)bt * h + q * (h / g) + s) * d_h + c, dtype)"),
+    ("paged_scale_dropped", "load_elem(K_pages, row + d, dtype);\n                            scores[s] = dot * scale;",
+     "load_elem(K_pages, row + d, dtype);\n                            scores[s] = dot;"),
+    ("paged_gate_dropped", "const double w = gate[sel] * scores[s] / denom;", "const double w = scores[s] / denom;"),
+    ("paged_query_from_slot", "const size_t q_off = ((size_t)b * h + j) * d_h;\n                        /* scores",
+     "const size_t q_off = ((size_t)b * h + q * hpg + r) * d_h;\n                        /* scores"),
+    ("bwd_query_from_slot", "const size_t q_off = (((size_t)b * T + t) * h + j) * d_h;",
+     "const size_t q_off = (((size_t)b * T + t) * h + q * hpg + s_) * d_h;"),
+    ("bwd_dgate_gated", "for (int d = 0; d < d_h; ++d) dg += dO[q_off + d] * o[d];",
+     "for (int d = 0; d < d_h; ++d) dg += gate[sel] * dO[q_off + d] * o[d];"),
+    ("bwd_weights_unnormalised", "for (int s = 0; s <= t; ++s) p[s] /= denom;", "for (int s = 0; s <= t; ++s) p[s] /= 1.0;"),
+    ("router_bwd_dlogits_slot_head", "dlogits[bt * h + idx[base + s]] = gate",
+     "dlogits[bt * h + q * hpg + s] = gate"),
     ("slots_in_reverse_order", "double* slot = cat_rows + (((size_t)r * g + q) * k + s) * d_h;",
      "double* slot = cat_rows + (((size_t)r * g + q) * k + (k - 1 - s)) * d_h;"),
 ]
@@ -83,6 +108,7 @@ import sys
 sys.path.insert(0, {root!r})
 import oracle
 from tests import oracle_pins
+oracle.compile_source({src!r}, {lib!r}, strict=False)
 o = oracle.Oracle({lib!r})
 failed = []
 for c in oracle_pins.ALL_CHECKS:
@@ -94,16 +120,36 @@ print("FAILED:" + ",".join(failed))
 """
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_mutant_is_caught(tmp_path, name, old, new):
+def _check_mutant(tmp_dir, name, old, new):
+    """Plant one mistake (at the anchor's first occurrence) in a copy of the
+    oracle's source, build it and run every pin against it in a child
+    process.  Returns (anchor found, caught, child output)."""
     src = open(oracle.SOURCE).read()
-    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
-    mutated = src.replace(old, new, 1)  # one planted mistake, at the anchor's first occurrence
-    c_path = tmp_path / "mutant.c"
-    c_path.write_text(mutated)
-    lib = str(tmp_path / "libmutant.so")
-    oracle.compile_source(str(c_path), lib, strict=False)
-    proc = subprocess.run([sys.executable, "-c", _CHILD.format(root=ROOT, lib=lib)],
-                          capture_output=True, text=True, timeout=300)
-    caught = proc.returncode != 0 or ("FAILED:" in proc.stdout and proc.stdout.split("FAILED:")[1].strip())
-    assert caught, f"mutant {name} passed every pin:\n{proc.stdout}\n{proc.stderr[-2000:]}"
+    if src.count(old) < 1:
+        return False, False, ""
+    c_path = os.path.join(tmp_dir, name + ".c")
+    with open(c_path, "w") as f:
+        f.write(src.replace(old, new, 1))
+    lib = os.path.join(tmp_dir, "lib" + name + ".so")
+    env = dict(os.environ, OMP_NUM_THREADS="1", OMP_WAIT_POLICY="PASSIVE")
+    proc = subprocess.run([sys.executable, "-c", _CHILD.format(root=ROOT, src=c_path, lib=lib)],
+                          capture_output=True, text=True, timeout=600, env=env)
+    caught = proc.returncode != 0 or ("FAILED:" in proc.stdout and proc.stdout.split("FAILED:")[1].strip() != "")
+    return True, caught, proc.stdout + proc.stderr[-2000:]
+
+
+@pytest.fixture(scope="module")
+def verdicts(tmp_path_factory):
+    """Every mutant checked once, in child processes run side by side (each
+    child spends most of its time importing torch)."""
+    tmp_dir = str(tmp_path_factory.mktemp("mutants"))
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        futs = {m[0]: ex.submit(_check_mutant, tmp_dir, *m) for m in MUTANTS}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_mutant_is_caught(verdicts, name):
+    found, caught, out = verdicts[name]
+    assert found, f"mutation anchor of {name} not found in the oracle's source"
+    assert caught, f"mutant {name} passed every pin:\n{out}"
