@@ -727,6 +727,53 @@ def compact_entry(r):
 
 
 # ---------------------------------------------------------------------------
+def workload_config(w, ws):
+    """The line's "config": the workload and how it is run, the same for both
+    arms (the GPU arm and the CPU oracle arm print identical configs)."""
+    return {"workload": w.name, "shape": w.describe(), "per_gpu_batch": w.B, "global_batch": w.B * ws,
+            "parallelism": f"replicas x{ws} (no exchange step)",
+            "l2": "GPU arm: flushed before every timed step, outside the step events (256 MB written, "
+                  "read back); CPU oracle arm: not applicable"}
+
+
+def gqe_line(metric, w, ws, steps, warmup, res, cpu, configs, extras):
+    """The GPU arm's JSON line from one timed run (res: time_workload's result)."""
+    line = {
+        "metric": metric, "value": res["value"], "unit": res["unit"], "n_gpus": ws, "steps": steps,
+        "warmup": warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded, gqe_synth recipe)",
+        "config": workload_config(w, ws),
+        "step_breakdown_ms": {"route": round(res["route_ms"], 5), "attn": round(res["attn_ms"], 5)},
+        "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"],
+        "gpu_launches": res["gpu_launches"],
+    }
+    if configs:
+        line["configs"] = configs
+    if extras:
+        line["extras"] = {"paged_decode_frac": extras["paged_decode"]["roofline"]["frac"],
+                          "qproj_frac": extras["layer_ops"]["routed_qproj"]["roofline"]["frac"],
+                          "oproj_frac": extras["layer_ops"]["routed_oproj"]["roofline"]["frac"],
+                          "shared_head_frac": extras["layer_ops"]["shared_head"]["roofline"]["frac"],
+                          "group_slots_frac": extras["layer_ops"]["group_slots"]["roofline"]["frac"],
+                          "backward_ms": round(extras["backward"]["ms"], 3),
+                          "backward_frac": extras["backward"]["roofline"]["frac"],
+                          "route_backward_ms": round(extras["backward"]["router"]["ms"], 4)}
+    return line
+
+
+def reference_line(metric, w, ws, steps, warmup, value, unit, secs, desc):
+    """The CPU oracle arm's JSON line."""
+    return {"metric": metric, "impl": "reference", "value": value, "unit": unit, "n_gpus": ws,
+            "steps": steps, "warmup": warmup, "ms_per_step": secs * 1e3 / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, gqe_synth recipe)",
+            "config": workload_config(w, ws),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -757,14 +804,7 @@ def main():
         if rank != 0:
             return
         value, unit, secs, desc = run_reference(w, args.steps, args.warmup)
-        line = {"metric": metric, "impl": "reference", "value": value, "unit": unit, "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic (seeded, gqe_synth recipe)",
-                "config": {"workload": w.name, "shape": w.describe()},
-                "cpu_baseline": {"value": value, "unit": unit, "cores": os.cpu_count(), "kind": "oracle",
-                                 "sample": desc + " per step"},
-                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        line = reference_line(metric, w, args.gpus, args.steps, args.warmup, value, unit, secs, desc)
         print(json.dumps(line))
         return
 
@@ -816,32 +856,10 @@ def main():
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, gqe_synth.make_inputs(w), args.cpu_seconds)
     if rank == 0:
-        line = {
-            "metric": metric, "value": res["value"], "unit": res["unit"], "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-            "data": "synthetic (seeded, gqe_synth recipe)",
-            "config": {"workload": w.name, "shape": w.describe(), "per_gpu_batch": w.B,
-                       "global_batch": w.B * ws, "parallelism": f"replicas x{ws} (no exchange step)",
-                       "l2": "flushed before every timed step, outside the step events (256 MB written, read back)",
-                       "attn_ms": round(res["attn_ms"], 5), "route_ms": round(res["route_ms"], 5)},
-            "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"],
-            "gpu_launches": res["gpu_launches"],
-        }
-        if configs:
-            line["configs"] = configs
-        if extras:
-            if args.extras_out:
-                with open(args.extras_out, "w") as f:
-                    json.dump(extras, f)
-            line["extras"] = {"paged_decode_frac": extras["paged_decode"]["roofline"]["frac"],
-                              "qproj_frac": extras["layer_ops"]["routed_qproj"]["roofline"]["frac"],
-                              "oproj_frac": extras["layer_ops"]["routed_oproj"]["roofline"]["frac"],
-                              "shared_head_frac": extras["layer_ops"]["shared_head"]["roofline"]["frac"],
-                              "group_slots_frac": extras["layer_ops"]["group_slots"]["roofline"]["frac"],
-                              "backward_ms": round(extras["backward"]["ms"], 3),
-                              "backward_frac": extras["backward"]["roofline"]["frac"],
-                              "route_backward_ms": round(extras["backward"]["router"]["ms"], 4)}
+        if extras and args.extras_out:
+            with open(args.extras_out, "w") as f:
+                json.dump(extras, f)
+        line = gqe_line(metric, w, ws, args.steps, args.warmup, res, cpu, configs, extras)
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist
