@@ -91,57 +91,163 @@ def load_peaks():
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clocks and clock-event reasons of the benchmarked GPU during the
+    timed region.  A thread polls NVML (read-only queries) every `poll_ms`,
+    so a region of a few milliseconds still holds samples; nvidia-smi's own
+    query runs beside it.  Every sample carries its host time, and the summary
+    takes the samples between mark_start() and mark_end() (NVML's if it
+    answered, else nvidia-smi's, else the nearest ones)."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    NVML_BITS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+                 "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+                 "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+                 "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, uuid: str | None = None, poll_ms: float = 2.0,
+                 smi_interval_ms: int = 100, smi_cmd: str = "nvidia-smi"):
         self.dev = device_index
+        self.uuid = uuid
+        self.poll_s = poll_ms * 1e-3
+        self.smi_interval_ms = smi_interval_ms
+        self.smi_cmd = smi_cmd
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.smi = []    # (host time, csv line)
+        self.nvml = []   # (host time, sm MHz, max MHz, reasons)
+        self.nvml_thread = None
+        self.stop_flag = threading.Event()
+        self.nvml_ready = threading.Event()
+        self.smi_ready = threading.Event()
+        self.t0 = self.t1 = None
 
-    def start(self):
+    # -- nvidia-smi -----------------------------------------------------------
+    def _read(self):
+        for line in self.proc.stdout:
+            self.smi.append((time.perf_counter(), line.strip()))
+            self.smi_ready.set()
+
+    # -- NVML -------------------------------------------------------------------
+    def _nvml_handle(self, nv):
+        if self.uuid:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(self.uuid)
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _poll(self):
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+        except Exception:
+            self.nvml_ready.set()
+            return
+        try:
+            hdl = self._nvml_handle(nv)
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(hdl, nv.NVML_CLOCK_SM))
+            bits = {n: getattr(nv, attr) for n, attr in self.NVML_BITS.items()}
+            while not self.stop_flag.is_set():
+                mhz = float(nv.nvmlDeviceGetClockInfo(hdl, nv.NVML_CLOCK_SM))
+                mask = int(nv.nvmlDeviceGetCurrentClocksEventReasons(hdl))
+                self.nvml.append((time.perf_counter(), mhz, mx, {n for n, b in bits.items() if mask & b}))
+                self.nvml_ready.set()
+                time.sleep(self.poll_s)
+        except Exception:
+            pass
+        finally:
+            self.nvml_ready.set()
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+
+    def start(self, wait_s: float = 3.0):
+        """Start both samplers and wait (at most wait_s) for their first samples."""
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                [self.smi_cmd, f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.smi_interval_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
+            self.smi_ready.set()
+        self.nvml_thread = threading.Thread(target=self._poll, daemon=True)
+        self.nvml_thread.start()
+        deadline = time.perf_counter() + wait_s
+        self.nvml_ready.wait(max(0.0, deadline - time.perf_counter()))
+        self.smi_ready.wait(max(0.0, deadline - time.perf_counter()))
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def mark_start(self):
+        self.t0 = time.perf_counter()
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        mhz, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def _parse_smi(self):
+        out = []
+        for t, line in self.smi:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                mhz.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
+                mhz, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not mhz:
+            reasons = {n for n, v in zip(self.REASONS, parts[5:9]) if v.lower().startswith("active")}
+            out.append((t, mhz, mx, reasons))
+        return out
+
+    def _window(self, samples):
+        if not samples:
+            return []
+        if self.t0 is None or self.t1 is None:
+            return samples
+        inside = [s for s in samples if self.t0 <= s[0] <= self.t1]
+        if inside:
+            return inside
+        # none inside a region shorter than the period: the first sample after it starts
+        after = [s for s in samples if s[0] >= self.t0]
+        return after[:1] if after else samples[-1:]
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(2 * self.smi_interval_ms * 1e-3)
+        self.stop_flag.set()
+        if self.nvml_thread is not None:
+            self.nvml_thread.join(timeout=2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+        nvml_all, smi_all = list(self.nvml), self._parse_smi()
+        nvml_in, smi_in = self._window(nvml_all), self._window(smi_all)
+        inside = lambda s: self.t0 is not None and self.t1 is not None and self.t0 <= s[0] <= self.t1  # noqa: E731
+        use, source = (nvml_in, "nvml") if any(inside(s) for s in nvml_in) or not smi_in else (smi_in, "nvidia-smi")
+        if not use:
             return None
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        reasons = set()
+        for s in nvml_in + smi_in:
+            reasons |= s[3]
+        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": max(s[2] for s in nvml_all + smi_all),
+                "reasons": sorted(reasons), "samples": sum(1 for s in use if inside(s)), "source": source,
+                "nvidia_smi_samples": sum(1 for s in smi_all if inside(s))}
+
+
+def device_uuid(dev):
+    """NVML's name of the torch device ("GPU-<uuid>"), or None."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+    return u if u.startswith("GPU-") else "GPU-" + u
 
 
 def l2_flush(buf):
@@ -279,12 +385,13 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    sampler = ClockSampler(dev.index) if with_clocks else None
+    sampler = ClockSampler(dev.index, uuid=device_uuid(dev)) if with_clocks else None
     if sampler:
         sampler.start()
-        time.sleep(0.3)
     barrier(ws)
     torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_start()
     for i in range(steps):
         l2_flush(flush)
         e0, e1, e2 = ev[i]
@@ -294,6 +401,8 @@ def time_workload(w, steps, warmup, ws, rank, peaks, peak_kind, with_clocks, wit
         r.attend()
         e2.record()
     torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_end()
     barrier(ws)
     clocks = sampler.stop() if sampler else None
     st = r.buf.status()
